@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""Throughput of the RTPurbo attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-prefill] [--no-cpu-baseline]
+
+One step = one decode token for the whole mixed layer on the 128K-cache,
+batch-8 workload (32 query / 4 kv heads, 1 retrieval kv head, p = 0.95,
+window 4096 + 4 sinks): indexer projection of the new token (q16 + k16 append),
+exact top-p over the 128K k16 cache, gathered sparse attention on the retrieval
+heads, sink+window attention on the local heads.  `value` is decode tokens/s
+(batch / step time) summed over ranks; each rank decodes its own batch (weak
+scaling, no data-path collective).  The prefill of the 128K workload (1 x 131072
+tokens, chained needles) is timed in the same run and reported in `prefill`.
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
+events on the launching stream with a 256 MB L2 flush between steps (outside the
+events); a barrier + synchronize on both sides; the max over ranks.
+
+--impl reference times the fp64 CPU oracle on this host's cores on the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill & decode tokens/s per layer at 128K (1 B200); % of HBM / tensor roofline"
+DECODE_WL = "decode_128k_b8"
+PREFILL_WL = "prefill_128k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sus=d["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ helpers
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    import torch
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def trace_read():
+    from long_context_sparse_rtp_b200 import rtp
+
+    class Entry(ctypes.Structure):
+        _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64),
+                    ("total_ms", ctypes.c_double)]
+    L = rtp.lib()
+    L.rtp_trace_read.restype = ctypes.c_int
+    arr = (Entry * 64)()
+    n = L.rtp_trace_read(arr, 64)
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(max(n, 0))}
+
+
+def trace(on: bool):
+    from long_context_sparse_rtp_b200 import rtp
+    rtp.lib().rtp_trace_reset()
+    rtp.lib().rtp_trace_enable(1 if on else 0)
+
+
+# ------------------------------------------------------------------ decode (ours)
+def decode_state(rank: int):
+    import torch
+    from long_context_sparse_rtp_b200 import rtp_index_scores, synth
+    w = synth.WORKLOADS[DECODE_WL]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = synth.make_inputs(w, "cuda")
+    q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
+    L = k.shape[1]
+    # the k16 cache a prefill would have written (state, not part of a step)
+    _, k16 = rtp_index_scores(q, k, Wq, Wk, role)
+    torch.cuda.synchronize()
+    return dict(w=w, q=q, k=k, v=v, Wq=Wq, Wk=Wk, role=role, k16=k16, L=L)
+
+
+def decode_step(st, o, lse):
+    from long_context_sparse_rtp_b200 import rtp_layer_decode
+    L = st["L"]
+    w = st["w"]
+    return rtp_layer_decode(st["q"], st["k"][:, L - 1:], st["k"], st["v"], st["k16"], st["Wq"],
+                            st["Wk"], st["role"], pos=L - 1, p=w.p, window=w.window,
+                            n_sink=w.n_sink)
+
+
+def time_steps(fn, steps, warmup, world, flush, traced=False):
+    """Per-step CUDA events, L2 flush between steps (outside the events)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+        flush()
+    trace(traced)
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        evs[i][0].record()
+        fn()
+        evs[i][1].record()
+    barrier(world)
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    per_kernel = trace_read() if traced else None
+    trace(False)
+    return ms, per_kernel
+
+
+def decode_bytes(st, sel_count_union):
+    """Algorithmic HBM bytes of one decode step."""
+    w = st["w"]
+    B, L = st["q"].shape[0], st["L"]
+    k16 = B * L * w.H_ret * 16 * 2
+    local = B * (w.Hkv - len(w.ret_kv)) * min(L, w.window + w.n_sink) * 2 * 128 * 2
+    gather = sel_count_union * 2 * 128 * 2
+    small = B * w.H * 128 * 2 * 2 + B * w.Hkv * 128 * 2 * 2 + B * w.Hkv * 128 * 2
+    return dict(k16=k16, local=local, gather=gather, small=small,
+                total=k16 + local + gather + small)
+
+
+def union_size(st, sel):
+    """Sum over (batch, retrieval kv head) of the union of the kept keys, derived
+    on the device from the thresholds (reporting only)."""
+    import torch
+    w = st["w"]
+    q16 = sel["q16"].float()[:, 0]                          # [B, H_ret, 16]
+    k16 = st["k16"][:, :st["L"]].float()                    # [B, L, H_ret, 16]
+    s = torch.einsum("bjhc,bhc->bhj", k16, q16)
+    thr = sel["sel"]["thr"][..., None]
+    jt = sel["sel"]["jtie"][..., None]
+    j = torch.arange(st["L"], device=s.device)[None, None]
+    keep = (s > thr) | ((s == thr) & (j <= jt))
+    tot = 0
+    for r in range(len(w.ret_kv)):
+        tot += int(keep[:, r * w.G:(r + 1) * w.G].any(dim=1).sum())
+    return tot, int(sel["sel"]["count"].sum())
+
+
+def bench_decode(args, world, rank, local, pk):
+    import torch
+    st = decode_state(rank)
+    flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flushbuf.fill_(1.0)
+
+    def step():
+        decode_step(st, None, None)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms, _ = time_steps(step, args.steps, args.warmup, world, flush)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    # traced pass for per-kernel durations (same steps, same flushes)
+    _, kern = time_steps(step, args.steps, 1, world, flush, traced=True)
+    res = decode_step(st, None, None)
+    torch.cuda.synchronize()
+    union, compute_sel = union_size(st, res)
+    B = st["q"].shape[0]
+    nbytes = decode_bytes(st, union)
+    return dict(st=st, ms_step=ms_step, clocks=clk, kern=kern, union=union,
+                compute_sel=compute_sel, bytes=nbytes, B=B, flush=flush)
+
+
+def bench_decode_e2e(dec, args, world):
+    """Through the public API with host buffers: H2D of the new token's q/k/v
+    rows from pinned memory, the layer call, D2H of the output."""
+    import torch
+    from long_context_sparse_rtp_b200 import rtp_layer_decode
+    st = dec["st"]
+    w, L = st["w"], st["L"]
+    hq = st["q"].cpu().pin_memory()
+    hk = st["k"][:, L - 1:].contiguous().cpu().pin_memory()
+    hv = st["v"][:, L - 1:].contiguous().cpu().pin_memory()
+    ho = torch.empty_like(hq).pin_memory()
+    dq = torch.empty_like(st["q"])
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        st["k"][:, L - 1:].copy_(hk, non_blocking=True)
+        st["v"][:, L - 1:].copy_(hv, non_blocking=True)
+        r = rtp_layer_decode(dq, st["k"][:, L - 1:], st["k"], st["v"], st["k16"], st["Wq"],
+                             st["Wk"], st["role"], pos=L - 1, p=w.p, window=w.window,
+                             n_sink=w.n_sink)
+        ho.copy_(r["o"], non_blocking=True)
+
+    ms, _ = time_steps(step, args.steps, args.warmup, world, dec["flush"])
+    ms = max_over_ranks(ms, world)
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    d2h = ho.numel() * 2
+    return ms / args.steps, h2d, d2h
+
+
+# ------------------------------------------------------------------ prefill (ours)
+def bench_prefill(args, world, rank, pk):
+    import torch
+    from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
+    w = synth.WORKLOADS[PREFILL_WL]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = synth.make_inputs(w, "cuda")
+    q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
+    flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flushbuf.fill_(1.0)
+
+    def step():
+        rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
+
+    steps = args.prefill_steps
+    ms, kern = time_steps(step, steps, 1, world, flush, traced=True)
+    ms = max_over_ranks(ms, world)
+    res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
+    torch.cuda.synchronize()
+    cnt = res["sel"]["count"].double()
+    L = q.shape[1]
+    sel_pairs = float(cnt.sum())
+    causal_pairs = w.H_ret * L * (L + 1) / 2
+    loc_heads = w.H - w.H_ret
+    loc_pairs = loc_heads * sum(min(i + 1, w.window + w.n_sink) for i in range(0, L, 1)) \
+        if L <= 1 << 16 else loc_heads * (L * (w.window + w.n_sink) - (w.window + w.n_sink) ** 2 / 2)
+    ms_step = ms / steps
+    per = {k_: dict(launches=n // steps, ms=t / steps) for k_, (n, t) in kern.items()}
+    # dense baseline at the same L (one run, for the ratio)
+    from long_context_sparse_rtp_b200 import rtp_dense_attn
+    o = torch.empty_like(q)
+    dms, dkern = time_steps(lambda: rtp_dense_attn(q, k, v, o=o), 1, 1, world, flush,
+                            traced=True)
+    return dict(ms_step=ms_step, tokens_per_s=L / (ms_step / 1e3) * world, L=L, per_kernel=per,
+                sel_pairs=sel_pairs, causal_pairs=causal_pairs, loc_pairs=loc_pairs,
+                dense_ms=dms, w=w)
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_decode_step_time(st_host, n_steps=1):
+    """The oracle on one full decode step: q16 projection of the new token, the
+    k16 append, top-p + exact attention on every retrieval row, sink+window
+    attention on every local row."""
+    import numpy as np
+    import oracle
+    w = st_host["w"]
+    qb, kb, vb, Wqb, Wkb, k16o = (st_host[x] for x in ("qb", "kb", "vb", "Wqb", "Wkb", "k16o"))
+    B, L = kb.shape[0], kb.shape[1]
+    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
+    scale = 1.0 / math.sqrt(128)
+    t0 = time.perf_counter()
+    for _ in range(n_steps):
+        q16 = np.zeros((B, 1, len(ret), 16), np.uint16)
+        for b in range(B):
+            for s, h in enumerate(ret):
+                q16[b, 0, s] = oracle.project(qb[b, 0, h][None], Wqb[s])[0][0]
+                k16o[b, L - 1, s] = oracle.project(kb[b, L - 1, h // w.G][None], Wkb[s])[0][0]
+        rows = np.array([(b, 0, h) for b in range(B) for h in ret])
+        slots = np.array([s for b in range(B) for s in range(len(ret))])
+        oracle.retrieval_rows(qb, kb, vb, q16, k16o, rows, slots, slots, H=w.H, Hkv=w.Hkv,
+                              q_pos0=L - 1, p=float(np.float32(w.p)), scale=scale)
+        lrows = np.array([(b, 0, h) for b in range(B) for h in loc])
+        oracle.local_rows(qb, kb, vb, lrows, H=w.H, Hkv=w.Hkv, q_pos0=L - 1, window=w.window,
+                          n_sink=w.n_sink, scale=scale)
+    return (time.perf_counter() - t0) / n_steps
+
+
+def oracle_host_state(w, device="cpu"):
+    import numpy as np
+    import oracle
+    from long_context_sparse_rtp_b200 import synth
+    inp = synth.make_inputs(w, device)
+    qb, kb, vb = synth.bits(inp["q"]), synth.bits(inp["k"]), synth.bits(inp["v"])
+    Wqb, Wkb = synth.bits(inp["Wq16"]), synth.bits(inp["Wk16"])
+    ret = w.retrieval_q_heads()
+    B, L = kb.shape[0], kb.shape[1]
+    k16o = np.empty((B, L, len(ret), 16), np.uint16)
+    for b in range(B):
+        for s, h in enumerate(ret):
+            k16o[b, :, s] = oracle.project(kb[b, :, h // w.G], Wkb[s])[0]
+    return dict(w=w, qb=qb, kb=kb, vb=vb, Wqb=Wqb, Wkb=Wkb, k16o=k16o)
+
+
+def cpu_cores():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    from long_context_sparse_rtp_b200 import synth
+    w = synth.WORKLOADS[DECODE_WL]
+    st = oracle_host_state(w, "cuda" if _cuda() else "cpu")
+    for _ in range(args.warmup):
+        oracle_decode_step_time(st, 1)
+    t = oracle_decode_step_time(st, args.steps)
+    B = st["kb"].shape[0]
+    value = B / t
+    sample = f"{args.steps} full decode steps ({B} x {w.H_ret} retrieval rows + " \
+             f"{B} x {w.H - w.H_ret} local rows each) of {DECODE_WL}"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DECODE_WL, "global_batch": B, "seq_len": w.L,
+                       "parallelism": "cpu-oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def _cuda():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    import torch
+    from long_context_sparse_rtp_b200 import build
+    world, rank, local = dist_setup()
+    if rank == 0:
+        build.build()
+    barrier(world)
+    pk = peaks()
+    dec = bench_decode(args, world, rank, local, pk)
+    e2e_ms, h2d, d2h = bench_decode_e2e(dec, args, world)
+    pre = None if args.no_prefill else bench_prefill(args, world, rank, pk)
+
+    B = dec["B"]
+    value = B * world / (dec["ms_step"] / 1e3)
+    kern = dec["kern"]
+    n_launch = sum(n for (n, _) in kern.values()) // args.steps
+    score_ms = kern["dec_score"][1] / kern["dec_score"][0]
+    score_bytes = dec["bytes"]["k16"]
+    achieved = score_bytes / (score_ms / 1e3) / 1e9
+    step_gbs = dec["bytes"]["total"] / (dec["ms_step"] / 1e3) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "dec_score_traffic.json")
+    if os.path.exists(prof):
+        traffic = json.load(open(prof)).get("bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dec["ms_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{DECODE_WL}: decode 1 token/seq, batch 8, 131072-token cache, "
+                               "32 q / 4 kv heads, 1 retrieval kv head, p=0.95, window 4096+4",
+                   "global_batch": B * world, "seq_len": dec["st"]["L"],
+                   "parallelism": f"dp{world}",
+                   "l2": "256 MB L2 flush between timed steps (outside the events)"},
+        "phase": "decode",
+        "roofline": {"bound": "hbm", "kernel": "dec_score", "achieved": achieved,
+                     "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                     "traffic": traffic, "peak_source": pk["src"],
+                     "algorithmic_bytes_per_launch": score_bytes},
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes": dec["bytes"],
+                          "achieved": step_gbs, "frac": step_gbs / pk["hbm"],
+                          "frac_of_8tbs": step_gbs / 8000.0},
+        "per_kernel_ms": {k_: t / n for k_, (n, t) in kern.items()},
+        "selection": {"union_keys": dec["union"], "kept_pairs": dec["compute_sel"]},
+        "gpu_launches": n_launch * args.steps,
+        "clocks": dec["clocks"],
+        "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "api": "rtp_layer_decode (python binding, host buffers)"},
+    }
+    if pre is not None:
+        per = pre["per_kernel"]
+        line["prefill"] = {
+            "workload": f"{PREFILL_WL}: causal prefill 1 x 131072, 32 q / 4 kv, 1 retrieval kv "
+                        "head, p=0.95, window 4096+4, chained needles",
+            "tokens_per_s": pre["tokens_per_s"], "ms_per_step": pre["ms_step"],
+            "steps": args.prefill_steps, "per_kernel_ms": {k_: d["ms"] for k_, d in per.items()},
+            "dense_baseline_ms": pre["dense_ms"], "speedup_vs_dense": pre["dense_ms"] / pre["ms_step"],
+            "kept_pairs": pre["sel_pairs"], "causal_pairs": pre["causal_pairs"],
+        }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        try:
+            stc = oracle_host_state(dec["st"]["w"], "cuda")
+            t = oracle_decode_step_time(stc, 1)
+            line["cpu_baseline"] = {"value": B / t, "unit": "tokens/s", "cores": cpu_cores(),
+                                    "kind": "oracle",
+                                    "sample": f"1 full decode step of {DECODE_WL} "
+                                              f"({B} x 8 retrieval + {B} x 24 local rows)"}
+        except Exception as e:  # report, never hide
+            line["cpu_baseline"] = {"error": repr(e)}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

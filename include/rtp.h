@@ -1,0 +1,226 @@
+/*
+ * rtp.h -- C ABI of librtp.so: the RTPurbo sparse-attention layer on NVIDIA B200
+ * (sm_100a).
+ *
+ * One attention layer with two kinds of heads (paper-graph-ui summary of
+ * "Full Attention Strikes Back: Transferring Full Attention into Sparse within
+ * Hundred Training Steps", arXiv 2605.16928, cited as [FASB §section]):
+ *
+ *  - retrieval heads keep the full KV cache.  A 16-dim indexer scores every
+ *    causal key, s(m, n) = (W^Q q_m) . (W^K k_n)   [FASB §Low-Dimensional
+ *    Projection Mechanism]; the keys are softmax-normalised on those scores and
+ *    the smallest highest-scoring set whose mass reaches p is kept, ties to the
+ *    lower index   [FASB §Dynamic Top-p Selection Mechanism, Eq. 5]; exact
+ *    attention then runs over the kept K/V rows only (same section);
+ *  - local heads attend to n_sink attention-sink tokens plus a sliding window
+ *    [FASB §Local Head Attention Pattern].
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises with the host.  Every call is
+ *    asynchronous on `stream` (0 = legacy default stream).
+ *  - bf16 tensors are passed as void* to bf16 data (IEEE bfloat16 bits).
+ *  - A strided view `rtp_view` describes a [B][L][heads][width] tensor whose
+ *    (heads x width) block per row is contiguous; stride_b / stride_l are in
+ *    ELEMENTS.  The base pointer and both strides must keep every row 16-byte
+ *    aligned (else RTP_ERR_ALIGNMENT).
+ *  - Head dimension D must be 128; indexer width is 16.
+ *  - Query heads h = 0..H-1 map to kv head g = h / (H / Hkv) (GQA).
+ *    kv_role (HOST array of Hkv bytes): 1 = retrieval kv head, 0 = local.  The
+ *    retrieval query heads are the query heads of retrieval kv heads, numbered
+ *    in increasing h as retrieval slots hr = 0..H_ret-1; q16, Wq16 and the
+ *    per-row selection outputs are indexed by hr.
+ *  - k16 layout: k16_per_kv_head = 0 gives one indexer key per retrieval
+ *    QUERY head (H_k16 = H_ret, slot hr uses Wk16[hr]; the summary gives every
+ *    retrieval head its own W^K); k16_per_kv_head = 1 gives one per retrieval
+ *    KV head (H_k16 = number of retrieval kv heads, slot = rank of the kv head
+ *    among retrieval kv heads, shared by its query heads).
+ *  - Query row i of batch b sits at absolute position P = q_pos0 + i and sees
+ *    keys 0..P (causal, the query's own key included); P must be < Lk.
+ *  - Outputs of retrieval calls touch only retrieval heads of `o`, local calls
+ *    only local heads, so one `o` buffer can receive both.
+ *  - Arguments are validated on the host before anything is launched; an error
+ *    return means nothing was enqueued.  Launch failures return RTP_ERR_CUDA.
+ *  - Workspace: `ws` is caller-owned device memory of at least
+ *    rtp_workspace_size(op, ...) bytes, 256-byte aligned.  It must be zeroed
+ *    once before first use (rtp_workspace_init); the kernels leave it ready for
+ *    the next call.  Concurrent calls must not share a workspace.  The first
+ *    bytes of every workspace hold a device status word that kernels set when a
+ *    bounded wait gives up; rtp_get_device_status reads it.
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RTP_API __attribute__((visibility("default")))
+#else
+#define RTP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* rtp_stream_t; /* == cudaStream_t */
+
+typedef enum rtp_status {
+    RTP_OK = 0,
+    RTP_ERR_INVALID_ARG = 1,         /* bad shape, null pointer, p outside [0,1], ... */
+    RTP_ERR_UNSUPPORTED = 2,         /* D != 128, too many heads, device not sm_100 */
+    RTP_ERR_ALIGNMENT = 3,           /* a pointer or stride breaks 16-byte row alignment */
+    RTP_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < rtp_workspace_size(...) */
+    RTP_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
+    RTP_ERR_DEVICE_TIMEOUT = 6       /* a kernel's bounded wait gave up (device status) */
+} rtp_status;
+
+typedef enum rtp_op {
+    RTP_OP_INDEX_SCORES = 0,
+    RTP_OP_TOPP_SELECT = 1,
+    RTP_OP_SPARSE_PREFILL = 2,
+    RTP_OP_SPARSE_DECODE = 3,
+    RTP_OP_LOCAL = 4,
+    RTP_OP_DENSE = 5
+} rtp_op;
+
+typedef struct rtp_shape {
+    int32_t B;      /* batch */
+    int32_t Lq;     /* query rows per batch entry */
+    int32_t Lk;     /* key rows per batch entry (cache length) */
+    int32_t H;      /* query heads */
+    int32_t Hkv;    /* kv heads; H % Hkv == 0 */
+    int32_t D;      /* head dimension, must be 128 */
+    int64_t q_pos0; /* absolute position of query row 0 (prefill 0, decode Lk-1) */
+} rtp_shape;
+
+typedef struct rtp_view {
+    void* ptr;        /* device pointer to element [0][0][0][0] */
+    int64_t stride_b; /* elements between batch entries */
+    int64_t stride_l; /* elements between consecutive rows */
+} rtp_view;
+
+/* Bytes of workspace `op` needs for this shape (always >= 256). */
+RTP_API size_t rtp_workspace_size(rtp_op op, const rtp_shape* shape, const uint8_t* kv_role,
+                          int32_t k16_per_kv_head);
+
+/* Zero a workspace (enqueued on `stream`). */
+RTP_API rtp_status rtp_workspace_init(void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Indexer projection [FASB §Low-Dimensional Projection Mechanism]:
+ *   q16[b][i][hr][c] = bf16_rn( sum_d q[b][i][h(hr)][d] * Wq16[hr][d][c] )
+ *   k16[b][j][s ][c] = bf16_rn( sum_d k[b][j][g(s)][d]  * Wk16[s][d][c] )
+ * with fp32 accumulation and one round-to-nearest-even to bf16.  Shapes: q has
+ * shape->Lq rows of H heads, k has shape->Lk rows of Hkv heads (either count may
+ * be 0 to skip that half).  Wq16 [H_ret][128][16], Wk16 [H_k16][128][16] bf16,
+ * contiguous.  Decode appends the new key by passing views offset to the new row.
+ * No workspace.
+ */
+RTP_API rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv_role,
+                            int32_t k16_per_kv_head, rtp_view q, rtp_view k,
+                            const void* Wq16, const void* Wk16, rtp_view q16,
+                            rtp_view k16, rtp_stream_t stream);
+
+/*
+ * Exact dynamic top-p per retrieval row [FASB §Dynamic Top-p Selection
+ * Mechanism, Eq. 5].  For every (b, hr, i) with P = q_pos0 + i:
+ *   s_j = q16[b][i][hr] . k16[b][j][slot]  for j = 0..P  (fp32),
+ *   w_j = exp(s_j - max s), Z = sum w_j,
+ *   kept set S = shortest prefix of the keys ordered by (s desc, j asc) whose
+ *   mass reaches p*Z (p >= 1: all keys; p == 0: the argmax).
+ * Outputs, [B][H_ret][Lq] contiguous:
+ *   thr[]   the row threshold t (score of the last kept key; -inf when p >= 1),
+ *   jtie[]  key j is kept  <=>  s_j > t  or  (s_j == t and j <= jtie),
+ *   count[] |S|,
+ *   mass[]  (nullable) kept mass / Z.
+ * The scores are recomputed by rtp_sparse_attn_prefill with the identical
+ * arithmetic, so (thr, jtie) reproduce S exactly there.
+ */
+RTP_API rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_role,
+                           int32_t k16_per_kv_head, rtp_view q16, rtp_view k16, float p,
+                           float* thr, int32_t* jtie, int32_t* count, float* mass,
+                           void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Exact attention over each retrieval row's kept set (prefill)
+ * [FASB §Dynamic Top-p Selection Mechanism, sparse attention formula]:
+ *   O[b][i][h] = sum_{j in S} softmax_S(scale * q.k_j) v_j,
+ * S given by (thr, jtie) from rtp_topp_select on the same q16/k16.
+ * o: retrieval heads written (bf16), lse (nullable): [B][H][Lq] fp32, natural
+ * log of the softmax denominator including the scale.
+ */
+RTP_API rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint8_t* kv_role,
+                                   int32_t k16_per_kv_head, rtp_view q, rtp_view k,
+                                   rtp_view v, rtp_view q16, rtp_view k16,
+                                   const float* thr, const int32_t* jtie,
+                                   float softmax_scale, rtp_view o, float* lse,
+                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * One decode step for the retrieval heads (shape->Lq == 1, q_pos0 == Lk - 1):
+ * indexer scores of the new query against the whole k16 cache, exact top-p,
+ * union gather of the kept K/V rows per kv head, exact attention, split-KV
+ * merge.  The k16 cache must already hold the new token's key (rtp_index_scores).
+ * Optional outputs ([B][H_ret], nullable): thr, jtie, count, mass as in
+ * rtp_topp_select.
+ */
+RTP_API rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8_t* kv_role,
+                                  int32_t k16_per_kv_head, rtp_view q, rtp_view k_cache,
+                                  rtp_view v_cache, rtp_view q16, rtp_view k16_cache,
+                                  float p, float softmax_scale, rtp_view o, float* lse,
+                                  float* thr, int32_t* jtie, int32_t* count, float* mass,
+                                  void* ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Local heads: keys j <= P with j < n_sink or j > P - window
+ * [FASB §Local Head Attention Pattern].  Prefill (Lq > 1) and decode (Lq == 1)
+ * both go through this call.  window >= 1, n_sink >= 0.
+ */
+RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role, int32_t window,
+                          int32_t n_sink, rtp_view q, rtp_view k, rtp_view v,
+                          float softmax_scale, rtp_view o, float* lse, void* ws,
+                          size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Baseline: dense causal softmax attention on every head (keys 0..P).
+ */
+RTP_API rtp_status rtp_dense_attn(const rtp_shape* shape, rtp_view q, rtp_view k, rtp_view v,
+                          float softmax_scale, rtp_view o, float* lse, void* ws,
+                          size_t ws_bytes, rtp_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+RTP_API const char* rtp_status_string(rtp_status status);
+
+/* Synchronises `stream`, reads and clears the device status word at the start
+ * of `ws`; RTP_OK if no kernel gave up a bounded wait since the last read. */
+RTP_API rtp_status rtp_get_device_status(void* ws, rtp_stream_t stream);
+
+/*
+ * Kernel trace (no counterpart in the paper; a measurement aid).  While
+ * enabled, every kernel the library launches is bracketed by two CUDA events
+ * recorded on its launch stream.  rtp_trace_read synchronises those events and
+ * returns, per kernel name, the number of launches and their summed device time
+ * (ms).  Not thread-safe against concurrent enable/reset; costs nothing while
+ * disabled.
+ */
+typedef struct rtp_trace_entry {
+    char name[48];
+    int64_t launches;
+    double total_ms;
+} rtp_trace_entry;
+
+RTP_API void rtp_trace_enable(int on);
+RTP_API void rtp_trace_reset(void);
+/* Fills up to max_entries entries; returns the number filled, or -1 on a CUDA error. */
+RTP_API int rtp_trace_read(rtp_trace_entry* out, int max_entries);
+
+/* Library version, e.g. "0.1.0". */
+RTP_API const char* rtp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H_ */

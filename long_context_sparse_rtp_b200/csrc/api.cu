@@ -1,0 +1,119 @@
+// api.cu -- status strings, version, workspace initialisation and the device
+// status word shared by every entry point.
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "rtp_host.h"
+
+using namespace rtp;
+
+extern "C" const char* rtp_status_string(rtp_status status) {
+  switch (status) {
+    case RTP_OK: return "RTP_OK";
+    case RTP_ERR_INVALID_ARG: return "RTP_ERR_INVALID_ARG";
+    case RTP_ERR_UNSUPPORTED: return "RTP_ERR_UNSUPPORTED";
+    case RTP_ERR_ALIGNMENT: return "RTP_ERR_ALIGNMENT";
+    case RTP_ERR_WORKSPACE_TOO_SMALL: return "RTP_ERR_WORKSPACE_TOO_SMALL";
+    case RTP_ERR_CUDA: return "RTP_ERR_CUDA";
+    case RTP_ERR_DEVICE_TIMEOUT: return "RTP_ERR_DEVICE_TIMEOUT";
+  }
+  return "RTP_ERR_UNKNOWN";
+}
+
+extern "C" const char* rtp_version(void) { return "0.1.0"; }
+
+extern "C" rtp_status rtp_workspace_init(void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  if (ws == nullptr || ws_bytes < kStatusBytes) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  if (!aligned16(ws)) return RTP_ERR_ALIGNMENT;
+  return check_cuda(cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+extern "C" rtp_status rtp_get_device_status(void* ws, rtp_stream_t stream) {
+  if (ws == nullptr) return RTP_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DevStatus host;
+  if (cudaMemcpyAsync(&host, ws, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RTP_ERR_CUDA;
+  if (host.code == 0) return RTP_OK;
+  const int32_t zero = 0;
+  if (cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RTP_ERR_CUDA;
+  return (rtp_status)host.code;
+}
+
+// ---------------------------------------------------------------- kernel trace
+namespace rtp {
+namespace {
+struct TraceRec {
+  std::string name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace;       // completed or in-flight launches
+std::vector<cudaEvent_t> g_free;     // recycled events
+thread_local int g_open = -1;        // index of the launch being bracketed
+
+cudaEvent_t take_event() {
+  if (!g_free.empty()) {
+    cudaEvent_t e = g_free.back();
+    g_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void trace_begin(const char* name, cudaStream_t s) {
+  if (!g_trace_on) return;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  TraceRec r{name, take_event(), take_event()};
+  cudaEventRecord(r.start, s);
+  g_trace.push_back(r);
+  g_open = (int)g_trace.size() - 1;
+}
+
+void trace_end(cudaStream_t s) {
+  if (!g_trace_on || g_open < 0) return;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (g_open < (int)g_trace.size()) cudaEventRecord(g_trace[g_open].stop, s);
+  g_open = -1;
+}
+}  // namespace rtp
+
+extern "C" void rtp_trace_enable(int on) { rtp::g_trace_on = on != 0; }
+
+extern "C" void rtp_trace_reset(void) {
+  std::lock_guard<std::mutex> lk(rtp::g_trace_mu);
+  for (auto& r : rtp::g_trace) {
+    rtp::g_free.push_back(r.start);
+    rtp::g_free.push_back(r.stop);
+  }
+  rtp::g_trace.clear();
+}
+
+extern "C" int rtp_trace_read(rtp_trace_entry* out, int max_entries) {
+  std::lock_guard<std::mutex> lk(rtp::g_trace_mu);
+  int n = 0;
+  for (auto& r : rtp::g_trace) {
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return -1;
+    int k = 0;
+    while (k < n && strncmp(out[k].name, r.name.c_str(), sizeof(out[k].name)) != 0) ++k;
+    if (k == n) {
+      if (n >= max_entries) continue;
+      memset(&out[n], 0, sizeof(out[n]));
+      strncpy(out[n].name, r.name.c_str(), sizeof(out[n].name) - 1);
+      ++n;
+    }
+    out[k].launches += 1;
+    out[k].total_ms += ms;
+  }
+  return n;
+}

@@ -1,0 +1,133 @@
+// proj.cu -- 16-dim indexer projection (rtp_index_scores).
+//
+// q16 = W^Q q and k16 = W^K k per retrieval head ("Low-Dimensional Projection
+// Mechanism" of the paper-graph-ui summary of arXiv 2605.16928), fp32
+// accumulation in a fixed order (d = 0..127), one bf16 round-to-nearest-even.
+//
+// HBM-bound: each CTA stages 32 input rows (256 B each) and one 128x16 weight
+// in shared memory; 4 threads per row each produce 4 of the 16 outputs.
+#include "rtp_host.h"
+
+namespace rtp {
+namespace {
+
+constexpr int kProjRows = 32;
+constexpr int kProjThreads = 128;
+
+struct ProjParams {
+  const uint16_t* x;   // [B][L][heads][128]
+  int64_t x_sb, x_sl;
+  const uint16_t* W;   // [slots][128][16]
+  uint16_t* out;       // [B][L][slots][16]
+  int64_t o_sb, o_sl;
+  int L;
+  int16_t head_of_slot[kMaxHeads];
+};
+
+__global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p) {
+  __shared__ float sW[kD][kR];
+  __shared__ float sX[kProjRows][kD + 1];
+  const int slot = blockIdx.y;
+  const int b = blockIdx.z;
+  const int row0 = blockIdx.x * kProjRows;
+  const int tid = threadIdx.x;
+
+  const uint16_t* W = p.W + (size_t)slot * kD * kR;
+  for (int e = tid; e < kD * kR; e += kProjThreads)
+    sW[e / kR][e % kR] = __uint_as_float((uint32_t)W[e] << 16);
+
+  const int head = p.head_of_slot[slot];
+  // 32 rows x 16 chunks of 16 bytes
+  for (int c = tid; c < kProjRows * 16; c += kProjThreads) {
+    const int r = c / 16, ch = c % 16;
+    const int row = row0 + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < p.L) {
+      const uint16_t* src = p.x + b * p.x_sb + (int64_t)row * p.x_sl + head * kD + ch * 8;
+      v = *reinterpret_cast<const uint4*>(src);
+    }
+    float* dst = &sX[r][ch * 8];
+    dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x);
+    dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
+    dst[4] = bf16_lo(v.z); dst[5] = bf16_hi(v.z);
+    dst[6] = bf16_lo(v.w); dst[7] = bf16_hi(v.w);
+  }
+  __syncthreads();
+
+  const int r = tid / 4;
+  const int c0 = (tid % 4) * 4;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll 8
+  for (int d = 0; d < kD; ++d) {
+    const float xv = sX[r][d];
+    const float4 w = *reinterpret_cast<const float4*>(&sW[d][c0]);
+    acc0 = fmaf(xv, w.x, acc0);
+    acc1 = fmaf(xv, w.y, acc1);
+    acc2 = fmaf(xv, w.z, acc2);
+    acc3 = fmaf(xv, w.w, acc3);
+  }
+  const int row = row0 + r;
+  if (row < p.L) {
+    uint2 o;
+    o.x = pack_bf16x2(acc0, acc1);
+    o.y = pack_bf16x2(acc2, acc3);
+    uint16_t* dst = p.out + b * p.o_sb + (int64_t)row * p.o_sl + slot * kR + c0;
+    *reinterpret_cast<uint2*>(dst) = o;
+  }
+}
+
+rtp_status launch_proj(const rtp_view& x, int L, int B, const void* W, int n_slots,
+                       const int16_t* head_of_slot, const rtp_view& out,
+                       cudaStream_t stream) {
+  if (L == 0 || B == 0 || n_slots == 0) return RTP_OK;
+  ProjParams p;
+  p.x = static_cast<const uint16_t*>(x.ptr);
+  p.x_sb = x.stride_b;
+  p.x_sl = x.stride_l;
+  p.W = static_cast<const uint16_t*>(W);
+  p.out = static_cast<uint16_t*>(out.ptr);
+  p.o_sb = out.stride_b;
+  p.o_sl = out.stride_l;
+  p.L = L;
+  for (int s = 0; s < n_slots; ++s) p.head_of_slot[s] = head_of_slot[s];
+  dim3 grid((L + kProjRows - 1) / kProjRows, n_slots, B);
+  if (grid.z > 65535 || grid.y > 65535) return RTP_ERR_UNSUPPORTED;
+  TraceScope tr("proj16", stream);
+  proj16_kernel<<<grid, kProjThreads, 0, stream>>>(p);
+  return check_cuda(cudaGetLastError());
+}
+
+}  // namespace
+}  // namespace rtp
+
+using namespace rtp;
+
+extern "C" rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv_role,
+                                       int32_t k16_per_kv_head, rtp_view q, rtp_view k,
+                                       const void* Wq16, const void* Wk16, rtp_view q16,
+                                       rtp_view k16, rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, k16_per_kv_head, &hm)) != RTP_OK) return st;
+  const bool do_q = shape->Lq > 0 && shape->B > 0 && hm.n_ret > 0;
+  const bool do_k = shape->Lk > 0 && shape->B > 0 && hm.n_ret > 0;
+  if ((st = check_view(q, shape->H, kD, do_q)) != RTP_OK) return st;
+  if ((st = check_view(q16, hm.n_ret, kR, do_q)) != RTP_OK) return st;
+  if ((st = check_view(k, shape->Hkv, kD, do_k)) != RTP_OK) return st;
+  if ((st = check_view(k16, hm.H_k16, kR, do_k)) != RTP_OK) return st;
+  if (do_q && Wq16 == nullptr) return RTP_ERR_INVALID_ARG;
+  if (do_k && Wk16 == nullptr) return RTP_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (do_q) {
+    st = launch_proj(q, shape->Lq, shape->B, Wq16, hm.n_ret, hm.ret_q, q16, s);
+    if (st != RTP_OK) return st;
+  }
+  if (do_k) {
+    int16_t kv_of_slot[kMaxHeads];
+    for (int sl = 0; sl < hm.H_k16; ++sl)
+      kv_of_slot[sl] = k16_per_kv_head ? hm.rkv[sl] : (int16_t)(hm.ret_q[sl] / hm.G);
+    st = launch_proj(k, shape->Lk, shape->B, Wk16, hm.H_k16, kv_of_slot, k16, s);
+  }
+  return st;
+}

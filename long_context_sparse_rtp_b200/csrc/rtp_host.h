@@ -1,0 +1,160 @@
+// rtp_host.h -- host-side helpers shared by the entry points: argument checks,
+// head maps and workspace layouts.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "rtp.h"
+#include "rtp_common.cuh"
+
+namespace rtp {
+
+constexpr int kDecChunk = 1024;    // tokens per decode scoring / compaction chunk
+constexpr int kDecHistChunk = 4096;// scores per decode histogram CTA
+constexpr int kDecBins = 256;      // level-0 histogram bins (decode)
+constexpr int kDecCap = 4096;      // candidates a decode row resolves in one sort
+constexpr int kDecChunksPerSplit = 2;
+constexpr int kMaxKeys = 1 << 21;  // composite (score, index) keys use 21 index bits
+
+// Kernel trace: events around each launch while rtp_trace_enable(1) is in force.
+void trace_begin(const char* name, cudaStream_t s);
+void trace_end(cudaStream_t s);
+struct TraceScope {
+  cudaStream_t s;
+  TraceScope(const char* name, cudaStream_t st) : s(st) { trace_begin(name, st); }
+  ~TraceScope() { trace_end(s); }
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline rtp_status check_cuda(cudaError_t e) {
+  return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// A [B][L][heads][width] bf16 view: non-null, rows 16-byte aligned.
+inline rtp_status check_view(const rtp_view& v, int heads, int width, bool needed) {
+  if (!needed) return RTP_OK;
+  if (v.ptr == nullptr) return RTP_ERR_INVALID_ARG;
+  if (v.stride_l < (int64_t)heads * width || v.stride_b < 0) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(v.ptr) || (v.stride_l * 2) % 16 != 0 || (v.stride_b * 2) % 16 != 0)
+    return RTP_ERR_ALIGNMENT;
+  return RTP_OK;
+}
+
+inline rtp_status check_shape(const rtp_shape* s) {
+  if (s == nullptr) return RTP_ERR_INVALID_ARG;
+  if (s->D != kD) return RTP_ERR_UNSUPPORTED;
+  if (s->B < 0 || s->Lq < 0 || s->Lk < 0 || s->H <= 0 || s->Hkv <= 0) return RTP_ERR_INVALID_ARG;
+  if (s->H % s->Hkv != 0) return RTP_ERR_INVALID_ARG;
+  if (s->H > kMaxHeads) return RTP_ERR_UNSUPPORTED;
+  if (s->q_pos0 < 0) return RTP_ERR_INVALID_ARG;
+  return RTP_OK;
+}
+
+// Causal consistency: every query row's position must have a key row.
+inline rtp_status check_causal(const rtp_shape* s) {
+  if (s->Lq > 0 && s->q_pos0 + s->Lq - 1 >= (int64_t)s->Lk) return RTP_ERR_INVALID_ARG;
+  return RTP_OK;
+}
+
+inline rtp_status make_headmap(const rtp_shape* s, const uint8_t* kv_role, int k16_per_kv,
+                               HeadMap* hm) {
+  if (kv_role == nullptr) return RTP_ERR_INVALID_ARG;
+  if (k16_per_kv != 0 && k16_per_kv != 1) return RTP_ERR_INVALID_ARG;
+  memset(hm, 0, sizeof(*hm));
+  hm->H = s->H;
+  hm->Hkv = s->Hkv;
+  hm->G = s->H / s->Hkv;
+  if (hm->G > 16) return RTP_ERR_UNSUPPORTED;  // decode packs one kv group into 16 mma rows
+  for (int g = 0; g < s->Hkv; ++g) {
+    if (kv_role[g] > 1) return RTP_ERR_INVALID_ARG;
+    if (kv_role[g]) {
+      const int rk = hm->n_rkv++;
+      hm->rkv[rk] = (int16_t)g;
+      for (int j = 0; j < hm->G; ++j) {
+        const int hr = hm->n_ret++;
+        hm->ret_q[hr] = (int16_t)(g * hm->G + j);
+        hm->ret_k16[hr] = (int16_t)(k16_per_kv ? rk : hr);
+      }
+    } else {
+      hm->lkv[hm->n_lkv++] = (int16_t)g;
+      hm->n_loc += hm->G;
+    }
+  }
+  hm->H_k16 = k16_per_kv ? hm->n_rkv : hm->n_ret;
+  return RTP_OK;
+}
+
+// ---------------------------------------------------------------- workspaces
+// Every workspace starts with the 256-byte DevStatus block.
+
+struct DecodeWs {   // retrieval decode
+  size_t scores, cmax, hist_m, hist_c, zsum, counter, rowres, cand, list, lcount, part,
+      mcount, total;
+  int n_chunks, n_splits, Lk_pad, rows;
+};
+
+// Per-row decode result kept in the workspace.
+struct RowRes {
+  float t;
+  int32_t jtie;
+  int32_t count;
+  float mass;
+};
+
+inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
+  DecodeWs w;
+  const int64_t N = s->Lk;
+  w.n_chunks = (int)((N + kDecChunk - 1) / kDecChunk);
+  w.Lk_pad = w.n_chunks * kDecChunk;
+  w.n_splits = (w.n_chunks + kDecChunksPerSplit - 1) / kDecChunksPerSplit;
+  w.rows = s->B * hm.n_ret;
+  const size_t groups = (size_t)s->B * hm.n_rkv;
+  size_t off = kStatusBytes;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  w.scores = take((size_t)w.rows * w.Lk_pad * 4);
+  w.cmax = take((size_t)w.rows * w.n_chunks * 4);
+  w.hist_m = take((size_t)w.rows * kDecBins * 8);
+  w.hist_c = take((size_t)w.rows * kDecBins * 4);
+  w.zsum = take((size_t)w.rows * 8);
+  w.counter = take((size_t)w.rows * 4 + groups * 4);
+  w.rowres = take((size_t)w.rows * sizeof(RowRes));
+  w.cand = 0;
+  w.list = take(groups * w.Lk_pad * 8);
+  w.lcount = take(groups * w.n_chunks * 4);
+  w.part = take(groups * w.n_splits * 16 * (2 + kD) * 4);
+  w.mcount = take(groups * 4);
+  w.total = off;
+  return w;
+}
+
+struct AttnDecodeWs {  // local / dense decode (range mode)
+  size_t part, mcount, total;
+  int n_splits;
+};
+
+constexpr int kRangeKeysPerSplit = 512;
+
+inline AttnDecodeWs range_decode_ws_layout(int64_t n_keys, int groups) {
+  AttnDecodeWs w;
+  w.n_splits = (int)((n_keys + kRangeKeysPerSplit - 1) / kRangeKeysPerSplit);
+  if (w.n_splits < 1) w.n_splits = 1;
+  size_t off = kStatusBytes;
+  w.part = off;
+  off = align_up(off + (size_t)groups * w.n_splits * 16 * (2 + kD) * 4, 256);
+  w.mcount = off;
+  off = align_up(off + (size_t)groups * 4, 256);
+  w.total = off;
+  return w;
+}
+
+}  // namespace rtp

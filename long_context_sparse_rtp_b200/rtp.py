@@ -1,0 +1,292 @@
+"""Thin Python binding of librtp.so (ctypes).
+
+Argument marshalling only: every step of the layer runs in the CUDA library.
+torch provides device memory and the current stream.  The functions carry the
+C entry points' names; see include/rtp.h for the exact contracts.
+
+If the shared library is missing or cannot be loaded this module raises on
+first use -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librtp.so")
+
+RTP_OK = 0
+STATUS = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_UNSUPPORTED",
+          3: "RTP_ERR_ALIGNMENT", 4: "RTP_ERR_WORKSPACE_TOO_SMALL", 5: "RTP_ERR_CUDA",
+          6: "RTP_ERR_DEVICE_TIMEOUT"}
+OP_INDEX_SCORES, OP_TOPP_SELECT, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_LOCAL, OP_DENSE = range(6)
+
+
+class RtpError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Lq", ctypes.c_int32), ("Lk", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("q_pos0", ctypes.c_int64)]
+
+
+class View(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_l", ctypes.c_int64)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """Load librtp.so (raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(
+                        f"{LIB_PATH} is not built; run `python -m long_context_sparse_rtp_b200.build`")
+                L = ctypes.CDLL(LIB_PATH)
+                V, S, P = View, ctypes.POINTER(Shape), ctypes.c_void_p
+                i32, f32, sz = ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+                L.rtp_workspace_size.restype = sz
+                L.rtp_workspace_size.argtypes = [ctypes.c_int, S, P, i32]
+                L.rtp_workspace_init.argtypes = [P, sz, P]
+                L.rtp_index_scores.argtypes = [S, P, i32, V, V, P, P, V, V, P]
+                L.rtp_topp_select.argtypes = [S, P, i32, V, V, f32, P, P, P, P, P, sz, P]
+                L.rtp_sparse_attn_prefill.argtypes = [S, P, i32, V, V, V, V, V, P, P, f32, V, P,
+                                                      P, sz, P]
+                L.rtp_sparse_attn_decode.argtypes = [S, P, i32, V, V, V, V, V, f32, f32, V, P,
+                                                     P, P, P, P, P, sz, P]
+                L.rtp_local_attn.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P, sz, P]
+                L.rtp_dense_attn.argtypes = [S, V, V, V, f32, V, P, P, sz, P]
+                L.rtp_status_string.restype = ctypes.c_char_p
+                L.rtp_status_string.argtypes = [ctypes.c_int]
+                L.rtp_get_device_status.argtypes = [P, P]
+                L.rtp_version.restype = ctypes.c_char_p
+                for fn in ("rtp_workspace_init", "rtp_index_scores", "rtp_topp_select",
+                           "rtp_sparse_attn_prefill", "rtp_sparse_attn_decode",
+                           "rtp_local_attn", "rtp_dense_attn", "rtp_get_device_status"):
+                    getattr(L, fn).restype = ctypes.c_int
+                _lib = L
+    return _lib
+
+
+def _check(fn: str, code: int):
+    if code != RTP_OK:
+        raise RtpError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def view(t: torch.Tensor | None, width: int = 128) -> View:
+    """[B][L][heads][width] tensor -> rtp_view (heads x width contiguous per row)."""
+    if t is None:
+        return View(None, 0, 0)
+    if t.dim() != 4 or t.stride(3) != 1 or t.stride(2) != width:
+        raise ValueError("expected a [B, L, heads, width] tensor with contiguous heads*width")
+    return View(ctypes.c_void_p(t.data_ptr()), t.stride(0), t.stride(1))
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _role(kv_role):
+    arr = (ctypes.c_uint8 * len(kv_role))(*[int(x) for x in kv_role])
+    return arr
+
+
+def _shape(B, Lq, Lk, H, Hkv, q_pos0):
+    return Shape(B, Lq, Lk, H, Hkv, 128, q_pos0)
+
+
+# --------------------------------------------------------------------- workspaces
+_ws_cache: dict = {}
+
+
+def workspace(op: int, shape: Shape, role, k16_per_kv: int, device, stream=None) -> torch.Tensor:
+    """A zero-initialised workspace of the size the library asks for, cached per
+    (device, stream, op); the kernels leave it clean for the next call."""
+    need = lib().rtp_workspace_size(op, ctypes.byref(shape), role, k16_per_kv)
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    key = (str(device), s.cuda_stream, op)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def rtp_workspace_size(op: int, shape: Shape, kv_role, k16_per_kv_head: int = 0) -> int:
+    return lib().rtp_workspace_size(op, ctypes.byref(shape), _role(kv_role), k16_per_kv_head)
+
+
+def rtp_status_string(code: int) -> str:
+    return lib().rtp_status_string(code).decode()
+
+
+def rtp_version() -> str:
+    return lib().rtp_version().decode()
+
+
+def rtp_get_device_status(ws: torch.Tensor, stream=None) -> int:
+    return lib().rtp_get_device_status(_ptr(ws), _stream(stream))
+
+
+# --------------------------------------------------------------------- entry points
+def _n_ret(kv_role, G):
+    return int(sum(int(x) for x in kv_role)) * G
+
+
+def rtp_index_scores(q, k, Wq16, Wk16, kv_role, *, q16=None, k16=None, k16_per_kv_head=0,
+                     stream=None):
+    """16-dim indexer projections.  q [B,Lq,H,128] (or None), k [B,Lk,Hkv,128] (or None).
+    Returns (q16 [B,Lq,H_ret,16], k16 [B,Lk,H_k16,16]); pass q16/k16 to write in place."""
+    ref = q if q is not None else k
+    B = ref.shape[0]
+    H = q.shape[2] if q is not None else None
+    Hkv = len(kv_role)
+    if H is None:
+        raise ValueError("q is needed for the head count")
+    G = H // Hkv
+    n_ret = _n_ret(kv_role, G)
+    H_k16 = int(sum(int(x) for x in kv_role)) if k16_per_kv_head else n_ret
+    Lq = q.shape[1] if q is not None else 0
+    Lk = k.shape[1] if k is not None else 0
+    dev = ref.device
+    if q is not None and q16 is None:
+        q16 = torch.empty(B, Lq, n_ret, 16, dtype=torch.bfloat16, device=dev)
+    if k is not None and k16 is None:
+        k16 = torch.empty(B, Lk, H_k16, 16, dtype=torch.bfloat16, device=dev)
+    shp = _shape(B, Lq, Lk, H, Hkv, 0)
+    _check("rtp_index_scores", lib().rtp_index_scores(
+        ctypes.byref(shp), _role(kv_role), k16_per_kv_head, view(q), view(k),
+        _ptr(Wq16), _ptr(Wk16), view(q16, 16), view(k16, 16), _stream(stream)))
+    return q16, k16
+
+
+def rtp_topp_select(q16, k16, kv_role, p, *, H, q_pos0=0, k16_per_kv_head=0, want_mass=True,
+                    stream=None):
+    """Exact top-p per retrieval row.  Returns dict(thr, jtie, count, mass) of [B,H_ret,Lq]."""
+    B, Lq, n_ret = q16.shape[0], q16.shape[1], q16.shape[2]
+    Lk = k16.shape[1]
+    Hkv = len(kv_role)
+    dev = q16.device
+    thr = torch.empty(B, n_ret, Lq, dtype=torch.float32, device=dev)
+    jtie = torch.empty(B, n_ret, Lq, dtype=torch.int32, device=dev)
+    count = torch.empty(B, n_ret, Lq, dtype=torch.int32, device=dev)
+    mass = torch.empty(B, n_ret, Lq, dtype=torch.float32, device=dev) if want_mass else None
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role(kv_role)
+    ws = workspace(OP_TOPP_SELECT, shp, role, k16_per_kv_head, dev, stream)
+    _check("rtp_topp_select", lib().rtp_topp_select(
+        ctypes.byref(shp), role, k16_per_kv_head, view(q16, 16), view(k16, 16),
+        ctypes.c_float(p), _ptr(thr), _ptr(jtie), _ptr(count), _ptr(mass), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return dict(thr=thr, jtie=jtie, count=count, mass=mass)
+
+
+def rtp_sparse_attn_prefill(q, k, v, q16, k16, thr, jtie, kv_role, *, scale=None, q_pos0=0,
+                            k16_per_kv_head=0, o=None, lse=None, stream=None):
+    """Exact attention over the kept sets (retrieval heads).  Returns (o, lse)."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, Lq), float("nan"), dtype=torch.float32, device=dev)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role(kv_role)
+    ws = workspace(OP_SPARSE_PREFILL, shp, role, k16_per_kv_head, dev, stream)
+    _check("rtp_sparse_attn_prefill", lib().rtp_sparse_attn_prefill(
+        ctypes.byref(shp), role, k16_per_kv_head, view(q), view(k), view(v), view(q16, 16),
+        view(k16, 16), _ptr(thr), _ptr(jtie), ctypes.c_float(scale), view(o), _ptr(lse),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def rtp_sparse_attn_decode(q, k_cache, v_cache, q16, k16_cache, kv_role, p, *, scale=None,
+                           q_pos0=None, k16_per_kv_head=0, o=None, lse=None, want_sel=True,
+                           stream=None):
+    """One decode step for the retrieval heads.  q [B,1,H,128].
+    Returns (o, lse, dict(thr, jtie, count, mass) of [B,H_ret])."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    n_ret = q16.shape[2]
+    q_pos0 = Lk - 1 if q_pos0 is None else q_pos0
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, 1), float("nan"), dtype=torch.float32, device=dev)
+    sel = None
+    if want_sel:
+        sel = dict(thr=torch.empty(B, n_ret, dtype=torch.float32, device=dev),
+                   jtie=torch.empty(B, n_ret, dtype=torch.int32, device=dev),
+                   count=torch.empty(B, n_ret, dtype=torch.int32, device=dev),
+                   mass=torch.empty(B, n_ret, dtype=torch.float32, device=dev))
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role(kv_role)
+    ws = workspace(OP_SPARSE_DECODE, shp, role, k16_per_kv_head, dev, stream)
+    g = (lambda key: _ptr(sel[key])) if sel else (lambda key: None)
+    _check("rtp_sparse_attn_decode", lib().rtp_sparse_attn_decode(
+        ctypes.byref(shp), role, k16_per_kv_head, view(q), view(k_cache), view(v_cache),
+        view(q16, 16), view(k16_cache, 16), ctypes.c_float(p), ctypes.c_float(scale), view(o),
+        _ptr(lse), g("thr"), g("jtie"), g("count"), g("mass"), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return o, lse, sel
+
+
+def rtp_local_attn(q, k, v, kv_role, *, window, n_sink, scale=None, q_pos0=0, o=None,
+                   lse=None, stream=None):
+    """Sink + sliding-window attention on the local heads (prefill or Lq == 1 decode)."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, Lq), float("nan"), dtype=torch.float32, device=dev)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role(kv_role)
+    ws = workspace(OP_LOCAL, shp, role, 0, dev, stream)
+    _check("rtp_local_attn", lib().rtp_local_attn(
+        ctypes.byref(shp), role, window, n_sink, view(q), view(k), view(v),
+        ctypes.c_float(scale), view(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def rtp_dense_attn(q, k, v, *, scale=None, q_pos0=0, o=None, lse=None, stream=None):
+    """Dense causal attention baseline on every head."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Lq), dtype=torch.float32, device=dev)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role([0] * Hkv)
+    ws = workspace(OP_DENSE, shp, role, 0, dev, stream)
+    _check("rtp_dense_attn", lib().rtp_dense_attn(
+        ctypes.byref(shp), view(q), view(k), view(v), ctypes.c_float(scale), view(o),
+        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse

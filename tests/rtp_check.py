@@ -1,0 +1,108 @@
+"""Shared checks for the GPU-vs-oracle parity tests.
+
+Tolerances ("Parity contract"):
+
+* selection: the kept set of every retrieval row equals the oracle's, except for
+  keys whose indexer score lies within SEL_BAND (relative, floor 1) of the row
+  threshold -- the oracle's or the GPU's own.  In addition the GPU threshold must
+  be a valid top-p cut under the oracle's fp64 masses: the mass strictly above it
+  stays below p and the mass at or above it reaches p, both up to MASS_EPS (the
+  GPU computes exp and the scores in fp32);
+* outputs: max-abs <= 2e-2 and mean-abs <= 2e-3 against the oracle's fp64
+  output (bf16 inputs, fp32 accumulation on the GPU); lse within 2e-2.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+from long_context_sparse_rtp_b200 import synth
+
+SEL_BAND = 1e-5
+MASS_EPS = 1e-5
+SCORE_SLACK = 2e-6
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+LSE_ABS = 2e-2
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return synth.bits(t)
+
+
+def f64(b: np.ndarray) -> np.ndarray:
+    return oracle.bf16_bits_to_f64(b)
+
+
+def check_row_selection(s64, p, t_orc, sel_orc, t_gpu, jtie_gpu, count_gpu, mass_gpu=None):
+    """One retrieval row.  s64: fp64 indexer scores of keys 0..P computed from the
+    GPU's q16/k16.  Returns the number of keys inside the tolerance band."""
+    n = s64.size
+    j = np.arange(n)
+    if p >= 1.0:
+        assert t_gpu == -math.inf and count_gpu == n and jtie_gpu == n - 1
+        return 0
+    sel_gpu = (s64 > t_gpu) | ((s64 == t_gpu) & (j <= jtie_gpu))
+    band = np.abs(s64 - t_orc) <= SEL_BAND * max(abs(t_orc), 1.0)
+    band |= np.abs(s64 - t_gpu) <= SEL_BAND * max(abs(t_gpu), 1.0)
+    out = ~band
+    bad = np.nonzero(sel_gpu[out] != sel_orc[out])[0]
+    assert bad.size == 0, (
+        f"selection differs outside the band at keys {j[out][bad][:8]} "
+        f"(t_orc={t_orc!r}, t_gpu={t_gpu!r}, count gpu={count_gpu} orc={int(sel_orc.sum())})")
+    n_out = int(sel_gpu[out].sum())
+    assert n_out <= count_gpu <= n_out + int(band.sum()), (count_gpu, n_out, int(band.sum()))
+    # the GPU cut is a valid top-p cut under fp64 masses
+    w = np.exp(s64 - s64.max())
+    Z = w.sum()
+    slack = SCORE_SLACK * max(abs(t_gpu), 1.0)
+    above = w[s64 > t_gpu + slack].sum() / Z
+    at_or_above = w[s64 >= t_gpu - slack].sum() / Z
+    assert above < p + MASS_EPS, (above, p)
+    assert at_or_above >= p - MASS_EPS, (at_or_above, p)
+    if mass_gpu is not None:
+        m_lo = w[sel_gpu & out].sum() / Z
+        m_hi = m_lo + w[band].sum() / Z
+        assert m_lo - MASS_EPS <= mass_gpu <= m_hi + MASS_EPS, (mass_gpu, m_lo, m_hi)
+    return int(band.sum())
+
+
+def check_outputs(o_gpu: np.ndarray, o_orc: np.ndarray, what: str):
+    err = np.abs(o_gpu.astype(np.float64) - o_orc)
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= O_MAX_ABS, f"{what}: max-abs {mx:.3e}"
+    assert mean <= O_MEAN_ABS, f"{what}: mean-abs {mean:.3e}"
+    return mx, mean
+
+
+def oracle_k16(k_bits, Wk_bits, w: synth.Workload, per_kv: bool = False):
+    """Oracle projection of every key row for every k16 slot: [B, Lk, H_k16, 16]."""
+    B, Lk = k_bits.shape[0], k_bits.shape[1]
+    ret = w.retrieval_q_heads()
+    if per_kv:
+        kvs = sorted(w.ret_kv)
+    else:
+        kvs = [h // w.G for h in ret]
+    out = np.empty((B, Lk, len(kvs), 16), np.uint16)
+    for b in range(B):
+        for s, g in enumerate(kvs):
+            out[b, :, s] = oracle.project(k_bits[b, :, g], Wk_bits[s])[0]
+    return out
+
+
+def oracle_q16(q_bits, Wq_bits, w: synth.Workload):
+    B, Lq = q_bits.shape[0], q_bits.shape[1]
+    ret = w.retrieval_q_heads()
+    out = np.empty((B, Lq, len(ret), 16), np.uint16)
+    for b in range(B):
+        for s, h in enumerate(ret):
+            out[b, :, s] = oracle.project(q_bits[b, :, h], Wq_bits[s])[0]
+    return out
+
+
+def row_scores(q16_bits_row, k16_bits, P):
+    """fp64 indexer scores of keys 0..P: k16_bits [Lk, 16] (one slot)."""
+    return f64(k16_bits[:P + 1]) @ f64(q16_bits_row)

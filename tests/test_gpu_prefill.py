@@ -1,0 +1,175 @@
+"""GPU parity: causal prefill of one mixed layer against the fp64 oracle.
+
+Stage by stage ("Parity contract"):
+ (i)   q16/k16 projections equal the oracle's bf16 values, or sit one bf16 ulp
+       away where the exact value lies within fp32-accumulation distance of a
+       rounding midpoint;
+ (ii)  the top-p selection, re-derived by the oracle from the GPU's own q16/k16,
+       matches outside the threshold band and the GPU cut is a valid top-p cut;
+ (iii) outputs match the oracle run end to end (its own projections).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
+from rtp_check import (LSE_ABS, bits, check_outputs, check_row_selection, f64, oracle_k16,
+                       oracle_q16, row_scores)
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from long_context_sparse_rtp_b200 import build
+    build.build()
+
+
+def check_projection(gpu_bits, x_bits_rows, W_bits):
+    """(i) for one slot: gpu_bits [n,16], x_bits_rows [n,128], W [128,16]."""
+    ref, pre = oracle.project(x_bits_rows, W_bits)
+    diff = np.nonzero(gpu_bits != ref)
+    if diff[0].size == 0:
+        return 0
+    a, b = f64(gpu_bits[diff]), f64(ref[diff])
+    mid = 0.5 * (a + b)
+    bound = 128 * 2.0 ** -24 * (np.abs(f64(x_bits_rows)) @ np.abs(f64(W_bits)))[diff]
+    # adjacent bf16 values only, and the exact value near their midpoint
+    assert np.all(np.abs(gpu_bits[diff].astype(np.int64) - ref[diff].astype(np.int64)) == 1)
+    assert np.all(np.abs(pre[diff] - mid) <= bound + 1e-30)
+    assert diff[0].size <= max(4, gpu_bits.size // 200)
+    return diff[0].size
+
+
+def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, seed=None):
+    if seed is not None:
+        w = w.with_(seed=seed)
+    inp = synth.make_inputs(w, "cuda", L=L, B=B)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    Wq, Wk = inp["Wq16"], inp["Wk16"]
+    if per_kv:  # one indexer key per retrieval kv head: the first query head's W_k16
+        Wk = Wk[[s for s in range(0, w.H_ret, w.G)]].contiguous()
+    role = inp["kv_role"]
+    res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=p, window=w.window, n_sink=w.n_sink,
+                            k16_per_kv_head=int(per_kv))
+    torch.cuda.synchronize()
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    Wqb, Wkb = bits(Wq), bits(Wk)
+    q16g, k16g = bits(res["q16"]), bits(res["k16"])
+    sel = {key: val.cpu().numpy() for key, val in res["sel"].items()}
+    o = res["o"].float().cpu().numpy()
+    lse = res["lse"].cpu().numpy()
+    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
+    p = float(np.float32(p))  # the C ABI takes p as fp32
+    k16slot = [s // w.G for s in range(w.H_ret)] if per_kv else list(range(w.H_ret))
+    if positions is None:
+        positions = np.arange(L)
+    positions = np.asarray(sorted(set(int(x) for x in positions)))
+
+    # (i) projections
+    if check_proj:
+        for b in range(B):
+            for s, h in enumerate(ret):
+                check_projection(q16g[b, positions, s], qb[b, positions, h], Wqb[s])
+            for s in sorted(set(k16slot)):
+                g = ret[s * (w.G if per_kv else 1)] // w.G
+                check_projection(k16g[b, :, s], kb[b, :, g], Wkb[s])
+    k16o = oracle_k16(kb, Wkb, w, per_kv)
+
+    n_band, o_ret_g, o_ret_o, o_loc_g, o_loc_o = 0, [], [], [], []
+    lse_err = 0.0
+    for b in range(B):
+        for i in positions:
+            rows = np.array([(0, 0, h) for h in ret])
+            q1, q16_1 = qb[b:b + 1, i:i + 1], q16g[b:b + 1, i:i + 1]
+            kb1, vb1, k16g1 = kb[b:b + 1], vb[b:b + 1], k16g[b:b + 1]
+            # (ii) selection on the GPU's q16/k16
+            r2 = oracle.retrieval_rows(q1, kb1, vb1, q16_1, k16g1, rows, np.arange(len(ret)),
+                                       np.array(k16slot), H=w.H, Hkv=w.Hkv, q_pos0=int(i), p=p,
+                                       scale=SCALE, want_sel=True)
+            for s in range(len(ret)):
+                s64 = row_scores(q16g[b, i, s], k16g[b, :, k16slot[s]], int(i))
+                n_band += check_row_selection(
+                    s64, p, r2["t"][s], r2["sel"][s], float(sel["thr"][b, s, i]),
+                    int(sel["jtie"][b, s, i]), int(sel["count"][b, s, i]),
+                    float(sel["mass"][b, s, i]))
+            # (iii) end to end with the oracle's own projections
+            q16o = np.stack([oracle.project(qb[b, i, h][None], Wqb[s])[0][0]
+                             for s, h in enumerate(ret)])[None, None]
+            r3 = oracle.retrieval_rows(q1, kb1, vb1, q16o, k16o[b:b + 1], rows,
+                                       np.arange(len(ret)), np.array(k16slot), H=w.H, Hkv=w.Hkv,
+                                       q_pos0=int(i), p=p, scale=SCALE)
+            o_ret_o.append(r3["o"])
+            o_ret_g.append(o[b, i, ret])
+            lse_err = max(lse_err, float(np.abs(lse[b, ret, i] - r3["lse"]).max()))
+            if loc:
+                rl = oracle.local_rows(q1, kb1, vb1, np.array([(0, 0, h) for h in loc]), H=w.H,
+                                       Hkv=w.Hkv, q_pos0=int(i), window=w.window,
+                                       n_sink=w.n_sink, scale=SCALE)
+                o_loc_o.append(rl["o"])
+                o_loc_g.append(o[b, i, loc])
+                lse_err = max(lse_err, float(np.abs(lse[b, loc, i] - rl["lse"]).max()))
+    check_outputs(np.concatenate(o_ret_g), np.concatenate(o_ret_o), "retrieval heads")
+    if loc:
+        check_outputs(np.concatenate(o_loc_g), np.concatenate(o_loc_o), "local heads")
+    assert lse_err <= LSE_ABS, lse_err
+    return dict(n_band=n_band, res=res, inp=inp)
+
+
+W = synth.WORKLOADS
+
+
+def test_prefill_2k_full():
+    """The 2K workload, every row of every head."""
+    run_prefill(W["prefill_2k"], 2048, 0.9)
+
+
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 130, 1000])
+@pytest.mark.parametrize("p", [0.0, 0.5, 0.9, 1.0])
+def test_prefill_ragged_and_limits(L, p):
+    run_prefill(W["prefill_2k"], L, p, check_proj=(p == 0.5))
+
+
+def test_prefill_batch2_per_kv_k16():
+    run_prefill(W["prefill_2k"], 700, 0.9, B=2, per_kv=True)
+
+
+@pytest.mark.parametrize("p", [0.8, 0.9, 0.95, 0.99])
+def test_prefill_temperature_sweep(p):
+    """The 32K workload's generator (per-query temperature, 2 retrieval kv heads)
+    at 4K rows, sampled positions."""
+    rng = np.random.default_rng(1)
+    pos = np.concatenate([np.arange(8), np.arange(4096 - 8, 4096), rng.integers(0, 4096, 48)])
+    run_prefill(W["prefill_32k"], 4096, p, positions=pos, check_proj=False)
+
+
+def test_prefill_multihop_and_group_needles():
+    rng = np.random.default_rng(2)
+    pos = np.concatenate([[0, 1, 4095, 4096, 4097, 8191], rng.integers(0, 8192, 32)])
+    run_prefill(W["prefill_128k"], 8192, 0.95, positions=pos, check_proj=False)
+    run_prefill(W["prefill_1m"], 8192, 0.95, positions=pos, check_proj=False)
+
+
+def test_prefill_all_scores_equal():
+    """W_q16 = 0: every indexer score is 0, so every key ties; the kept set is the
+    ceil(p * N) lowest indices."""
+    w = W["prefill_2k"]
+    inp = synth.make_inputs(w, "cuda", L=300)
+    Wq = torch.zeros_like(inp["Wq16"])
+    for p in (0.0, 0.37, 0.9):
+        res = rtp_layer_prefill(inp["q"], inp["k"], inp["v"], Wq, inp["Wk16"], inp["kv_role"],
+                                p=p, window=w.window, n_sink=w.n_sink)
+        cnt = res["sel"]["count"].cpu().numpy()
+        jt = res["sel"]["jtie"].cpu().numpy()
+        N = np.arange(1, 301)
+        expect = np.maximum(1, np.ceil(float(np.float32(p)) * N)).astype(int)
+        assert np.array_equal(cnt[0, 0], expect)
+        assert np.array_equal(jt[0, 0], expect - 1)
+        assert np.all(res["sel"]["thr"].cpu().numpy() == 0.0)

@@ -172,7 +172,8 @@ def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None =
     key_adds, q_adds = [], []
     if w.needles == "residue8":
         for slot in range(H_ret):
-            pos = rng.choice(np.arange(4, Lk), size=8, replace=False)
+            cnt = min(8, max(Lk - 4, 0))
+            pos = rng.choice(np.arange(4, Lk), size=cnt, replace=False) if cnt else []
             for gidx, n in enumerate(pos):
                 key_adds.append((0, int(n), slot))
                 rows = np.arange(Lq)
@@ -181,8 +182,8 @@ def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None =
     elif w.needles == "uniform64":
         for b in range(B):
             for slot in range(H_ret):
-                cnt = int(rng.integers(0, 65))
-                pos = rng.choice(Lk - 1, size=cnt, replace=False)
+                cnt = min(int(rng.integers(0, 65)), max(Lk - 1, 0))
+                pos = rng.choice(Lk - 1, size=cnt, replace=False) if cnt else []
                 for n in pos:
                     key_adds.append((b, int(n), slot))
                 if cnt:

@@ -42,11 +42,13 @@
  *  - Arguments are validated on the host before anything is launched; an error
  *    return means nothing was enqueued.  Launch failures return RTP_ERR_CUDA.
  *  - Workspace: `ws` is caller-owned device memory of at least
- *    rtp_workspace_size(op, ...) bytes, 256-byte aligned.  It must be zeroed
- *    once before first use (rtp_workspace_init); the kernels leave it ready for
- *    the next call.  Concurrent calls must not share a workspace.  The first
- *    bytes of every workspace hold a device status word that kernels set when a
- *    bounded wait gives up; rtp_get_device_status reads it.
+ *    rtp_workspace_size(op, ...) bytes, 256-byte aligned.  Zero it once before
+ *    first use (rtp_workspace_init) so the device status word starts clear; each
+ *    call resets whatever it accumulates into, so one workspace may serve calls
+ *    of any shape in turn.  Concurrent calls must not share a workspace.  The
+ *    first 256 bytes of every workspace hold a device status word that kernels
+ *    set when an internal consistency check fails; rtp_get_device_status reads
+ *    it.
  */
 #ifndef RTP_H_
 #define RTP_H_

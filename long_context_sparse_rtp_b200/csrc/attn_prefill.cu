@@ -270,16 +270,21 @@ __global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const AttnParams
         alpha[hh] = (mrow[hh] == -INFINITY) ? 0.f : exp2f(mrow[hh] - mnew);
         mrow[hh] = mnew;
       }
+      // probabilities rounded to bf16 once: the same values feed PV and the
+      // normaliser, so the output stays an exact convex combination of them
+      uint32_t pp[8][2];
       float ls[2] = {0.f, 0.f};
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+      for (int nt = 0; nt < 8; ++nt) {
+        float pr[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool hi = e >= 2;
-          const float pr = (s[nt][e] == -INFINITY) ? 0.f : exp2f(s[nt][e] - mrow[hi]);
-          s[nt][e] = pr;
-          ls[hi] += pr;
-        }
+        for (int e = 0; e < 4; ++e)
+          pr[e] = (s[nt][e] == -INFINITY) ? 0.f : exp2f(s[nt][e] - mrow[e >= 2]);
+        pp[nt][0] = pack_bf16x2(pr[0], pr[1]);
+        pp[nt][1] = pack_bf16x2(pr[2], pr[3]);
+        ls[0] += bf16_lo(pp[nt][0]) + bf16_hi(pp[nt][0]);
+        ls[1] += bf16_lo(pp[nt][1]) + bf16_hi(pp[nt][1]);
+      }
       lrow[0] = lrow[0] * alpha[0] + ls[0];
       lrow[1] = lrow[1] * alpha[1] + ls[1];
 #pragma unroll
@@ -292,11 +297,8 @@ __global__ void __launch_bounds__(kThreads) attn_prefill_kernel(const AttnParams
       // O += P V
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        uint32_t pa[4];
-        pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
-        pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
-        pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+        const uint32_t pa[4] = {pp[2 * kk][0], pp[2 * kk][1], pp[2 * kk + 1][0],
+                                pp[2 * kk + 1][1]};
 #pragma unroll
         for (int dp = 0; dp < 8; ++dp) {
           const int q = lane >> 3;

@@ -60,6 +60,11 @@ struct ScoreParams {
   int64_t k16_sb, k16_sl;
   float* scores;
   float* cmax;
+  unsigned long long* hist_m;   // zeroed here for this group's rows
+  uint32_t* hist_c;
+  unsigned long long* zsum;
+  uint32_t* counter;
+  uint32_t* mcount;
   int N, Lk_pad, n_chunks, n_ret, n_rkv, G;
   int per_kv;
 };
@@ -84,6 +89,19 @@ __global__ void __launch_bounds__(kScoreThreads) dec_score_kernel(const ScorePar
     q[4] = bf16_lo(a.z); q[5] = bf16_hi(a.z); q[6] = bf16_lo(a.w); q[7] = bf16_hi(a.w);
     q[8] = bf16_lo(c.x); q[9] = bf16_hi(c.x); q[10] = bf16_lo(c.y); q[11] = bf16_hi(c.y);
     q[12] = bf16_lo(c.z); q[13] = bf16_hi(c.z); q[14] = bf16_lo(c.w); q[15] = bf16_hi(c.w);
+  }
+  if (chunk == 0) {
+    // later kernels accumulate into these with atomics: start them at zero
+    const int row0 = b * p.n_ret + rk * G;
+    for (int x = tid; x < G * kDecBins; x += kScoreThreads) {
+      p.hist_m[(int64_t)row0 * kDecBins + x] = 0ull;
+      p.hist_c[(int64_t)row0 * kDecBins + x] = 0u;
+    }
+    if (tid < G) {
+      p.zsum[row0 + tid] = 0ull;
+      p.counter[row0 + tid] = 0u;
+    }
+    if (tid == 0) p.mcount[grp] = 0u;
   }
   const int slot = p.per_kv ? rk : hr;
   const uint16_t* kb = p.k16 + b * p.k16_sb + (int64_t)slot * kR;
@@ -705,16 +723,19 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
       alpha[hh] = (mrow[hh] == -INFINITY) ? 0.f : exp2f(mrow[hh] - mnew);
       mrow[hh] = mnew;
     }
+    uint32_t pp[2][2];
     float ls[2] = {0.f, 0.f};
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+    for (int n = 0; n < 2; ++n) {
+      float pr[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool hi = e >= 2;
-        const float pr = (s[n][e] == -INFINITY) ? 0.f : exp2f(s[n][e] - mrow[hi]);
-        s[n][e] = pr;
-        ls[hi] += pr;
-      }
+      for (int e = 0; e < 4; ++e)
+        pr[e] = (s[n][e] == -INFINITY) ? 0.f : exp2f(s[n][e] - mrow[e >= 2]);
+      pp[n][0] = pack_bf16x2(pr[0], pr[1]);
+      pp[n][1] = pack_bf16x2(pr[2], pr[3]);
+      ls[0] += bf16_lo(pp[n][0]) + bf16_hi(pp[n][0]);
+      ls[1] += bf16_lo(pp[n][1]) + bf16_hi(pp[n][1]);
+    }
     lrow[0] = lrow[0] * alpha[0] + ls[0];
     lrow[1] = lrow[1] * alpha[1] + ls[1];
 #pragma unroll
@@ -724,11 +745,7 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
       oacc[d][2] *= alpha[1];
       oacc[d][3] *= alpha[1];
     }
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(s[0][0], s[0][1]);
-    pa[1] = pack_bf16x2(s[0][2], s[0][3]);
-    pa[2] = pack_bf16x2(s[1][0], s[1][1]);
-    pa[3] = pack_bf16x2(s[1][2], s[1][3]);
+    const uint32_t pa[4] = {pp[0][0], pp[0][1], pp[1][0], pp[1][1]};
 #pragma unroll
     for (int dp = 0; dp < 8; ++dp) {
       const int q = lane >> 3;
@@ -860,6 +877,9 @@ rtp_status decode_range(const rtp_shape* shape, const int16_t* kv_heads, int n_g
   prm.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part);
   prm.mcount = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.mcount);
   for (int i = 0; i < n_groups; ++i) prm.kvh[i] = kv_heads[i];
+  if (cudaMemsetAsync(prm.mcount, 0, (size_t)shape->B * n_groups * sizeof(uint32_t), s) !=
+      cudaSuccess)
+    return RTP_ERR_CUDA;
   return launch_dec_attn<false>(prm, shape->B, s);
 }
 
@@ -1024,6 +1044,11 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     sp.n_rkv = hm.n_rkv;
     sp.G = hm.G;
     sp.per_kv = k16_per_kv_head;
+    sp.hist_m = reinterpret_cast<unsigned long long*>(w + L.hist_m);
+    sp.hist_c = reinterpret_cast<uint32_t*>(w + L.hist_c);
+    sp.zsum = reinterpret_cast<unsigned long long*>(w + L.zsum);
+    sp.counter = reinterpret_cast<uint32_t*>(w + L.counter);
+    sp.mcount = reinterpret_cast<uint32_t*>(w + L.mcount);
     const size_t smem = (size_t)hm.G * (kDecChunk + 4) * sizeof(float);
     if (cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)

@@ -71,11 +71,37 @@ def check_row_selection(s64, p, t_orc, sel_orc, t_gpu, jtie_gpu, count_gpu, mass
 
 
 def check_outputs(o_gpu: np.ndarray, o_orc: np.ndarray, what: str):
+    if o_gpu.size == 0:
+        return 0.0, 0.0
     err = np.abs(o_gpu.astype(np.float64) - o_orc)
     mx, mean = float(err.max()), float(err.mean())
     assert mx <= O_MAX_ABS, f"{what}: max-abs {mx:.3e}"
     assert mean <= O_MEAN_ABS, f"{what}: mean-abs {mean:.3e}"
     return mx, mean
+
+
+def check_row_outputs(o_gpu, o_same_sel, o_e2e, same_count, same_sel, what,
+                      max_skip_count=0.01, max_skip_sel=0.05):
+    """Output parity of retrieval rows.
+
+    o_same_sel: the oracle run on the GPU's own q16/k16 (same kept sets up to
+    in-band keys); checked on every row where the kept-set sizes agree.
+    o_e2e: the oracle run end to end on its own projections; checked on the rows
+    whose oracle kept set does not change between the two projections (a 1-ulp
+    bf16 difference in q16/k16 can legitimately reorder near-tied keys, and in
+    a row with few kept keys that changes the output by O(1)).  The fraction of
+    rows skipped by either rule is bounded."""
+    n = len(o_gpu)
+    same_count = np.asarray(same_count, bool)
+    same_sel = np.asarray(same_sel, bool)
+    assert (~same_count).sum() <= max(2, max_skip_count * n), (int((~same_count).sum()), n)
+    assert (~same_sel).sum() <= max(2, max_skip_sel * n), (int((~same_sel).sum()), n)
+    r1 = check_outputs(o_gpu[same_count], o_same_sel[same_count],
+                       what + " vs oracle on the GPU's q16/k16")
+    both = same_count & same_sel
+    r2 = check_outputs(o_gpu[both], o_e2e[both], what + " vs oracle end to end")
+    return dict(skip_count=int((~same_count).sum()), skip_sel=int((~same_sel).sum()),
+                max_abs=r1[0], mean_abs=r1[1], e2e_max_abs=r2[0], e2e_mean_abs=r2[1])
 
 
 def oracle_k16(k_bits, Wk_bits, w: synth.Workload, per_kv: bool = False):

@@ -13,8 +13,8 @@ from long_context_sparse_rtp_b200 import (rtp_dense_attn, rtp_index_scores, rtp_
                                           rtp_layer_prefill, rtp_local_attn,
                                           rtp_sparse_attn_decode, rtp_sparse_attn_prefill,
                                           rtp_topp_select, synth)
-from rtp_check import (LSE_ABS, bits, check_outputs, check_row_selection, oracle_k16,
-                       row_scores)
+from rtp_check import (LSE_ABS, bits, check_outputs, check_row_outputs, check_row_selection,
+                       oracle_k16, row_scores)
 
 pytestmark = pytest.mark.gpu
 
@@ -82,10 +82,14 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
             q16o[b, 0, s] = oracle.project(qb[b, 0, h][None], Wqb[s])[0][0]
     k16o = oracle_k16(kb, Wkb, w, per_kv)
     r3 = oracle.retrieval_rows(qb, kb, vb, q16o, k16o, rows, slots, ks, H=w.H, Hkv=w.Hkv,
-                               q_pos0=P, p=p, scale=SCALE)
+                               q_pos0=P, p=p, scale=SCALE, want_sel=True)
     og = np.stack([o[b, 0, h] for (b, _, h) in rows])
-    check_outputs(og, r3["o"], "retrieval decode")
-    assert np.abs(np.array([lse[b, h, 0] for (b, _, h) in rows]) - r3["lse"]).max() <= LSE_ABS
+    same_count = np.array([int(sel["count"][b, slots[r]]) == int(r2["count"][r])
+                           for r, (b, _, h) in enumerate(rows)])
+    same_sel = np.array([np.array_equal(a, c) for a, c in zip(r2["sel"], r3["sel"])])
+    check_row_outputs(og, r2["o"], r3["o"], same_count, same_sel, "retrieval decode")
+    lg = np.array([lse[b, h, 0] for (b, _, h) in rows])
+    assert np.abs(lg - r2["lse"])[same_count].max(initial=0.0) <= LSE_ABS
     if loc:
         lrows = np.array([(b, 0, h) for b in range(B) for h in loc])
         rl = oracle.local_rows(qb, kb, vb, lrows, H=w.H, Hkv=w.Hkv, q_pos0=P, window=w.window,

@@ -1,0 +1,46 @@
+"""GPU parity at the workloads' full sizes, on sampled query rows (the oracle
+computes those rows one by one): 32K with the p sweep, 128K multi-hop, 1M.
+Sampled rows always include the first and last rows and the rows around the
+local window's edge."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_rtp_b200 import synth
+from test_gpu_prefill import run_prefill
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+W = synth.WORKLOADS
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def sample_rows(L, window, n_sink, n_random, seed):
+    rng = np.random.default_rng(seed)
+    edge = [window - 1, window, window + 1, window + n_sink - 1, window + n_sink,
+            window + n_sink + 1]
+    pos = [0, 1, 2, 3, 4, 5, 63, 64, 65, L - 2, L - 1] + edge + list(rng.integers(0, L, n_random))
+    return sorted(set(int(x) for x in pos if 0 <= x < L))
+
+
+@pytest.mark.parametrize("p", [0.8, 0.9, 0.95, 0.99])
+def test_prefill_32k_p_sweep(p):
+    w = W["prefill_32k"]
+    run_prefill(w, w.L, p, positions=sample_rows(w.L, w.window, w.n_sink, 12, 30),
+                check_proj=False)
+
+
+def test_prefill_128k_multihop():
+    w = W["prefill_128k"]
+    run_prefill(w, w.L, w.p, positions=sample_rows(w.L, w.window, w.n_sink, 16, 31),
+                check_proj=False)
+
+
+def test_prefill_1m():
+    w = W["prefill_1m"]
+    run_prefill(w, w.L, w.p, positions=sample_rows(w.L, w.window, w.n_sink, 8, 32),
+                check_proj=False)

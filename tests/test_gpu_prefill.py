@@ -60,24 +60,27 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=p, window=w.window, n_sink=w.n_sink,
                             k16_per_kv_head=int(per_kv))
     torch.cuda.synchronize()
-    qb, kb, vb = bits(q), bits(k), bits(v)
-    Wqb, Wkb = bits(Wq), bits(Wk)
-    q16g, k16g = bits(res["q16"]), bits(res["k16"])
-    sel = {key: val.cpu().numpy() for key, val in res["sel"].items()}
-    o = res["o"].float().cpu().numpy()
-    lse = res["lse"].cpu().numpy()
-    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
-    p = float(np.float32(p))  # the C ABI takes p as fp32
-    k16slot = [s // w.G for s in range(w.H_ret)] if per_kv else list(range(w.H_ret))
     if positions is None:
         positions = np.arange(L)
     positions = np.asarray(sorted(set(int(x) for x in positions)))
+    # only the sampled query rows travel to the host
+    pidx = torch.as_tensor(positions, device=q.device)
+    kb, vb = bits(k), bits(v)
+    Wqb, Wkb = bits(Wq), bits(Wk)
+    qs, q16s = bits(q[:, pidx]), bits(res["q16"][:, pidx])
+    k16g = bits(res["k16"])
+    sel = {key: val[:, :, pidx].cpu().numpy() for key, val in res["sel"].items()}
+    o = res["o"][:, pidx].float().cpu().numpy()
+    lse = res["lse"][:, :, pidx].cpu().numpy()
+    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
+    p = float(np.float32(p))  # the C ABI takes p as fp32
+    k16slot = [s // w.G for s in range(w.H_ret)] if per_kv else list(range(w.H_ret))
 
     # (i) projections
     if check_proj:
         for b in range(B):
             for s, h in enumerate(ret):
-                check_projection(q16g[b, positions, s], qb[b, positions, h], Wqb[s])
+                check_projection(q16s[b, :, s], qs[b, :, h], Wqb[s])
             for s in sorted(set(k16slot)):
                 g = ret[s * (w.G if per_kv else 1)] // w.G
                 check_projection(k16g[b, :, s], kb[b, :, g], Wkb[s])
@@ -87,41 +90,41 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     same_count, same_sel = [], []
     lse_err = 0.0
     for b in range(B):
-        for i in positions:
+        for x, i in enumerate(positions):
             rows = np.array([(0, 0, h) for h in ret])
-            q1, q16_1 = qb[b:b + 1, i:i + 1], q16g[b:b + 1, i:i + 1]
+            q1, q16_1 = qs[b:b + 1, x:x + 1], q16s[b:b + 1, x:x + 1]
             kb1, vb1, k16g1 = kb[b:b + 1], vb[b:b + 1], k16g[b:b + 1]
             # (ii) selection on the GPU's q16/k16
             r2 = oracle.retrieval_rows(q1, kb1, vb1, q16_1, k16g1, rows, np.arange(len(ret)),
                                        np.array(k16slot), H=w.H, Hkv=w.Hkv, q_pos0=int(i), p=p,
                                        scale=SCALE, want_sel=True)
             for s in range(len(ret)):
-                s64 = row_scores(q16g[b, i, s], k16g[b, :, k16slot[s]], int(i))
+                s64 = row_scores(q16s[b, x, s], k16g[b, :, k16slot[s]], int(i))
                 n_band += check_row_selection(
-                    s64, p, r2["t"][s], r2["sel"][s], float(sel["thr"][b, s, i]),
-                    int(sel["jtie"][b, s, i]), int(sel["count"][b, s, i]),
-                    float(sel["mass"][b, s, i]))
-                same_count.append(int(sel["count"][b, s, i]) == int(r2["count"][s]))
+                    s64, p, r2["t"][s], r2["sel"][s], float(sel["thr"][b, s, x]),
+                    int(sel["jtie"][b, s, x]), int(sel["count"][b, s, x]),
+                    float(sel["mass"][b, s, x]))
+                same_count.append(int(sel["count"][b, s, x]) == int(r2["count"][s]))
             o_ret_a.append(r2["o"])
             # (iii) end to end with the oracle's own projections
-            q16o = np.stack([oracle.project(qb[b, i, h][None], Wqb[s])[0][0]
+            q16o = np.stack([oracle.project(qs[b, x, h][None], Wqb[s])[0][0]
                              for s, h in enumerate(ret)])[None, None]
             r3 = oracle.retrieval_rows(q1, kb1, vb1, q16o, k16o[b:b + 1], rows,
                                        np.arange(len(ret)), np.array(k16slot), H=w.H, Hkv=w.Hkv,
                                        q_pos0=int(i), p=p, scale=SCALE, want_sel=True)
             same_sel.extend(np.array_equal(a, c) for a, c in zip(r2["sel"], r3["sel"]))
             o_ret_o.append(r3["o"])
-            o_ret_g.append(o[b, i, ret])
-            ok = np.array([int(sel["count"][b, s, i]) == int(r2["count"][s]) for s in range(len(ret))])
+            o_ret_g.append(o[b, x, ret])
+            ok = np.array([int(sel["count"][b, s, x]) == int(r2["count"][s]) for s in range(len(ret))])
             if ok.any():
-                lse_err = max(lse_err, float(np.abs(lse[b, ret, i] - r2["lse"])[ok].max()))
+                lse_err = max(lse_err, float(np.abs(lse[b, ret, x] - r2["lse"])[ok].max()))
             if loc:
                 rl = oracle.local_rows(q1, kb1, vb1, np.array([(0, 0, h) for h in loc]), H=w.H,
                                        Hkv=w.Hkv, q_pos0=int(i), window=w.window,
                                        n_sink=w.n_sink, scale=SCALE)
                 o_loc_o.append(rl["o"])
-                o_loc_g.append(o[b, i, loc])
-                lse_err = max(lse_err, float(np.abs(lse[b, loc, i] - rl["lse"]).max()))
+                o_loc_g.append(o[b, x, loc])
+                lse_err = max(lse_err, float(np.abs(lse[b, loc, x] - rl["lse"]).max()))
     stats = check_row_outputs(np.concatenate(o_ret_g), np.concatenate(o_ret_a),
                               np.concatenate(o_ret_o), same_count, same_sel, "retrieval heads")
     if loc:

@@ -49,7 +49,38 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=3)
+    ap.add_argument("--case", default=None, choices=["decode", "select", "prefill", "dense"],
+                    help="run one small case twice and exit (for profilers)")
+    ap.add_argument("--L", type=int, default=16384, help="sequence length for --case")
     return ap.parse_args()
+
+
+def run_case(args):
+    """One case, run twice (the second is the one to capture), then exit."""
+    import torch
+    from long_context_sparse_rtp_b200 import (build, rtp_dense_attn, rtp_index_scores,
+                                              rtp_layer_prefill, rtp_topp_select, synth)
+    build.build()
+    torch.cuda.set_device(0)
+    if args.case == "decode":
+        st = decode_state(0)
+        for _ in range(2):
+            decode_step(st, None, None)
+    else:
+        w = synth.WORKLOADS[PREFILL_WL]
+        inp = synth.make_inputs(w, "cuda", L=args.L)
+        q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
+        for _ in range(2):
+            if args.case == "select":
+                q16, k16 = rtp_index_scores(q, k, Wq, Wk, role)
+                rtp_topp_select(q16, k16, role, w.p, H=w.H)
+            elif args.case == "prefill":
+                rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window,
+                                  n_sink=w.n_sink)
+            else:
+                rtp_dense_attn(q, k, v)
+    torch.cuda.synchronize()
+    print(f"case {args.case} ok")
 
 
 def peaks():
@@ -423,6 +454,9 @@ def _cuda():
 # ------------------------------------------------------------------ main
 def main():
     args = parse()
+    if args.case is not None:
+        run_case(args)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

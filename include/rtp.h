@@ -75,7 +75,8 @@ typedef enum rtp_status {
     RTP_ERR_ALIGNMENT = 3,           /* a pointer or stride breaks 16-byte row alignment */
     RTP_ERR_WORKSPACE_TOO_SMALL = 4, /* ws_bytes < rtp_workspace_size(...) */
     RTP_ERR_CUDA = 5,                /* a CUDA runtime call or launch failed */
-    RTP_ERR_DEVICE_TIMEOUT = 6       /* a kernel's bounded wait gave up (device status) */
+    RTP_ERR_DEVICE_TIMEOUT = 6,      /* a kernel's bounded wait gave up (device status) */
+    RTP_ERR_SCRATCH_LIMIT = 7        /* shape needs more than the built-in scratch array */
 } rtp_status;
 
 typedef enum rtp_op {
@@ -184,6 +185,35 @@ RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role
                           int32_t n_sink, rtp_view q, rtp_view k, rtp_view v,
                           float softmax_scale, rtp_view o, float* lse, void* ws,
                           size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Local-head decode that allocates nothing (the paper has no counterpart; this
+ * is a deployment variant of rtp_local_attn with shape->Lq == 1).
+ *
+ * For callers that cannot hand the library a workspace: code that runs under a
+ * memory allocator it does not own (a host framework's fixed pool, a plugin
+ * interface that passes only inputs and outputs) or in a phase where device
+ * allocation is not allowed.  The split-KV partials and merge counters live in
+ * one file-scope device array of RTP_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU
+ * which loads the library holds until the process exits.
+ *  - Same arguments and results as rtp_local_attn for one decode token, minus
+ *    the workspace.  Shapes whose partials exceed the array return
+ *    RTP_ERR_SCRATCH_LIMIT before anything is enqueued (the need is about
+ *    B * local_kv_heads * ceil(n_keys / 512) * 8320 bytes; n_keys is the
+ *    number of sink and window keys, at most window + n_sink).
+ *  - The first call on a device looks the array's device address up
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    outside any stream capture.
+ *  - Every call reuses the same array and clears the counters it needs; calls
+ *    that overlap on the GPU (other streams, other threads) race on it and
+ *    must be serialised by the caller.
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define RTP_NOALLOC_SCRATCH_BYTES (8u << 20)
+RTP_API rtp_status rtp_local_attn_decode_noalloc(const rtp_shape* shape, const uint8_t* kv_role,
+                                                 int32_t window, int32_t n_sink, rtp_view q,
+                                                 rtp_view k, rtp_view v, float softmax_scale,
+                                                 rtp_view o, float* lse, rtp_stream_t stream);
 
 /*
  * Baseline: dense causal softmax attention on every head (keys 0..P).

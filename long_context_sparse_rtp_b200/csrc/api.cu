@@ -17,6 +17,7 @@ extern "C" const char* rtp_status_string(rtp_status status) {
     case RTP_ERR_WORKSPACE_TOO_SMALL: return "RTP_ERR_WORKSPACE_TOO_SMALL";
     case RTP_ERR_CUDA: return "RTP_ERR_CUDA";
     case RTP_ERR_DEVICE_TIMEOUT: return "RTP_ERR_DEVICE_TIMEOUT";
+    case RTP_ERR_SCRATCH_LIMIT: return "RTP_ERR_SCRATCH_LIMIT";
   }
   return "RTP_ERR_UNKNOWN";
 }

@@ -17,6 +17,7 @@
 //                G heads as mma rows, per-head masks, online softmax; the last
 //                CTA of a group merges the splits.
 #include <algorithm>
+#include <mutex>
 
 #include "rtp_host.h"
 
@@ -1118,4 +1119,70 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
   prm.mcount = reinterpret_cast<uint32_t*>(w + L.mcount);
   for (int i = 0; i < hm.n_rkv; ++i) prm.kvh[i] = hm.rkv[i];
   return launch_dec_attn<true>(prm, shape->B, s);
+}
+
+// ====================================================================== no-allocation variant
+// Scratch for rtp_local_attn_decode_noalloc: split-KV partials and merge
+// counters in a file-scope device array instead of a caller workspace.
+namespace rtp {
+namespace {
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device (looked up once per device;
+// in host code the symbol itself is only a host-side stand-in).
+rtp_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RTP_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RTP_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return RTP_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RTP_OK;
+}
+
+}  // namespace
+}  // namespace rtp
+
+extern "C" rtp_status rtp_local_attn_decode_noalloc(const rtp_shape* shape,
+                                                    const uint8_t* kv_role, int32_t window,
+                                                    int32_t n_sink, rtp_view q, rtp_view k,
+                                                    rtp_view v, float softmax_scale, rtp_view o,
+                                                    float* lse, rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  if (shape->Lq != 1) return RTP_ERR_INVALID_ARG;
+  if ((st = check_causal(shape)) != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, 0, &hm)) != RTP_OK) return st;
+  if (window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return RTP_ERR_INVALID_ARG;
+  if (shape->B == 0 || hm.n_lkv == 0) return RTP_OK;
+  if (hm.G > 16 || (256 % hm.G) != 0) return RTP_ERR_UNSUPPORTED;
+  if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(k, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
+  // the same key set decode_range visits
+  const int64_t P = shape->q_pos0;
+  const int64_t n_sink_eff = std::min<int64_t>((int64_t)n_sink, P + 1);
+  int64_t win_lo = P - window + 1;
+  if (win_lo < n_sink_eff) win_lo = n_sink_eff;
+  const int64_t n_keys = n_sink_eff + (P - win_lo + 1);
+  const size_t need = range_decode_ws_layout(n_keys, shape->B * hm.n_lkv).total;
+  if (need > (size_t)RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != RTP_OK) return st;
+  return decode_range(shape, hm.lkv, hm.n_lkv, window, n_sink, q, k, v, softmax_scale, o, lse,
+                      scratch, (size_t)RTP_NOALLOC_SCRATCH_BYTES,
+                      reinterpret_cast<cudaStream_t>(stream));
 }

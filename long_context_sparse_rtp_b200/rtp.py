@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "librtp.so")
 RTP_OK = 0
 STATUS = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_UNSUPPORTED",
           3: "RTP_ERR_ALIGNMENT", 4: "RTP_ERR_WORKSPACE_TOO_SMALL", 5: "RTP_ERR_CUDA",
-          6: "RTP_ERR_DEVICE_TIMEOUT"}
+          6: "RTP_ERR_DEVICE_TIMEOUT", 7: "RTP_ERR_SCRATCH_LIMIT"}
 OP_INDEX_SCORES, OP_TOPP_SELECT, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_LOCAL, OP_DENSE = range(6)
 
 
@@ -69,13 +69,15 @@ def lib():
                                                      P, P, P, P, P, sz, P]
                 L.rtp_local_attn.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P, sz, P]
                 L.rtp_dense_attn.argtypes = [S, V, V, V, f32, V, P, P, sz, P]
+                L.rtp_local_attn_decode_noalloc.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P]
                 L.rtp_status_string.restype = ctypes.c_char_p
                 L.rtp_status_string.argtypes = [ctypes.c_int]
                 L.rtp_get_device_status.argtypes = [P, P]
                 L.rtp_version.restype = ctypes.c_char_p
                 for fn in ("rtp_workspace_init", "rtp_index_scores", "rtp_topp_select",
                            "rtp_sparse_attn_prefill", "rtp_sparse_attn_decode",
-                           "rtp_local_attn", "rtp_dense_attn", "rtp_get_device_status"):
+                           "rtp_local_attn", "rtp_dense_attn", "rtp_get_device_status",
+                           "rtp_local_attn_decode_noalloc"):
                     getattr(L, fn).restype = ctypes.c_int
                 _lib = L
     return _lib
@@ -289,4 +291,24 @@ def rtp_dense_attn(q, k, v, *, scale=None, q_pos0=0, o=None, lse=None, stream=No
     _check("rtp_dense_attn", lib().rtp_dense_attn(
         ctypes.byref(shp), view(q), view(k), view(v), ctypes.c_float(scale), view(o),
         _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def rtp_local_attn_decode_noalloc(q, k, v, kv_role, *, window, n_sink, scale=None, q_pos0=None,
+                                  o=None, lse=None, stream=None):
+    """Local-head decode (Lq == 1) that allocates nothing inside the library: its
+    scratch is a fixed 8 MiB device array.  For callers that cannot provide a
+    workspace.  Calls that overlap on the GPU race on that array."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    q_pos0 = Lk - 1 if q_pos0 is None else q_pos0
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, Lq), float("nan"), dtype=torch.float32, device=q.device)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    _check("rtp_local_attn_decode_noalloc", lib().rtp_local_attn_decode_noalloc(
+        ctypes.byref(shp), _role(kv_role), window, n_sink, view(q), view(k), view(v),
+        ctypes.c_float(scale), view(o), _ptr(lse), _stream(stream)))
     return o, lse

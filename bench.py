@@ -272,54 +272,63 @@ def union_size(st, sel):
 
 
 def bench_decode(args, world, rank, local, pk):
+    """Device time of the decode step, replayed from one CUDA graph."""
     import torch
+    from long_context_sparse_rtp_b200 import DecodeGraph
     st = decode_state(rank)
+    w, L = st["w"], st["L"]
     flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
 
     def flush():
         flushbuf.fill_(1.0)
 
-    def step():
-        decode_step(st, None, None)
+    def make(trace_on=False):
+        g = DecodeGraph(st["k"], st["v"], st["k16"], st["Wq"], st["Wk"], st["role"], H=w.H,
+                        pos=L - 1, p=w.p, window=w.window, n_sink=w.n_sink, trace=trace_on)
+        g.q.copy_(st["q"])
+        return g
 
+    g = make()
     clocks = ClockSampler(local)
     clocks.start()
-    ms, _ = time_steps(step, args.steps, args.warmup, world, flush)
+    ms, _ = time_steps(g.replay, args.steps, args.warmup, world, flush)
     clk = clocks.stop()
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
-    # traced pass for per-kernel durations (same steps, same flushes)
-    _, kern = time_steps(step, args.steps, 1, world, flush, traced=True)
+    # per-kernel device times: a second graph whose trace events are graph nodes
+    gt = make(trace_on=True)
+    kern = {}
+    for _ in range(args.steps):
+        flush()
+        gt.replay()
+        torch.cuda.synchronize()
+        for name, (n, t) in trace_read().items():
+            a0, a1 = kern.get(name, (0, 0.0))
+            kern[name] = (a0 + n, a1 + t)
+    trace(False)
     res = decode_step(st, None, None)
     torch.cuda.synchronize()
     union, compute_sel = union_size(st, res)
     B = st["q"].shape[0]
     nbytes = decode_bytes(st, union)
     return dict(st=st, ms_step=ms_step, clocks=clk, kern=kern, union=union,
-                compute_sel=compute_sel, bytes=nbytes, B=B, flush=flush)
+                compute_sel=compute_sel, bytes=nbytes, B=B, flush=flush, graph=g)
 
 
 def bench_decode_e2e(dec, args, world):
     """Through the public API with host buffers: H2D of the new token's q/k/v
-    rows from pinned memory, the layer call, D2H of the output."""
+    rows from pinned memory, one DecodeGraph step, D2H of the output."""
     import torch
-    from long_context_sparse_rtp_b200 import rtp_layer_decode
     st = dec["st"]
-    w, L = st["w"], st["L"]
+    g = dec["graph"]
+    L = st["L"]
     hq = st["q"].cpu().pin_memory()
     hk = st["k"][:, L - 1:].contiguous().cpu().pin_memory()
     hv = st["v"][:, L - 1:].contiguous().cpu().pin_memory()
     ho = torch.empty_like(hq).pin_memory()
-    dq = torch.empty_like(st["q"])
 
     def step():
-        dq.copy_(hq, non_blocking=True)
-        st["k"][:, L - 1:].copy_(hk, non_blocking=True)
-        st["v"][:, L - 1:].copy_(hv, non_blocking=True)
-        r = rtp_layer_decode(dq, st["k"][:, L - 1:], st["k"], st["v"], st["k16"], st["Wq"],
-                             st["Wk"], st["role"], pos=L - 1, p=w.p, window=w.window,
-                             n_sink=w.n_sink)
-        ho.copy_(r["o"], non_blocking=True)
+        g.step(hq, hk, hv, ho)
 
     ms, _ = time_steps(step, args.steps, args.warmup, world, dec["flush"])
     ms = max_over_ranks(ms, world)
@@ -478,7 +487,7 @@ def main():
     B = dec["B"]
     value = B * world / (dec["ms_step"] / 1e3)
     kern = dec["kern"]
-    n_launch = sum(n for (n, _) in kern.values()) // args.steps
+    n_launch = sum(n for (n, _) in kern.values()) // args.steps  # our kernels per step
     score_ms = kern["dec_score"][1] / kern["dec_score"][0]
     score_bytes = dec["bytes"]["k16"]
     achieved = score_bytes / (score_ms / 1e3) / 1e9
@@ -511,7 +520,8 @@ def main():
         "clocks": dec["clocks"],
         "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms, "api": "rtp_layer_decode (python binding, host buffers)"},
+                "ms_per_step": e2e_ms,
+                "api": "DecodeGraph.step (pinned host q/k/v in, o out; one graph replay)"},
     }
     if pre is not None:
         per = pre["per_kernel"]

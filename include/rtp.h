@@ -199,8 +199,9 @@ RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role
  *  - Same arguments and results as rtp_local_attn for one decode token, minus
  *    the workspace.  Shapes whose partials exceed the array return
  *    RTP_ERR_SCRATCH_LIMIT before anything is enqueued (the need is about
- *    B * local_kv_heads * ceil(n_keys / 512) * 8320 bytes; n_keys is the
- *    number of sink and window keys, at most window + n_sink).
+ *    8320 bytes per (batch entry, local kv head, split), with
+ *    min(ceil(296 / (B * local_kv_heads)), ceil(n_keys / 64)) splits; n_keys
+ *    is the number of sink and window keys, at most window + n_sink).
  *  - The first call on a device looks the array's device address up
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    outside any stream capture.
@@ -232,10 +233,12 @@ RTP_API rtp_status rtp_get_device_status(void* ws, rtp_stream_t stream);
 /*
  * Kernel trace (no counterpart in the paper; a measurement aid).  While
  * enabled, every kernel the library launches is bracketed by two CUDA events
- * recorded on its launch stream.  rtp_trace_read synchronises those events and
- * returns, per kernel name, the number of launches and their summed device time
- * (ms).  Not thread-safe against concurrent enable/reset; costs nothing while
- * disabled.
+ * recorded on its launch stream (inside a stream capture they become external
+ * event-record nodes, so each replay of the graph re-times its kernels).
+ * rtp_trace_read synchronises those events and returns, per kernel name, the
+ * number of recorded launches and their summed device time (ms) as of the last
+ * time each event completed.  Not thread-safe against concurrent enable/reset;
+ * costs nothing while disabled.
  */
 typedef struct rtp_trace_entry {
     char name[48];

@@ -20,4 +20,4 @@ from .rtp import (  # noqa: F401
     rtp_version,
     rtp_workspace_size,
 )
-from .layer import rtp_layer_decode, rtp_layer_prefill  # noqa: F401
+from .layer import DecodeGraph, rtp_layer_decode, rtp_layer_prefill  # noqa: F401

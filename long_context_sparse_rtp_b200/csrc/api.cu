@@ -70,11 +70,21 @@ cudaEvent_t take_event() {
 }
 }  // namespace
 
+// Under stream capture the events become event-record nodes of the graph
+// (external records), so every replay of the graph times its kernels again.
+void record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
+}
+
 void trace_begin(const char* name, cudaStream_t s) {
   if (!g_trace_on) return;
   std::lock_guard<std::mutex> lk(g_trace_mu);
   TraceRec r{name, take_event(), take_event()};
-  cudaEventRecord(r.start, s);
+  record(r.start, s);
   g_trace.push_back(r);
   g_open = (int)g_trace.size() - 1;
 }
@@ -82,12 +92,22 @@ void trace_begin(const char* name, cudaStream_t s) {
 void trace_end(cudaStream_t s) {
   if (!g_trace_on || g_open < 0) return;
   std::lock_guard<std::mutex> lk(g_trace_mu);
-  if (g_open < (int)g_trace.size()) cudaEventRecord(g_trace[g_open].stop, s);
+  if (g_open < (int)g_trace.size()) record(g_trace[g_open].stop, s);
   g_open = -1;
 }
 }  // namespace rtp
 
-extern "C" void rtp_trace_enable(int on) { rtp::g_trace_on = on != 0; }
+extern "C" void rtp_trace_enable(int on) {
+  rtp::g_trace_on = on != 0;
+  if (on) {  // keep a few events ready so that a capture does not have to create them
+    std::lock_guard<std::mutex> lk(rtp::g_trace_mu);
+    while (rtp::g_free.size() < 64) {
+      cudaEvent_t e = nullptr;
+      if (cudaEventCreate(&e) != cudaSuccess) break;
+      rtp::g_free.push_back(e);
+    }
+  }
+}
 
 extern "C" void rtp_trace_reset(void) {
   std::lock_guard<std::mutex> lk(rtp::g_trace_mu);

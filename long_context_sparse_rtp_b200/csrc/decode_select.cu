@@ -1,0 +1,933 @@
+// decode_select.cu -- exact top-p for one decode token per batch entry
+// (rtp_sparse_attn_decode): "Dynamic Top-p Selection Mechanism" of the
+// paper-graph-ui summary of arXiv 2605.16928, token-exact.
+//
+// Masses are kept relative to score-bin edges so that no kernel needs the row
+// max before it has seen the row: a key with score s sits in the absolute bin
+// b = floor(4 s) and contributes exp(s - (b+1)/4) in (0.78, 1] to that bin, as
+// 21-bit fixed point.  Integer sums are exact and order-free, so every decision
+// below is deterministic.  Per kv group of G retrieval query heads:
+//   1. score     stream the k16 cache once (HBM-bound), s = q16 . k16 in fp32
+//                with a fixed FMA order, scores kept in the workspace; each CTA
+//                bins its 1024 x G scores in shared memory (one 256-bin window per
+//                head, 32-bit atomics) and adds the occupied bins into the row's
+//                2048-bin absolute histogram in global memory;
+//   2. merge     per row: bin masses scaled to the top occupied bin in fp64, Z,
+//                T = p Z, and the crossing bin, by fixed-order block scans;
+//   3. collect   per chunk: keys above the crossing bin are kept, keys in it are
+//                candidates (collected per row); one ordered list per kv group of
+//                every token some head may keep.  The last CTA of a group sorts
+//                each row's candidates by (score desc, index asc), one warp per
+//                row, and walks them to the exact cut (t, jtie);
+//   4. attend    gathered split-KV attention over the lists (decode.cu); the
+//                candidate heads are settled there with s > t or (s == t, j <= jtie).
+// Rows with scores outside [-256, 256) or more than 4096 keys in the crossing bin
+// are resolved by a radix refinement over the stored scores (slower, rare).
+#include <algorithm>
+
+#include "rtp_host.h"
+
+namespace rtp {
+namespace {
+
+constexpr int kIdxBits = 21;
+constexpr unsigned long long kIdxMask = (1ull << kIdxBits) - 1;
+constexpr int kKeyBits = 32 + kIdxBits;
+constexpr int kThreads = 256;
+constexpr double kFix21 = 1.0 / 2097152.0;  // 2^-21
+constexpr int kWarpCap = 512;               // candidates one warp sorts on its own
+
+// Absolute score bin floor(s * kappa), rounding toward -inf; clamped far outside
+// the histogram's range so that bin arithmetic never overflows.
+__device__ __forceinline__ int sbin(float s) {
+  const float x = fminf(fmaxf(__fmul_rn(s, kDecKappa), -1073741824.0f), 1073741824.0f);
+  return __float2int_rd(x);
+}
+// Mass of a key relative to the upper edge (b+1)/kappa of its bin: (0.78, 1].
+__device__ __forceinline__ float wbin(float s, int b) {
+  const float edge = __fmul_rn((float)(b + 1), 1.0f / kDecKappa);
+  return exp2f(__fmul_rn(__fsub_rn(s, edge), kLog2e));
+}
+__device__ __forceinline__ uint32_t fixed21(float w) {
+  return __float2uint_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f));
+}
+// Mass relative to a reference score m (refinement path).
+__device__ __forceinline__ float wrel(float s, float m) {
+  return exp2f(__fmul_rn(__fsub_rn(s, m), kLog2e));
+}
+__device__ __forceinline__ unsigned long long comp_key(float s, int j) {
+  return ((unsigned long long)score_key(s) << kIdxBits) | (kIdxMask - (unsigned long long)j);
+}
+__device__ __forceinline__ float key_score(uint32_t key) {
+  const uint32_t b = (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
+  return __uint_as_float(b);
+}
+
+// ------------------------------------------------------------------ 1. score + histogram
+struct ScoreParams {
+  const uint16_t* q16;
+  int64_t q16_sb;
+  const uint16_t* k16;
+  int64_t k16_sb, k16_sl;
+  float* scores;
+  unsigned long long* hist_m;  // [rows][kDecGBins]
+  uint32_t* hist_c;
+  uint32_t* flags;             // [rows]: 1 = a score fell outside the histogram range
+  uint32_t* ncand;
+  uint32_t* counter;
+  uint32_t* mcount;
+  int N, Lk_pad, n_ret, n_rkv, G, per_kv;
+};
+
+__global__ void __launch_bounds__(kThreads) dec_score_kernel(const ScoreParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int G = p.G;
+  float* sc = reinterpret_cast<float*>(smem_raw);                        // [G][kDecChunk+4]
+  uint32_t* hm = reinterpret_cast<uint32_t*>(sc + G * (kDecChunk + 4));  // [G][kDecWin]
+  uint32_t* hc = hm + G * kDecWin;                                       // [G][kDecWin]
+  int* top = reinterpret_cast<int*>(hc + G * kDecWin);                   // [G]
+
+  const int chunk = blockIdx.x;
+  const int grp = blockIdx.y;  // b * n_rkv + rk
+  const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
+  const int tid = threadIdx.x;
+  const int row0 = b * p.n_ret + rk * G;
+  if (chunk == 0) {  // the later kernels of this call count into these
+    if (tid < G) p.ncand[row0 + tid] = 0u;
+    if (tid == 0) {
+      p.counter[grp] = 0u;
+      p.mcount[grp] = 0u;
+    }
+  }
+  for (int x = tid; x < G * kDecWin; x += kThreads) {
+    hm[x] = 0u;
+    hc[x] = 0u;
+  }
+
+  const int hh = tid % G;  // G divides 256: constant per thread
+  const int hr = rk * G + hh;
+  float q[kR];
+  {
+    const uint16_t* qp = p.q16 + b * p.q16_sb + (int64_t)hr * kR;
+    const uint4 a = *reinterpret_cast<const uint4*>(qp);
+    const uint4 c = *reinterpret_cast<const uint4*>(qp + 8);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      q[2 * i] = bf16_lo(w[i]);
+      q[2 * i + 1] = bf16_hi(w[i]);
+    }
+  }
+  const int slot = p.per_kv ? rk : hr;
+  const uint16_t* kb = p.k16 + b * p.k16_sb + (int64_t)slot * kR;
+  const int j0 = chunk * kDecChunk;
+  const int pairs = kDecChunk * G;
+  constexpr int kUnroll = 4;
+  for (int base = 0; base < pairs; base += kThreads * kUnroll) {
+    uint4 ka[kUnroll], kc[kUnroll];
+    int tok[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int pr = base + u * kThreads + tid;
+      tok[u] = pr / G;
+      const int j = j0 + tok[u];
+      if (pr < pairs && j < p.N) {
+        const uint16_t* src = kb + (int64_t)j * p.k16_sl;
+        ka[u] = __ldcs(reinterpret_cast<const uint4*>(src));
+        kc[u] = __ldcs(reinterpret_cast<const uint4*>(src + 8));
+      } else {
+        ka[u] = make_uint4(0, 0, 0, 0);
+        kc[u] = ka[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int pr = base + u * kThreads + tid;
+      if (pr >= pairs) continue;
+      const uint32_t w[8] = {ka[u].x, ka[u].y, ka[u].z, ka[u].w,
+                             kc[u].x, kc[u].y, kc[u].z, kc[u].w};
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        s = fmaf(q[2 * c], bf16_lo(w[c]), s);
+        s = fmaf(q[2 * c + 1], bf16_hi(w[c]), s);
+      }
+      s = s + 0.0f;
+      const int j = j0 + tok[u];
+      sc[hh * (kDecChunk + 4) + tok[u]] = (j < p.N) ? s : -INFINITY;
+    }
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int h = warp; h < G; h += kThreads / 32) {
+    const float* row = sc + h * (kDecChunk + 4);
+    float mx = -INFINITY;
+    float* dst = p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0;
+    for (int x = lane * 4; x < kDecChunk; x += 128) {
+      const float4 v = *reinterpret_cast<const float4*>(row + x);
+      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+      *reinterpret_cast<float4*>(dst + x) = v;
+    }
+    mx = warp_max(mx);
+    if (lane == 0) top[h] = sbin(mx);
+  }
+  __syncthreads();
+  const int nvalid = min(kDecChunk, p.N - j0);
+  for (int idx = tid; idx < G * kDecChunk; idx += kThreads) {
+    const int h = idx / kDecChunk, x = idx % kDecChunk;
+    if (x >= nvalid) continue;
+    const float s = sc[h * (kDecChunk + 4) + x];
+    const int bb = sbin(s);
+    const int wi = top[h] - bb;  // 0 = the chunk's top bin
+    const uint32_t f = fixed21(wbin(s, bb));
+    if (wi < kDecWin) {
+      atomicAdd(&hm[h * kDecWin + wi], f);
+      atomicAdd(&hc[h * kDecWin + wi], 1u);
+    } else {  // far below this chunk's max: straight into the row histogram
+      int gb = bb - kDecGLo;
+      if (gb < 0) {
+        gb = 0;
+        atomicOr(&p.flags[row0 + h], 1u);
+      }
+      atomicAdd(&p.hist_m[(int64_t)(row0 + h) * kDecGBins + gb], (unsigned long long)f);
+      atomicAdd(&p.hist_c[(int64_t)(row0 + h) * kDecGBins + gb], 1u);
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < G * kDecWin; x += kThreads) {
+    const uint32_t c = hc[x];
+    if (c == 0) continue;
+    const int h = x / kDecWin, wi = x % kDecWin;
+    int gb = top[h] - wi - kDecGLo;
+    if (gb < 0 || gb >= kDecGBins) {
+      gb = gb < 0 ? 0 : kDecGBins - 1;
+      atomicOr(&p.flags[row0 + h], 1u);
+    }
+    atomicAdd(&p.hist_m[(int64_t)(row0 + h) * kDecGBins + gb], (unsigned long long)hm[x]);
+    atomicAdd(&p.hist_c[(int64_t)(row0 + h) * kDecGBins + gb], c);
+  }
+}
+
+// ------------------------------------------------------------------ 2. per-row merge
+struct MergeParams {
+  const unsigned long long* hist_m;
+  const uint32_t* hist_c;
+  const uint32_t* flags;
+  RowSel* rowsel;
+  float p;
+};
+
+constexpr int kBinsPerThread = kDecGBins / kThreads;  // 8
+
+__global__ void __launch_bounds__(kThreads) dec_merge_kernel(const MergeParams p) {
+  __shared__ double wsum[kThreads / 32];
+  __shared__ uint32_t wcnt[kThreads / 32];
+  __shared__ int s_top;
+  __shared__ int s_cross;
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // thread t holds the bins t*8 .. t*8+7 counted down from the top bin
+  unsigned long long hmv[kBinsPerThread];
+  uint32_t hcv[kBinsPerThread];
+  int occ = -1;  // highest occupied absolute bin seen by this thread
+#pragma unroll
+  for (int i = 0; i < kBinsPerThread; ++i) {
+    const int gb = kDecGBins - 1 - (tid * kBinsPerThread + i);
+    hmv[i] = p.hist_m[(int64_t)row * kDecGBins + gb];
+    hcv[i] = p.hist_c[(int64_t)row * kDecGBins + gb];
+    if (hcv[i] && occ < 0) occ = gb;
+  }
+  if (tid == 0) {
+    s_top = -1;
+    s_cross = 0x7FFFFFFF;
+  }
+  __syncthreads();
+  if (occ >= 0) atomicMax(&s_top, occ);
+  __syncthreads();
+  const int gtop = s_top < 0 ? 0 : s_top;  // every row has at least one key
+  const double etop = (double)(gtop + kDecGLo + 1) / (double)kDecKappa;
+  double M[kBinsPerThread];
+  double tsum = 0.0;
+  uint32_t tcnt = 0;
+#pragma unroll
+  for (int i = 0; i < kBinsPerThread; ++i) {
+    const int gb = kDecGBins - 1 - (tid * kBinsPerThread + i);
+    M[i] = hcv[i] ? (double)hmv[i] * kFix21 *
+                        exp((double)(gb + kDecGLo + 1) / (double)kDecKappa - etop)
+                  : 0.0;
+    tsum += M[i];
+    tcnt += hcv[i];
+  }
+  // fixed-order scans over threads (bins in descending order)
+  double incl = tsum;
+  uint32_t cincl = tcnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, o);
+    if (lane >= o) {
+      incl += y;
+      cincl += cy;
+    }
+  }
+  if (lane == 31) {
+    wsum[warp] = incl;
+    wcnt[warp] = cincl;
+  }
+  __syncthreads();
+  double before = 0.0, Z = 0.0;
+  uint32_t cbefore = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) {
+      before += wsum[w];
+      cbefore += wcnt[w];
+    }
+    Z += wsum[w];
+  }
+  before += incl - tsum;
+  cbefore += cincl - tcnt;
+  const double T = (double)p.p * Z;
+  // this thread's bins: the first one where the running mass reaches T
+  double acc = before;
+  int my_cross = 0x7FFFFFFF;
+  double my_above = 0.0;
+  uint32_t my_cnt = 0, my_nin = 0;
+  uint32_t c = cbefore;
+#pragma unroll
+  for (int i = 0; i < kBinsPerThread; ++i) {
+    if (hcv[i] && my_cross == 0x7FFFFFFF && acc + M[i] >= T) {
+      my_cross = tid * kBinsPerThread + i;
+      my_above = acc;
+      my_cnt = c;
+      my_nin = hcv[i];
+    }
+    acc += M[i];
+    c += hcv[i];
+  }
+  if (my_cross != 0x7FFFFFFF) atomicMin(&s_cross, my_cross);
+  __syncthreads();
+  const int cross = s_cross;
+  const bool flagged = p.flags[row] != 0;
+  if (cross != 0x7FFFFFFF && my_cross == cross) {
+    RowSel rs;
+    rs.bstar = (kDecGBins - 1 - cross) + kDecGLo;
+    rs.T = T;
+    rs.Z = Z;
+    rs.above = my_above;
+    rs.cnt_above = my_cnt;
+    rs.n_in = my_nin;
+    rs.scale_b = kFix21 * exp((double)(rs.bstar + 1) / (double)kDecKappa - etop);
+    rs.mode = (p.p >= 1.f) ? 1 : ((flagged || rs.n_in > (uint32_t)kDecCap) ? 2 : 0);
+    p.rowsel[row] = rs;
+  }
+  if (cross == 0x7FFFFFFF && tid == 0) {  // T out of reach by rounding, or p >= 1
+    RowSel rs;
+    rs.bstar = kDecGLo - 1;
+    rs.T = T;
+    rs.Z = Z;
+    rs.above = 0.0;
+    rs.cnt_above = 0;
+    rs.n_in = 0;
+    rs.scale_b = 0.0;
+    rs.mode = (p.p >= 1.f) ? 1 : 2;
+    p.rowsel[row] = rs;
+  }
+}
+
+// ------------------------------------------------------------------ 3. collect + compact + cut
+struct CollectParams {
+  const float* scores;
+  const RowSel* rowsel;
+  unsigned long long* cand;  // [rows][kDecCap]
+  uint32_t* ncand;
+  uint2* list;               // [groups][Lk_pad]
+  int32_t* lcount;           // [groups][nc]
+  int32_t* loff;             // [groups][nc + 1]
+  uint32_t* counter;
+  RowRes* rowres;
+  float* thr;
+  int32_t* jtie;
+  int32_t* count;
+  float* mass;
+  DevStatus* status;
+  int N, Lk_pad, nc, n_ret, n_rkv, G;
+  float p;
+};
+
+struct CollectSmem {
+  RowSel rs[16];
+  int wsum[kThreads / 32];
+  int is_last;
+  int big[16];                       // rows left for the block-wide paths
+  int nbig;
+  // last CTA
+  unsigned long long wc[kThreads / 32][kWarpCap];  // per-warp candidate sort
+  unsigned long long cand[kDecCap];                // block-wide sort
+  unsigned long long tsum[kThreads];
+  unsigned long long hm[256];
+  uint32_t hc[256];
+  unsigned long long red[kThreads / 32];
+  int ncand;
+  int cut;
+  unsigned long long s_acc;
+  uint32_t s_cnt, s_nin;
+  int s_k;
+};
+
+__device__ unsigned long long block_sum_u64(unsigned long long v, unsigned long long* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o);
+    v += ((unsigned long long)hi << 32) | lo;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  unsigned long long s = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+  __syncthreads();
+  return s;
+}
+
+// Bitonic sort of a[0..n) descending (padded with zeros to a power of two), one block.
+__device__ void sort_desc_block(unsigned long long* a, int n) {
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  for (int i = n + threadIdx.x; i < n2; i += blockDim.x) a[i] = 0ull;
+  __syncthreads();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n2; i += blockDim.x) {
+        const int l = i ^ j;
+        if (l > i) {
+          const bool desc = (i & k) == 0;
+          const unsigned long long x = a[i], y = a[l];
+          if (desc ? (x < y) : (x > y)) {
+            a[i] = y;
+            a[l] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// The same, one warp.
+__device__ void sort_desc_warp(unsigned long long* a, int n) {
+  const int lane = threadIdx.x & 31;
+  int n2 = 1;
+  while (n2 < n) n2 <<= 1;
+  for (int i = n + lane; i < n2; i += 32) a[i] = 0ull;
+  __syncwarp();
+  for (int k = 2; k <= n2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = lane; i < n2; i += 32) {
+        const int l = i ^ j;
+        if (l > i) {
+          const bool desc = (i & k) == 0;
+          const unsigned long long x = a[i], y = a[l];
+          if (desc ? (x < y) : (x > y)) {
+            a[i] = y;
+            a[l] = x;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Walk the sorted candidates a[0..n) of a normal row with one warp: the first k
+// with above + scale * sum_{a<=k} fixed21(w(a)) >= T.  Lane 0 returns the result.
+__device__ RowRes warp_walk(const unsigned long long* a, int n, const RowSel& rs) {
+  const int lane = threadIdx.x & 31;
+  const int per = (n + 31) / 32;
+  const int a0 = lane * per, a1 = min(n, a0 + per);
+  unsigned long long seg = 0;
+  for (int i = a0; i < a1; ++i)
+    seg += fixed21(wbin(key_score((uint32_t)(a[i] >> kIdxBits)), rs.bstar));
+  unsigned long long incl = seg;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t lo = __shfl_up_sync(0xffffffffu, (uint32_t)incl, o);
+    const uint32_t hi = __shfl_up_sync(0xffffffffu, (uint32_t)(incl >> 32), o);
+    if (lane >= o) incl += ((unsigned long long)hi << 32) | lo;
+  }
+  unsigned long long cum = incl - seg;
+  int my = 0x7FFFFFFF;
+  unsigned long long mycum = 0;
+  for (int i = a0; i < a1; ++i) {
+    cum += fixed21(wbin(key_score((uint32_t)(a[i] >> kIdxBits)), rs.bstar));
+    if (rs.above + (double)cum * rs.scale_b >= rs.T) {
+      my = i;
+      mycum = cum;
+      break;
+    }
+  }
+  int cut = my;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cut = min(cut, __shfl_xor_sync(0xffffffffu, cut, o));
+  unsigned long long cutcum;
+  if (cut == 0x7FFFFFFF) {  // rounding kept T out of reach: keep every candidate
+    cut = n - 1;
+    cutcum = __shfl_sync(0xffffffffu, incl, 31);
+  } else {
+    const unsigned ball = __ballot_sync(0xffffffffu, my == cut);
+    const int src = __ffs(ball) - 1;
+    const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)mycum, src);
+    const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(mycum >> 32), src);
+    cutcum = ((unsigned long long)hi << 32) | lo;
+  }
+  RowRes out;
+  const unsigned long long ck = a[cut];
+  out.t = key_score((uint32_t)(ck >> kIdxBits));
+  out.jtie = (int32_t)(kIdxMask - (ck & kIdxMask));
+  out.count = (int32_t)(rs.cnt_above + cut + 1);
+  out.mass = (float)((rs.above + (double)cutcum * rs.scale_b) / rs.Z);
+  return out;
+}
+
+// Block-wide walk for rows with more than kWarpCap candidates.
+template <class F>
+__device__ int walk_cut(CollectSmem& sm, int n, F&& fmass, double base, double scale, double T,
+                        unsigned long long& cum_out) {
+  const int tid = threadIdx.x;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int a0 = tid * per, a1 = min(n, a0 + per);
+  unsigned long long seg = 0;
+  for (int a = a0; a < a1; ++a) seg += fmass(a);
+  sm.tsum[tid] = seg;
+  if (tid == 0) sm.cut = 0x7FFFFFFF;
+  __syncthreads();
+  unsigned long long before = 0;
+  for (int q = 0; q < tid; ++q) before += sm.tsum[q];
+  unsigned long long cum = before;
+  for (int a = a0; a < a1; ++a) {
+    cum += fmass(a);
+    if (base + (double)cum * scale >= T) {
+      atomicMin(&sm.cut, a);
+      break;
+    }
+  }
+  __syncthreads();
+  int cut = sm.cut;
+  if (cut == 0x7FFFFFFF) cut = n - 1;
+  if (tid == 0) {
+    unsigned long long c2 = 0;
+    for (int a = 0; a <= cut; ++a) c2 += fmass(a);
+    sm.tsum[0] = c2;
+  }
+  __syncthreads();
+  cum_out = sm.tsum[0];
+  __syncthreads();
+  return cut;
+}
+
+// Exact cut of one row by radix refinement over all its stored scores (masses
+// relative to the row max, composite (score, index) keys, 8-bit digits).  One CTA.
+__device__ void refine_row(CollectSmem& sm, const CollectParams& p, const float* srow,
+                           RowRes& out) {
+  const int tid = threadIdx.x;
+  const int N = p.N;
+  float mx = -INFINITY;
+  for (int j = tid; j < N; j += kThreads) mx = fmaxf(mx, srow[j]);
+  mx = warp_max(mx);
+  __syncthreads();
+  if ((tid & 31) == 0) sm.tsum[tid >> 5] = (unsigned long long)__float_as_uint(mx);
+  __syncthreads();
+  float m = -INFINITY;
+  for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, __uint_as_float((uint32_t)sm.tsum[w]));
+  __syncthreads();
+  unsigned long long z = 0;
+  for (int j = tid; j < N; j += kThreads) z += mass_fixed40(wrel(srow[j], m));
+  const unsigned long long Z = block_sum_u64(z, sm.red);
+  const double T = (double)p.p * (double)Z;
+  int pb = 0;
+  unsigned long long prefix = 0, acc_above = 0;
+  uint32_t cnt_above = 0, n_in = (uint32_t)N;
+  auto member = [&](float s, int j, unsigned long long& ck) -> bool {
+    ck = comp_key(s, j);
+    return pb == 0 || (ck >> (kKeyBits - pb)) == prefix;
+  };
+  for (int lvl = 0; lvl < 8 && n_in > (uint32_t)kDecCap && pb < kKeyBits; ++lvl) {
+    const int w = min(8, kKeyBits - pb);
+    for (int bb = tid; bb < 256; bb += kThreads) {
+      sm.hm[bb] = 0;
+      sm.hc[bb] = 0;
+    }
+    __syncthreads();
+    for (int j = tid; j < N; j += kThreads) {
+      const float s = srow[j];
+      unsigned long long ck;
+      if (!member(s, j, ck)) continue;
+      const int digit = (int)((ck >> (kKeyBits - pb - w)) & ((1ull << w) - 1));
+      atomicAdd(&sm.hm[(1 << w) - 1 - digit], mass_fixed40(wrel(s, m)));
+      atomicAdd(&sm.hc[(1 << w) - 1 - digit], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned long long a = acc_above;
+      uint32_t c = cnt_above, nin = 0;
+      int last = -1, k = -1;
+      for (int bb = 0; bb < (1 << w); ++bb) {
+        if (sm.hc[bb] == 0) continue;
+        last = bb;
+        if ((double)(a + sm.hm[bb]) >= T) {
+          k = bb;
+          nin = sm.hc[bb];
+          break;
+        }
+        a += sm.hm[bb];
+        c += sm.hc[bb];
+      }
+      if (k < 0) {
+        k = last;
+        a -= sm.hm[last];
+        c -= sm.hc[last];
+        nin = sm.hc[last];
+      }
+      sm.s_acc = a;
+      sm.s_cnt = c;
+      sm.s_nin = nin;
+      sm.s_k = (1 << w) - 1 - k;
+    }
+    __syncthreads();
+    acc_above = sm.s_acc;
+    cnt_above = sm.s_cnt;
+    n_in = sm.s_nin;
+    prefix = (prefix << w) | (unsigned long long)sm.s_k;
+    pb += w;
+    __syncthreads();
+  }
+  if (tid == 0) sm.ncand = 0;
+  __syncthreads();
+  for (int j = tid; j < N; j += kThreads) {
+    unsigned long long ck;
+    if (!member(srow[j], j, ck)) continue;
+    const int idx = atomicAdd(&sm.ncand, 1);
+    if (idx < kDecCap) sm.cand[idx] = ck;
+  }
+  __syncthreads();
+  int n = min(sm.ncand, kDecCap);
+  if (sm.ncand > kDecCap && tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 31);
+  sort_desc_block(sm.cand, n);
+  unsigned long long cum = 0;
+  const int cut = walk_cut(
+      sm, n,
+      [&](int a) {
+        return mass_fixed40(wrel(key_score((uint32_t)(sm.cand[a] >> kIdxBits)), m));
+      },
+      (double)acc_above, 1.0, T, cum);
+  const unsigned long long ck = sm.cand[cut];
+  out.t = key_score((uint32_t)(ck >> kIdxBits));
+  out.jtie = (int32_t)(kIdxMask - (ck & kIdxMask));
+  out.count = (int32_t)(cnt_above + cut + 1);
+  out.mass = (float)((double)(acc_above + cum) / (double)Z);
+}
+
+__device__ void write_result(const CollectParams& p, int row, const RowRes& rr) {
+  p.rowres[row] = rr;
+  if (p.thr) p.thr[row] = rr.t;
+  if (p.jtie) p.jtie[row] = rr.jtie;
+  if (p.count) p.count[row] = rr.count;
+  if (p.mass) p.mass[row] = rr.mass;
+}
+
+__global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  CollectSmem& sm = *reinterpret_cast<CollectSmem*>(smem_raw);
+  const int chunk = blockIdx.x, grp = blockIdx.y;
+  const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
+  const int tid = threadIdx.x;
+  const int G = p.G;
+  const int row0 = b * p.n_ret + rk * G;
+  if (tid < G) sm.rs[tid] = p.rowsel[row0 + tid];
+  __syncthreads();
+  const int j0 = chunk * kDecChunk + tid * 4;
+  uint32_t keep[4] = {0, 0, 0, 0}, cand[4] = {0, 0, 0, 0};
+  for (int h = 0; h < G; ++h) {
+    const RowSel& rs = sm.rs[h];
+    const float4 v =
+        *reinterpret_cast<const float4*>(p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0);
+    const float vs[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = j0 + e;
+      if (j >= p.N) continue;
+      if (rs.mode == 1) {
+        keep[e] |= 1u << h;
+        continue;
+      }
+      if (rs.mode == 2) {  // settled per key by the attention kernel
+        cand[e] |= 1u << h;
+        continue;
+      }
+      const int bb = sbin(vs[e]);
+      if (bb > rs.bstar) {
+        keep[e] |= 1u << h;
+      } else if (bb == rs.bstar) {
+        cand[e] |= 1u << h;
+        const uint32_t idx = atomicAdd(&p.ncand[row0 + h], 1u);
+        if (idx < (uint32_t)kDecCap)
+          p.cand[(int64_t)(row0 + h) * kDecCap + idx] = comp_key(vs[e], j);
+      }
+    }
+  }
+  // ordered compaction of the tokens some head may keep
+  const int lane = tid & 31, warp = tid >> 5;
+  int cnt = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) cnt += (keep[e] | cand[e]) != 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sm.wsum[warp] = incl;
+  __syncthreads();
+  int off = incl - cnt;
+  for (int w = 0; w < warp; ++w) off += sm.wsum[w];
+  uint2* dst = p.list + (int64_t)grp * p.Lk_pad + chunk * kDecChunk;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (keep[e] | cand[e]) dst[off++] = make_uint2((uint32_t)(j0 + e), keep[e] | (cand[e] << 16));
+  if (tid == kThreads - 1) {
+    int tot = 0;
+    for (int w = 0; w < kThreads / 32; ++w) tot += sm.wsum[w];
+    p.lcount[(int64_t)grp * p.nc + chunk] = tot;
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sm.is_last = (atomicAdd(&p.counter[grp], 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+
+  // ---- last CTA of the group
+  // list offsets: exclusive prefix of the chunk counts
+  {
+    const int nc = p.nc;
+    const int per = (nc + kThreads - 1) / kThreads;
+    const int c0 = tid * per, c1 = min(nc, c0 + per);
+    int segsum = 0;
+    for (int c = c0; c < c1; ++c) segsum += __ldcg(&p.lcount[(int64_t)grp * nc + c]);
+    int inc = segsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    __syncthreads();
+    if (lane == 31) sm.wsum[warp] = inc;
+    __syncthreads();
+    int run = inc - segsum;
+    for (int w = 0; w < warp; ++w) run += sm.wsum[w];
+    int32_t* lo = p.loff + (int64_t)grp * (nc + 1);
+    for (int c = c0; c < c1; ++c) {
+      lo[c] = run;
+      run += __ldcg(&p.lcount[(int64_t)grp * nc + c]);
+    }
+    if (tid == kThreads - 1) {
+      int tot = 0;
+      for (int w = 0; w < kThreads / 32; ++w) tot += sm.wsum[w];
+      lo[nc] = tot;
+    }
+  }
+  // rows: one warp each for the common case
+  if (tid == 0) sm.nbig = 0;
+  __syncthreads();
+  for (int h = warp; h < G; h += kThreads / 32) {
+    const RowSel rs = sm.rs[h];
+    const int row = row0 + h;
+    if (rs.mode == 1) {
+      if (lane == 0) {
+        RowRes rr;
+        rr.t = -INFINITY;
+        rr.jtie = p.N - 1;
+        rr.count = p.N;
+        rr.mass = 1.f;
+        write_result(p, row, rr);
+      }
+      continue;
+    }
+    const int n = (int)__ldcg(&p.ncand[row]);
+    if (rs.mode == 2 || n > kWarpCap || n == 0) {
+      if (lane == 0) sm.big[atomicAdd(&sm.nbig, 1)] = h;
+      continue;
+    }
+    unsigned long long* a = sm.wc[warp];
+    for (int i = lane; i < n; i += 32) a[i] = __ldcg(&p.cand[(int64_t)row * kDecCap + i]);
+    __syncwarp();
+    sort_desc_warp(a, n);
+    const RowRes rr = warp_walk(a, n, rs);
+    if (lane == 0) write_result(p, row, rr);
+    __syncwarp();
+  }
+  __syncthreads();
+  // rows left: many candidates (block sort) or refinement over all scores
+  const int nbig = sm.nbig;
+  for (int q = 0; q < nbig; ++q) {
+    const int h = sm.big[q];
+    const RowSel rs = sm.rs[h];
+    const int row = row0 + h;
+    RowRes rr;
+    const int n = (int)min(__ldcg(&p.ncand[row]), (uint32_t)kDecCap);
+    if (rs.mode == 0 && n > 0) {
+      for (int a = tid; a < n; a += kThreads)
+        sm.cand[a] = __ldcg(&p.cand[(int64_t)row * kDecCap + a]);
+      __syncthreads();
+      sort_desc_block(sm.cand, n);
+      unsigned long long cum = 0;
+      const int bst = rs.bstar;
+      const int cut = walk_cut(
+          sm, n,
+          [&](int a) {
+            return (unsigned long long)fixed21(
+                wbin(key_score((uint32_t)(sm.cand[a] >> kIdxBits)), bst));
+          },
+          rs.above, rs.scale_b, rs.T, cum);
+      const unsigned long long ck = sm.cand[cut];
+      rr.t = key_score((uint32_t)(ck >> kIdxBits));
+      rr.jtie = (int32_t)(kIdxMask - (ck & kIdxMask));
+      rr.count = (int32_t)(rs.cnt_above + cut + 1);
+      rr.mass = (float)((rs.above + (double)cum * rs.scale_b) / rs.Z);
+    } else {
+      refine_row(sm, p, p.scores + (int64_t)row * p.Lk_pad, rr);
+    }
+    if (tid == 0) write_result(p, row, rr);
+    __syncthreads();
+  }
+  if (tid == 0) p.counter[grp] = 0u;
+}
+
+}  // namespace
+}  // namespace rtp
+
+using namespace rtp;
+
+extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8_t* kv_role,
+                                             int32_t k16_per_kv_head, rtp_view q,
+                                             rtp_view k_cache, rtp_view v_cache, rtp_view q16,
+                                             rtp_view k16_cache, float p, float softmax_scale,
+                                             rtp_view o, float* lse, float* thr, int32_t* jtie,
+                                             int32_t* count, float* mass, void* ws,
+                                             size_t ws_bytes, rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  if (shape->Lq != 1) return RTP_ERR_INVALID_ARG;
+  if ((st = check_causal(shape)) != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, k16_per_kv_head, &hm)) != RTP_OK) return st;
+  if (!(p >= 0.f && p <= 1.f)) return RTP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return RTP_ERR_INVALID_ARG;
+  if (hm.G > 16 || (256 % hm.G) != 0) return RTP_ERR_UNSUPPORTED;
+  if (shape->Lk > kMaxKeys) return RTP_ERR_UNSUPPORTED;
+  const bool work = shape->B > 0 && hm.n_ret > 0;
+  if (!work) return RTP_OK;
+  if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(k_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
+  if ((st = check_view(k16_cache, hm.H_k16, kR, true)) != RTP_OK) return st;
+  const DecodeWs L = decode_ws_layout(shape, hm);
+  if (ws == nullptr || ws_bytes < L.total) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int N = (int)(shape->q_pos0 + 1);  // keys 0..P
+  const int nc = (N + kDecChunk - 1) / kDecChunk;
+  const int groups = shape->B * hm.n_rkv;
+  auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+
+  // the row histograms and flags accumulate with atomics: clear them
+  if (cudaMemsetAsync(at(L.hist_m), 0, L.rowsel - L.hist_m, s) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  {  // 1. scores + histograms
+    ScoreParams sp;
+    sp.q16 = static_cast<const uint16_t*>(q16.ptr);
+    sp.q16_sb = q16.stride_b;
+    sp.k16 = static_cast<const uint16_t*>(k16_cache.ptr);
+    sp.k16_sb = k16_cache.stride_b;
+    sp.k16_sl = k16_cache.stride_l;
+    sp.scores = static_cast<float*>(at(L.scores));
+    sp.hist_m = static_cast<unsigned long long*>(at(L.hist_m));
+    sp.hist_c = static_cast<uint32_t*>(at(L.hist_c));
+    sp.flags = static_cast<uint32_t*>(at(L.flags));
+    sp.ncand = static_cast<uint32_t*>(at(L.ncand));
+    sp.counter = static_cast<uint32_t*>(at(L.counter));
+    sp.mcount = static_cast<uint32_t*>(at(L.mcount));
+    sp.N = N;
+    sp.Lk_pad = L.Lk_pad;
+    sp.n_ret = hm.n_ret;
+    sp.n_rkv = hm.n_rkv;
+    sp.G = hm.G;
+    sp.per_kv = k16_per_kv_head;
+    const size_t smem =
+        (size_t)hm.G * (kDecChunk + 4) * 4 + (size_t)hm.G * kDecWin * 8 + (size_t)hm.G * 4 + 16;
+    if (cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    TraceScope tr("dec_score", s);
+    dec_score_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(sp);
+    if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+  }
+  {  // 2. per-row merge
+    MergeParams mp;
+    mp.hist_m = static_cast<const unsigned long long*>(at(L.hist_m));
+    mp.hist_c = static_cast<const uint32_t*>(at(L.hist_c));
+    mp.flags = static_cast<const uint32_t*>(at(L.flags));
+    mp.rowsel = static_cast<RowSel*>(at(L.rowsel));
+    mp.p = p;
+    TraceScope tr("dec_merge", s);
+    dec_merge_kernel<<<L.rows, kThreads, 0, s>>>(mp);
+    if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+  }
+  {  // 3. collect, compact, exact cut
+    CollectParams cp;
+    cp.scores = static_cast<const float*>(at(L.scores));
+    cp.rowsel = static_cast<const RowSel*>(at(L.rowsel));
+    cp.cand = static_cast<unsigned long long*>(at(L.cand));
+    cp.ncand = static_cast<uint32_t*>(at(L.ncand));
+    cp.list = static_cast<uint2*>(at(L.list));
+    cp.lcount = static_cast<int32_t*>(at(L.lcount));
+    cp.loff = static_cast<int32_t*>(at(L.loff));
+    cp.counter = static_cast<uint32_t*>(at(L.counter));
+    cp.rowres = static_cast<RowRes*>(at(L.rowres));
+    cp.thr = thr;
+    cp.jtie = jtie;
+    cp.count = count;
+    cp.mass = mass;
+    cp.status = static_cast<DevStatus*>(ws);
+    cp.N = N;
+    cp.Lk_pad = L.Lk_pad;
+    cp.nc = nc;
+    cp.n_ret = hm.n_ret;
+    cp.n_rkv = hm.n_rkv;
+    cp.G = hm.G;
+    cp.p = p;
+    const size_t smem = sizeof(CollectSmem);
+    if (cudaFuncSetAttribute(dec_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    TraceScope tr("dec_collect", s);
+    dec_collect_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(cp);
+    if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+  }
+  // 4. attention over the kept union
+  DecodeLists dl;
+  dl.list = static_cast<const uint2*>(at(L.list));
+  dl.loff = static_cast<const int32_t*>(at(L.loff));
+  dl.scores = static_cast<const float*>(at(L.scores));
+  dl.rowres = static_cast<const RowRes*>(at(L.rowres));
+  dl.part = static_cast<float*>(at(L.part));
+  dl.mcount = static_cast<uint32_t*>(at(L.mcount));
+  dl.Lk_pad = L.Lk_pad;
+  dl.n_chunks = nc;
+  dl.n_splits = decode_list_splits(groups, nc);
+  if (dl.n_splits > L.n_splits) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  return decode_list_attention(shape, hm, q, k_cache, v_cache, softmax_scale, o, lse, dl, s);
+}

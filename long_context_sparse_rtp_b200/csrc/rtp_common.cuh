@@ -130,6 +130,7 @@ __device__ __forceinline__ float quad_sum(float v) {
 // keeps every top-p decision deterministic.
 __device__ __forceinline__ unsigned long long mass_fixed40(float w) {
   const uint32_t b = __float_as_uint(w);
+  if (b >= 0x3F800000u) return 1ull << 40;  // w >= 1 (or inf / nan): saturate at 1
   const int e = int(b >> 23) & 0xFF;
   if (e == 0) return 0ull;  // zero / subnormal: below 2^-126
   const unsigned long long m = (b & 0x7FFFFFu) | 0x800000u;

@@ -13,10 +13,6 @@
 namespace rtp {
 
 constexpr int kDecChunk = 1024;    // tokens per decode scoring / compaction chunk
-constexpr int kDecHistChunk = 4096;// scores per decode histogram CTA
-constexpr int kDecBins = 256;      // level-0 histogram bins (decode)
-constexpr int kDecCap = 4096;      // candidates a decode row resolves in one sort
-constexpr int kDecChunksPerSplit = 2;
 constexpr int kMaxKeys = 1 << 21;  // composite (score, index) keys use 21 index bits
 
 // Kernel trace: events around each launch while rtp_trace_enable(1) is in force.
@@ -93,12 +89,6 @@ inline rtp_status make_headmap(const rtp_shape* s, const uint8_t* kv_role, int k
 // ---------------------------------------------------------------- workspaces
 // Every workspace starts with the 256-byte DevStatus block.
 
-struct DecodeWs {   // retrieval decode
-  size_t scores, cmax, hist_m, hist_c, zsum, counter, rowres, cand, list, lcount, part,
-      mcount, total;
-  int n_chunks, n_splits, Lk_pad, rows;
-};
-
 // Per-row decode result kept in the workspace.
 struct RowRes {
   float t;
@@ -107,14 +97,49 @@ struct RowRes {
   float mass;
 };
 
+// Retrieval decode: the per-row top-p state the merge kernel leaves for the
+// collection kernel.  Masses are relative to E_top, the upper edge of the row's
+// highest occupied score bin.
+struct RowSel {
+  double T;          // p * Z
+  double above;      // mass of the bins above the crossing bin
+  double scale_b;    // 2^-21 * exp((bstar + 1) / kappa - E_top): fixed21 -> relative mass
+  double Z;
+  int32_t bstar;     // absolute score bin holding the cut
+  int32_t mode;      // 0 normal, 1 keep all (p >= 1), 2 refine over the stored scores
+  uint32_t cnt_above;
+  uint32_t n_in;
+};
+
+constexpr int kDecWin = 256;           // score bins a scoring CTA keeps per head
+constexpr float kDecKappa = 4.0f;      // bins per unit of indexer score
+constexpr int kDecGBins = 2048;        // absolute bins per row: scores in [-256, 256)
+constexpr int kDecGLo = -1024;         // absolute bin of global bin 0
+constexpr int kDecCap = 4096;          // candidates a decode row resolves with one sort
+
+struct DecodeWs {   // retrieval decode
+  size_t scores, hist_m, hist_c, flags, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
+      part, mcount, total;
+  int n_chunks, n_splits, Lk_pad, rows, groups;
+};
+
+inline int decode_list_splits(int groups, int n_chunks) {
+  int want = groups > 0 ? (296 + groups - 1) / groups : 1;
+  if (want > 4 * n_chunks) want = 4 * n_chunks;  // at least ~256 tokens of list per split
+  return want < 1 ? 1 : want;
+}
+
 inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
   DecodeWs w;
   const int64_t N = s->Lk;
   w.n_chunks = (int)((N + kDecChunk - 1) / kDecChunk);
+  if (w.n_chunks < 1) w.n_chunks = 1;
   w.Lk_pad = w.n_chunks * kDecChunk;
-  w.n_splits = (w.n_chunks + kDecChunksPerSplit - 1) / kDecChunksPerSplit;
   w.rows = s->B * hm.n_ret;
-  const size_t groups = (size_t)s->B * hm.n_rkv;
+  w.groups = s->B * hm.n_rkv;
+  w.n_splits = decode_list_splits(w.groups, w.n_chunks);  // largest count any N <= Lk asks for
+  const size_t groups = (size_t)w.groups;
+  const size_t nc = (size_t)w.n_chunks;
   size_t off = kStatusBytes;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -122,35 +147,62 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
     return o;
   };
   w.scores = take((size_t)w.rows * w.Lk_pad * 4);
-  w.cmax = take((size_t)w.rows * w.n_chunks * 4);
-  w.hist_m = take((size_t)w.rows * kDecBins * 8);
-  w.hist_c = take((size_t)w.rows * kDecBins * 4);
-  w.zsum = take((size_t)w.rows * 8);
-  w.counter = take((size_t)w.rows * 4 + groups * 4);
+  w.hist_m = take((size_t)w.rows * kDecGBins * 8);   // hist_m, hist_c, flags are one
+  w.hist_c = take((size_t)w.rows * kDecGBins * 4);   // contiguous range (cleared per call)
+  w.flags = take((size_t)w.rows * 4);
+  w.rowsel = take((size_t)w.rows * sizeof(RowSel));
   w.rowres = take((size_t)w.rows * sizeof(RowRes));
-  w.cand = 0;
+  w.cand = take((size_t)w.rows * kDecCap * 8);
+  w.ncand = take((size_t)w.rows * 4);
+  w.counter = take(groups * 4);
   w.list = take(groups * w.Lk_pad * 8);
-  w.lcount = take(groups * w.n_chunks * 4);
+  w.lcount = take(groups * nc * 4);
+  w.loff = take(groups * (nc + 1) * 4);
   w.part = take(groups * w.n_splits * 16 * (2 + kD) * 4);
   w.mcount = take(groups * 4);
   w.total = off;
   return w;
 }
 
-struct AttnDecodeWs {  // local / dense decode (range mode)
-  size_t part, mcount, total;
-  int n_splits;
+// Buffers the gathered decode attention reads (decode.cu).
+struct DecodeLists {
+  const uint2* list;       // [groups][Lk_pad], chunk c's entries at c * kDecChunk
+  const int32_t* loff;     // [groups][n_chunks + 1] exclusive prefix of the chunk counts
+  const float* scores;
+  const RowRes* rowres;
+  float* part;
+  uint32_t* mcount;
+  int Lk_pad, n_chunks, n_splits;
 };
 
-constexpr int kRangeKeysPerSplit = 512;
+rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, const rtp_view& q,
+                                 const rtp_view& k, const rtp_view& v, float scale,
+                                 const rtp_view& o, float* lse, const DecodeLists& lists,
+                                 cudaStream_t s);
+
+struct AttnDecodeWs {  // local / dense decode (range mode)
+  size_t part, mcount, total;
+  int n_splits, keys_per_split;
+};
 
 inline AttnDecodeWs range_decode_ws_layout(int64_t n_keys, int groups) {
   AttnDecodeWs w;
-  w.n_splits = (int)((n_keys + kRangeKeysPerSplit - 1) / kRangeKeysPerSplit);
+  // about two CTAs per SM, at least 64 keys per split
+  int64_t want = groups > 0 ? (296 + groups - 1) / groups : 1;
+  const int64_t max_splits = (n_keys + 63) / 64;
+  if (want > max_splits) want = max_splits;
+  if (want < 1) want = 1;
+  int64_t kps = (n_keys + want - 1) / want;
+  kps = (kps + 63) / 64 * 64;
+  if (kps < 64) kps = 64;
+  w.keys_per_split = (int)kps;
+  w.n_splits = (int)((n_keys + kps - 1) / kps);
   if (w.n_splits < 1) w.n_splits = 1;
+  // sized for `want` splits: a workspace sized for an upper bound on the key
+  // count then also fits every smaller key count
   size_t off = kStatusBytes;
   w.part = off;
-  off = align_up(off + (size_t)groups * w.n_splits * 16 * (2 + kD) * 4, 256);
+  off = align_up(off + (size_t)groups * want * 16 * (2 + kD) * 4, 256);
   w.mcount = off;
   off = align_up(off + (size_t)groups * 4, 256);
   w.total = off;

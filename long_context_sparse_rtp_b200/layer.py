@@ -33,19 +33,72 @@ def rtp_layer_prefill(q, k, v, Wq16, Wk16, kv_role, *, p, window, n_sink, scale=
 
 
 def rtp_layer_decode(q, k_new, k_cache, v_cache, k16_cache, Wq16, Wk16, kv_role, *, pos, p,
-                     window, n_sink, scale=None, k16_per_kv_head=0, stream=None):
+                     window, n_sink, scale=None, k16_per_kv_head=0, stream=None, o=None,
+                     lse=None, want_sel=True):
     """One decode token at position `pos` (the caches already hold its k/v row;
     its k16 row is written here).  Returns dict(o, lse, q16, sel)."""
     H = q.shape[2]
     k16_row = k16_cache[:, pos:pos + 1]
     q16, _ = rtp_index_scores(q, k_new, Wq16, Wk16, kv_role, k16=k16_row,
                               k16_per_kv_head=k16_per_kv_head, stream=stream)
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[0], H, 1, dtype=torch.float32, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[0], H, 1, dtype=torch.float32, device=q.device)
     kc, vc = k_cache[:, :pos + 1], v_cache[:, :pos + 1]
     _, _, sel = rtp_sparse_attn_decode(q, kc, vc, q16, k16_cache[:, :pos + 1], kv_role, p,
                                        scale=scale, q_pos0=pos, k16_per_kv_head=k16_per_kv_head,
-                                       o=o, lse=lse, stream=stream)
+                                       o=o, lse=lse, want_sel=want_sel, stream=stream)
     rtp_local_attn(q, kc, vc, kv_role, window=window, n_sink=n_sink, scale=scale, q_pos0=pos,
                    o=o, lse=lse, stream=stream)
     return dict(o=o, lse=lse, q16=q16, sel=sel)
+
+
+class DecodeGraph:
+    """One decode step of the layer captured once in a CUDA graph and replayed.
+
+    The step (indexer projection of the new token with its k16 append, exact
+    top-p and gathered attention on the retrieval heads, sink+window attention on
+    the local heads) issues several kernels; replaying them as one graph removes
+    the per-launch host cost.  Inputs live in fixed device buffers: `q`
+    [B, 1, H, 128] and row `pos` of the k/v caches; outputs in `o`, `lse`.
+    """
+
+    def __init__(self, k_cache, v_cache, k16_cache, Wq16, Wk16, kv_role, *, H, pos, p, window,
+                 n_sink, scale=None, k16_per_kv_head=0, trace=False):
+        B = k_cache.shape[0]
+        dev = k_cache.device
+        self.k_cache, self.v_cache, self.pos = k_cache, v_cache, pos
+        self.q = torch.zeros(B, 1, H, 128, dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(B, H, 1, dtype=torch.float32, device=dev)
+        args = (self.q, k_cache[:, pos:pos + 1], k_cache, v_cache, k16_cache, Wq16, Wk16, kv_role)
+        kw = dict(pos=pos, p=p, window=window, n_sink=n_sink, scale=scale,
+                  k16_per_kv_head=k16_per_kv_head, o=self.o, lse=self.lse, want_sel=False)
+        self._call = lambda: rtp_layer_decode(*args, **kw)
+        self._call()                      # eager once: workspaces and buffers exist
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        if trace:  # the library's kernel-trace events become nodes of this graph
+            from .rtp import lib
+            lib().rtp_trace_reset()
+            lib().rtp_trace_enable(1)
+        try:
+            with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+                self._call()
+        finally:
+            if trace:
+                lib().rtp_trace_enable(0)
+
+    def replay(self):
+        self.graph.replay()
+
+    def step(self, q_host, k_host, v_host, o_host):
+        """Copy the new token in from (pinned) host buffers, run, copy o out."""
+        pos = self.pos
+        self.q.copy_(q_host, non_blocking=True)
+        self.k_cache[:, pos:pos + 1].copy_(k_host, non_blocking=True)
+        self.v_cache[:, pos:pos + 1].copy_(v_host, non_blocking=True)
+        self.graph.replay()
+        o_host.copy_(self.o, non_blocking=True)
+        return o_host

@@ -121,10 +121,11 @@ _ws_cache: dict = {}
 
 def workspace(op: int, shape: Shape, role, k16_per_kv: int, device, stream=None) -> torch.Tensor:
     """A zero-initialised workspace of the size the library asks for, cached per
-    (device, stream, op); the kernels leave it clean for the next call."""
+    (device, op) and grown on demand.  The binding's convenience functions share
+    it, so they must not run concurrently on several streams; callers that need
+    that pass their own workspace through the C ABI."""
     need = lib().rtp_workspace_size(op, ctypes.byref(shape), role, k16_per_kv)
-    s = torch.cuda.current_stream(device) if stream is None else stream
-    key = (str(device), s.cuda_stream, op)
+    key = (str(torch.device(device)), op)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(need, dtype=torch.uint8, device=device)

@@ -174,3 +174,27 @@ def test_repeatable_bitwise():
     assert torch.equal(r1[2], r2[2]) and torch.equal(r1[3], r2[3])
     for key in ("thr", "jtie", "count", "mass"):
         assert torch.equal(r1[4][key], r2[4][key]), key
+
+
+def test_decode_graph_matches_eager():
+    """DecodeGraph replays the same kernels as the eager layer call."""
+    from long_context_sparse_rtp_b200 import DecodeGraph
+    w = W["decode_128k_b8"]
+    d = synth.make_inputs(w, "cuda", L=5000, B=2)
+    q, k, v, Wq, Wk, role = (d[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
+    _, k16 = rtp_index_scores(q, k, Wq, Wk, role)
+    eager = rtp_layer_decode(q, k[:, 4999:], k, v, k16.clone(), Wq, Wk, role, pos=4999, p=w.p,
+                             window=w.window, n_sink=w.n_sink)
+    g = DecodeGraph(k, v, k16, Wq, Wk, role, H=w.H, pos=4999, p=w.p, window=w.window,
+                    n_sink=w.n_sink)
+    g.q.copy_(q)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(g.o, eager["o"])
+        assert torch.equal(g.lse, eager["lse"])
+    hq = q.cpu().pin_memory()
+    ho = torch.empty_like(hq).pin_memory()
+    g.step(hq, k[:, 4999:].cpu().pin_memory(), v[:, 4999:].cpu().pin_memory(), ho)
+    torch.cuda.synchronize()
+    assert torch.equal(ho, eager["o"].cpu())

@@ -28,11 +28,11 @@ def _args(inp, q_pos0):
 
 
 def test_rejects_shapes_beyond_the_scratch_array():
-    """Host-side check, nothing enqueued: 64 x 3 local kv heads x 8192-key window
-    needs ~25 MiB of partials, more than the 8 MiB array."""
+    """Host-side check, nothing enqueued: 400 batch entries x 3 local kv heads
+    need at least one 8320-byte partial each, ~10 MB, more than the 8 MiB array."""
     build.build()
     L = rtp.lib()
-    shape = rtp.Shape(64, 1, 9000, 32, 4, 128, 8999)
+    shape = rtp.Shape(400, 1, 9000, 32, 4, 128, 8999)
     role = (ctypes.c_uint8 * 4)(1, 0, 0, 0)
     v = rtp.View(ctypes.c_void_p(0x10000), 9000 * 4 * 128, 4 * 128)
     vq = rtp.View(ctypes.c_void_p(0x10000), 32 * 128, 32 * 128)

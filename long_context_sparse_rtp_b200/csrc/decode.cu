@@ -59,7 +59,8 @@ struct DecAttnParams {
 
 constexpr int kDecThreads = 128;
 constexpr int kTile = 64;
-constexpr int kMaxSplits = 512;
+constexpr int kMaxSplits = kDecMaxSplits;  // the merge keeps 3 x 256 x 16 floats in K/V smem
+constexpr int kRound = 512;  // list entries a CTA resolves into shared memory at once
 
 struct DecSmem {
   uint16_t q[16][kD];
@@ -69,6 +70,8 @@ struct DecSmem {
   float wm[4][16], wl[4][16];
   float t[16];
   int jt[16];
+  int etok[kRound];        // list mode: resolved tokens and head masks of this round
+  uint32_t emask[kRound];
   float lsum[16], mmax[16];
   int is_last;
   int loffs[1];  // list mode: n_chunks + 1 entries (dynamic tail)
@@ -116,7 +119,6 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
     e_end = min(p.n_keys, e_begin + p.keys_per_split);
     n_entries = (int)max((int64_t)0, e_end - e_begin);
   }
-  const int n_tiles = (n_entries + kTile - 1) / kTile;
   const uint16_t* kb = p.k + b * p.k_sb + (int64_t)kvh * kD;
   const uint16_t* vb = p.v + b * p.v_sb + (int64_t)kvh * kD;
 
@@ -128,10 +130,11 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
     }
     __syncthreads();
   }
-  // entry e (0..n_entries) -> (token, head mask)
-  auto entry = [&](int e, uint32_t& msk) -> int64_t {
-    if (LIST) {
-      const int ge = (int)(e_begin + e);
+  // list mode: entries are resolved a round at a time, all loads in flight together
+  auto resolve_round = [&](int r0, int nr) {
+#pragma unroll 4
+    for (int e = tid; e < nr; e += kDecThreads) {
+      const int ge = (int)(e_begin + r0 + e);
       int lo = 0, hi = p.n_chunks - 1;  // last chunk c with loffs[c] <= ge
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -146,32 +149,41 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
         const float sc = p.scores[(int64_t)(b * p.n_ret + grp * G + hh) * p.Lk_pad + x.x];
         if (sc > sm.t[hh] || (sc == sm.t[hh] && (int)x.x <= sm.jt[hh])) keep |= 1u << hh;
       }
-      msk = keep;
-      return (int64_t)x.x;
-    } else {
-      const int64_t ve = e_begin + e;
-      msk = allmask;
-      return ve < p.n_sink_eff ? ve : p.win_lo + (ve - p.n_sink_eff);
+      sm.etok[e] = (int)x.x;
+      sm.emask[e] = keep;
     }
   };
+  // range mode: entry e -> key
+  auto range_key = [&](int e) -> int64_t {
+    const int64_t ve = e_begin + e;
+    return ve < p.n_sink_eff ? ve : p.win_lo + (ve - p.n_sink_eff);
+  };
+  int round0 = 0, n_round = n_entries;  // entries [round0, round0 + n_round) of this pass
   auto load_tile = [&](int it, int buf) {
     // 64 rows x 16 chunks for K and for V: 16 cp.async per thread
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = u * kDecThreads + tid;
       const int r = c >> 4, ch = c & 15;
-      const int e = it * kTile + r;
-      const bool ok = e < n_entries;
+      const int e = it * kTile + r;  // within the round
+      const bool ok = e < n_round;
+      int64_t j = 0;
       uint32_t msk = 0;
-      const int64_t j = ok ? entry(e, msk) : 0;
+      if (ok) {
+        if (LIST) {
+          j = sm.etok[e];
+          msk = sm.emask[e];
+        } else {
+          j = range_key(round0 + e);
+          msk = allmask;
+        }
+      }
       cp_async16(dswz(sm.k[buf], r, ch), kb + j * p.k_sl + ch * 8, ok);
       cp_async16(dswz(sm.v[buf], r, ch), vb + j * p.v_sl + ch * 8, ok);
       if (ch == 0) sm.mask[buf][r] = ok ? msk : 0u;
     }
   };
 
-  if (n_tiles > 0) load_tile(0, 0);
-  cp_async_commit();
   __syncthreads();
   uint32_t qa[8][4];
 #pragma unroll
@@ -187,6 +199,16 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
   float mrow[2] = {-INFINITY, -INFINITY};
   float lrow[2] = {0.f, 0.f};
 
+  for (round0 = 0; round0 < max(n_entries, 1); round0 += (LIST ? kRound : max(n_entries, 1))) {
+  n_round = LIST ? min(kRound, n_entries - round0) : n_entries;
+  if (LIST) {
+    __syncthreads();  // the previous round's entries are no longer read
+    resolve_round(round0, n_round);
+    __syncthreads();
+  }
+  const int n_tiles = (n_round + kTile - 1) / kTile;
+  if (n_tiles > 0) load_tile(0, 0);
+  cp_async_commit();
   for (int it = 0; it < n_tiles; ++it) {
     const int buf = it & 1;
     if (it + 1 < n_tiles) {
@@ -267,6 +289,8 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
     __syncthreads();
   }
 
+  }  // rounds
+
   // ---- merge the 4 warps (each saw a quarter of every tile); the K/V staging
   // buffers are free now and hold the warps' partial outputs
   float (*wo)[16][kD] = reinterpret_cast<float (*)[16][kD]>(&sm.k[0][0][0]);
@@ -313,40 +337,66 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
   if (!sm.is_last) return;
   __threadfence();
 
-  // ---- last CTA of the group: merge splits in a fixed order
+  // ---- last CTA of the group: merge splits in a fixed order.  Every global load
+  // below is independent of the others, so they are all issued before use.
   const float* pg = p.part + (int64_t)gg * p.n_splits * 16 * (2 + kD);
   const int ns = min(p.n_splits, kMaxSplits);
-  float (*fsplit)[16] = reinterpret_cast<float (*)[16]>(&sm.k[0][0][0]);
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, __ldcg(pg + ((int64_t)sp * 16 + tid) * (2 + kD)));
-    sm.mmax[tid] = M;
-  }
-  __syncthreads();
+  float* pm = reinterpret_cast<float*>(&sm.k[0][0][0]);  // [ns][16] split maxima
+  float* pl = pm + kMaxSplits * 16;                      // [ns][16] split sums
+  float* fs = pl + kMaxSplits * 16;                      // [ns][16] split weights
+  static_assert(3 * kMaxSplits * 16 * sizeof(float) <= 2 * kTile * kD * 2 * sizeof(uint16_t),
+                "merge scratch must fit in the K/V staging buffers");
   for (int x = tid; x < ns * G; x += kDecThreads) {
     const int sp = x / G, r = x % G;
-    const float ms = __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD));
-    fsplit[sp][r] = (ms == -INFINITY) ? 0.f : exp2f(ms - sm.mmax[r]);
+    pm[sp * 16 + r] = __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD));
+    pl[sp * 16 + r] = __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD) + 1);
   }
   __syncthreads();
   if (tid < G) {
+    float M = -INFINITY;
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, pm[sp * 16 + tid]);
     float l = 0.f;
-    for (int sp = 0; sp < ns; ++sp)
-      l += fsplit[sp][tid] * __ldcg(pg + ((int64_t)sp * 16 + tid) * (2 + kD) + 1);
+    for (int sp = 0; sp < ns; ++sp) {
+      const float ms = pm[sp * 16 + tid];
+      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      fs[sp * 16 + tid] = f;
+      l += f * pl[sp * 16 + tid];
+    }
+    sm.mmax[tid] = M;
     sm.lsum[tid] = l;
   }
   __syncthreads();
-  for (int x = tid; x < G * kD; x += kDecThreads) {
-    const int r = x / kD, d = x % kD;
-    float o = 0.f;
-#pragma unroll 8
-    for (int sp = 0; sp < ns; ++sp)
-      o += fsplit[sp][r] * __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD) + 2 + d);
-    const float l = sm.lsum[r];
-    const int h = kvh * G + r;
-    p.o[b * p.o_sb + (int64_t)h * kD + d] = f32_to_bf16_bits(l > 0.f ? o / l : 0.f);
-    if (d == 0 && p.lse != nullptr)
-      p.lse[b * p.lse_sb + h] = l > 0.f ? (sm.mmax[r] + log2f(l)) * kLn2 : -INFINITY;
+  {
+    const int d = tid;  // one dimension per thread, every head
+    float acc[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+    int sp = 0;
+    for (; sp + 4 <= ns; sp += 4) {
+      float v[4][16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int r = 0; r < 16; ++r)
+          v[u][r] = r < G ? __ldcg(pg + ((int64_t)(sp + u) * 16 + r) * (2 + kD) + 2 + d) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) acc[r] += fs[(sp + u) * 16 + r] * v[u][r];
+    }
+    for (; sp < ns; ++sp)
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (r < G) acc[r] += fs[sp * 16 + r] * __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD) + 2 + d);
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (r >= G) break;
+      const float l = sm.lsum[r];
+      const int h = kvh * G + r;
+      p.o[b * p.o_sb + (int64_t)h * kD + d] = f32_to_bf16_bits(l > 0.f ? acc[r] / l : 0.f);
+      if (d == 0 && p.lse != nullptr)
+        p.lse[b * p.lse_sb + h] = l > 0.f ? (sm.mmax[r] + log2f(l)) * kLn2 : -INFINITY;
+    }
   }
   if (tid == 0) p.mcount[gg] = 0;
 }

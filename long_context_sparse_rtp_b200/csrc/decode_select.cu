@@ -628,6 +628,120 @@ __device__ void refine_row(CollectSmem& sm, const CollectParams& p, const float*
   out.mass = (float)((double)(acc_above + cum) / (double)Z);
 }
 
+// A normal row whose crossing bin holds more than kWarpCap keys: radix levels
+// over the candidates' composite keys (in shared memory) narrow the crossing down
+// to a few keys, which warp 0 sorts and walks.  Block-wide.
+__device__ RowRes resolve_many(CollectSmem& sm, const CollectParams& p, int row, RowSel rs,
+                               int n) {
+  const int tid = threadIdx.x;
+  for (int a = tid; a < n; a += kThreads) sm.cand[a] = __ldcg(&p.cand[(int64_t)row * kDecCap + a]);
+  __syncthreads();
+  // common prefix of every candidate key
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  for (int a = tid; a < n; a += kThreads) {
+    kmin = min(kmin, sm.cand[a]);
+    kmax = max(kmax, sm.cand[a]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if ((tid & 31) == 0) {
+    sm.tsum[tid >> 5] = kmin;
+    sm.tsum[8 + (tid >> 5)] = kmax;
+  }
+  __syncthreads();
+  kmin = ~0ull;
+  kmax = 0ull;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    kmin = min(kmin, sm.tsum[w]);
+    kmax = max(kmax, sm.tsum[8 + w]);
+  }
+  __syncthreads();
+  int pb = (kmin == kmax) ? kKeyBits : (__clzll(kmin ^ kmax) - (64 - kKeyBits));
+  unsigned long long prefix = pb > 0 ? (kmax >> (kKeyBits - pb)) : 0ull;
+  unsigned long long base = 0;  // fixed21 mass of candidates above the current range
+  uint32_t cbase = 0;
+  uint32_t n_in = (uint32_t)n;
+  auto member = [&](unsigned long long ck) {
+    return pb == 0 || (ck >> (kKeyBits - pb)) == prefix;
+  };
+  for (int lvl = 0; lvl < 8 && n_in > (uint32_t)kWarpCap && pb < kKeyBits; ++lvl) {
+    const int w = min(8, kKeyBits - pb);
+    for (int bb = tid; bb < 256; bb += kThreads) {
+      sm.hm[bb] = 0;
+      sm.hc[bb] = 0;
+    }
+    __syncthreads();
+    for (int a = tid; a < n; a += kThreads) {
+      const unsigned long long ck = sm.cand[a];
+      if (!member(ck)) continue;
+      const int digit = (int)((ck >> (kKeyBits - pb - w)) & ((1ull << w) - 1));
+      atomicAdd(&sm.hm[(1 << w) - 1 - digit],
+                (unsigned long long)fixed21(wbin(key_score((uint32_t)(ck >> kIdxBits)), rs.bstar)));
+      atomicAdd(&sm.hc[(1 << w) - 1 - digit], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned long long a = base;
+      uint32_t c = cbase, nin = 0;
+      int last = -1, k = -1;
+      for (int bb = 0; bb < (1 << w); ++bb) {
+        if (sm.hc[bb] == 0) continue;
+        last = bb;
+        if (rs.above + (double)(a + sm.hm[bb]) * rs.scale_b >= rs.T) {
+          k = bb;
+          nin = sm.hc[bb];
+          break;
+        }
+        a += sm.hm[bb];
+        c += sm.hc[bb];
+      }
+      if (k < 0) {
+        k = last;
+        a -= sm.hm[last];
+        c -= sm.hc[last];
+        nin = sm.hc[last];
+      }
+      sm.s_acc = a;
+      sm.s_cnt = c;
+      sm.s_nin = nin;
+      sm.s_k = (1 << w) - 1 - k;
+    }
+    __syncthreads();
+    base = sm.s_acc;
+    cbase = sm.s_cnt;
+    n_in = sm.s_nin;
+    prefix = (prefix << w) | (unsigned long long)sm.s_k;
+    pb += w;
+    __syncthreads();
+  }
+  // the remaining candidates -> warp 0
+  if (tid == 0) sm.ncand = 0;
+  __syncthreads();
+  for (int a = tid; a < n; a += kThreads) {
+    const unsigned long long ck = sm.cand[a];
+    if (!member(ck)) continue;
+    const int idx = atomicAdd(&sm.ncand, 1);
+    if (idx < kWarpCap) sm.wc[0][idx] = ck;
+  }
+  __syncthreads();
+  RowRes rr;
+  if (tid < 32) {
+    const int m = min(sm.ncand, kWarpCap);
+    if (sm.ncand > kWarpCap && tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 33);
+    RowSel r2 = rs;
+    r2.above = rs.above + (double)base * rs.scale_b;
+    r2.cnt_above = rs.cnt_above + cbase;
+    sort_desc_warp(sm.wc[0], m);
+    rr = warp_walk(sm.wc[0], m, r2);
+    // the walk's mass counts only the narrowed keys; add the candidates above them
+  }
+  __syncthreads();
+  return rr;
+}
+
 __device__ void write_result(const CollectParams& p, int row, const RowRes& rr) {
   p.rowres[row] = rr;
   if (p.thr) p.thr[row] = rr.t;
@@ -777,24 +891,7 @@ __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectPara
     RowRes rr;
     const int n = (int)min(__ldcg(&p.ncand[row]), (uint32_t)kDecCap);
     if (rs.mode == 0 && n > 0) {
-      for (int a = tid; a < n; a += kThreads)
-        sm.cand[a] = __ldcg(&p.cand[(int64_t)row * kDecCap + a]);
-      __syncthreads();
-      sort_desc_block(sm.cand, n);
-      unsigned long long cum = 0;
-      const int bst = rs.bstar;
-      const int cut = walk_cut(
-          sm, n,
-          [&](int a) {
-            return (unsigned long long)fixed21(
-                wbin(key_score((uint32_t)(sm.cand[a] >> kIdxBits)), bst));
-          },
-          rs.above, rs.scale_b, rs.T, cum);
-      const unsigned long long ck = sm.cand[cut];
-      rr.t = key_score((uint32_t)(ck >> kIdxBits));
-      rr.jtie = (int32_t)(kIdxMask - (ck & kIdxMask));
-      rr.count = (int32_t)(rs.cnt_above + cut + 1);
-      rr.mass = (float)((rs.above + (double)cum * rs.scale_b) / rs.Z);
+      rr = resolve_many(sm, p, row, rs, n);
     } else {
       refine_row(sm, p, p.scores + (int64_t)row * p.Lk_pad, rr);
     }

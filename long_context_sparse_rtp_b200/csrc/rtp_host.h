@@ -116,6 +116,7 @@ constexpr float kDecKappa = 4.0f;      // bins per unit of indexer score
 constexpr int kDecGBins = 2048;        // absolute bins per row: scores in [-256, 256)
 constexpr int kDecGLo = -1024;         // absolute bin of global bin 0
 constexpr int kDecCap = 4096;          // candidates a decode row resolves with one sort
+constexpr int kDecMaxSplits = 256;     // split-KV partials per (batch, kv head) in decode
 
 struct DecodeWs {   // retrieval decode
   size_t scores, hist_m, hist_c, flags, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
@@ -126,6 +127,7 @@ struct DecodeWs {   // retrieval decode
 inline int decode_list_splits(int groups, int n_chunks) {
   int want = groups > 0 ? (296 + groups - 1) / groups : 1;
   if (want > 4 * n_chunks) want = 4 * n_chunks;  // at least ~256 tokens of list per split
+  if (want > kDecMaxSplits) want = kDecMaxSplits;
   return want < 1 ? 1 : want;
 }
 
@@ -191,6 +193,7 @@ inline AttnDecodeWs range_decode_ws_layout(int64_t n_keys, int groups) {
   int64_t want = groups > 0 ? (296 + groups - 1) / groups : 1;
   const int64_t max_splits = (n_keys + 63) / 64;
   if (want > max_splits) want = max_splits;
+  if (want > kDecMaxSplits) want = kDecMaxSplits;
   if (want < 1) want = 1;
   int64_t kps = (n_keys + want - 1) / want;
   kps = (kps + 63) / 64 * 64;

@@ -38,20 +38,37 @@ def rtp_layer_decode(q, k_new, k_cache, v_cache, k16_cache, Wq16, Wk16, kv_role,
     """One decode token at position `pos` (the caches already hold its k/v row;
     its k16 row is written here).  Returns dict(o, lse, q16, sel)."""
     H = q.shape[2]
-    k16_row = k16_cache[:, pos:pos + 1]
-    q16, _ = rtp_index_scores(q, k_new, Wq16, Wk16, kv_role, k16=k16_row,
-                              k16_per_kv_head=k16_per_kv_head, stream=stream)
     if o is None:
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(q.shape[0], H, 1, dtype=torch.float32, device=q.device)
+    main = torch.cuda.current_stream(q.device) if stream is None else stream
+    # the local heads depend on nothing the retrieval heads compute: side stream
+    side = _side_stream(q.device)
+    side.wait_stream(main)
     kc, vc = k_cache[:, :pos + 1], v_cache[:, :pos + 1]
+    rtp_local_attn(q, kc, vc, kv_role, window=window, n_sink=n_sink, scale=scale, q_pos0=pos,
+                   o=o, lse=lse, stream=side)
+    k16_row = k16_cache[:, pos:pos + 1]
+    q16, _ = rtp_index_scores(q, k_new, Wq16, Wk16, kv_role, k16=k16_row,
+                              k16_per_kv_head=k16_per_kv_head, stream=stream)
     _, _, sel = rtp_sparse_attn_decode(q, kc, vc, q16, k16_cache[:, :pos + 1], kv_role, p,
                                        scale=scale, q_pos0=pos, k16_per_kv_head=k16_per_kv_head,
                                        o=o, lse=lse, want_sel=want_sel, stream=stream)
-    rtp_local_attn(q, kc, vc, kv_role, window=window, n_sink=n_sink, scale=scale, q_pos0=pos,
-                   o=o, lse=lse, stream=stream)
+    main.wait_stream(side)
     return dict(o=o, lse=lse, q16=q16, sel=sel)
+
+
+_side_streams: dict = {}
+
+
+def _side_stream(device):
+    key = str(torch.device(device))
+    s = _side_streams.get(key)
+    if s is None:
+        s = torch.cuda.Stream(device=device)
+        _side_streams[key] = s
+    return s
 
 
 class DecodeGraph:

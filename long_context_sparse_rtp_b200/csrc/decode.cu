@@ -46,7 +46,7 @@ struct DecAttnParams {
   // list mode: per kv group, per chunk of kDecChunk tokens, an ordered list of
   // {token, kept-head bits | candidate-head bits << 16}; candidate bits are
   // settled here with the exact predicate on the stored indexer score.
-  const uint2* list; const int32_t* loff; int Lk_pad, n_chunks;
+  const uint2* list; const int32_t* lcount; int Lk_pad, n_chunks;
   const float* scores;                    // [rows][Lk_pad]
   const RowRes* rowres;                   // [rows]: t, jtie of each retrieval row
   int n_ret;
@@ -74,6 +74,7 @@ struct DecSmem {
   uint32_t emask[kRound];
   float lsum[16], mmax[16];
   int is_last;
+  int wsc[kDecThreads / 32];
   int loffs[1];  // list mode: n_chunks + 1 entries (dynamic tail)
 };
 
@@ -107,8 +108,39 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
   int64_t e_begin = 0, e_end = 0;  // range mode: virtual key index range
   int n_entries = 0;
   if (LIST) {  // an equal share of the group's list entries
-    const int32_t* lo = p.loff + (int64_t)gg * (p.n_chunks + 1);
-    for (int c = tid; c <= p.n_chunks; c += kDecThreads) sm.loffs[c] = lo[c];
+    // exclusive prefix of the chunk counts (block scan)
+    const int nc = p.n_chunks;
+    const int32_t* lc = p.lcount + (int64_t)gg * nc;
+    const int per = (nc + kDecThreads - 1) / kDecThreads;  // <= 16 (nc <= 2048)
+    const int c0 = tid * per, c1 = min(nc, c0 + per);
+    int cv[16];
+    int seg = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      cv[i] = (c0 + i < c1) ? lc[c0 + i] : 0;
+      seg += cv[i];
+    }
+    int inc = seg;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) sm.wsc[warp] = inc;
+    __syncthreads();
+    int run = inc - seg;
+    for (int w2 = 0; w2 < warp; ++w2) run += sm.wsc[w2];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (c0 + i < c1) sm.loffs[c0 + i] = run;
+      run += cv[i];
+    }
+    __syncthreads();
+    if (tid == kDecThreads - 1) {
+      int tot = 0;
+      for (int w2 = 0; w2 < kDecThreads / 32; ++w2) tot += sm.wsc[w2];
+      sm.loffs[nc] = tot;
+    }
     __syncthreads();
     const int64_t total = sm.loffs[p.n_chunks];
     e_begin = total * split / p.n_splits;
@@ -469,7 +501,7 @@ rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, cons
   fill_dec_common(prm, shape, q, k, v, o, lse, scale);
   prm.groups = hm.n_rkv;
   prm.list = lists.list;
-  prm.loff = lists.loff;
+  prm.lcount = lists.lcount;
   prm.Lk_pad = lists.Lk_pad;
   prm.n_chunks = lists.n_chunks;
   prm.n_splits = lists.n_splits;

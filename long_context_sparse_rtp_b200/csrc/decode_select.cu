@@ -51,6 +51,12 @@ __device__ __forceinline__ float wbin(float s, int b) {
 __device__ __forceinline__ uint32_t fixed21(float w) {
   return __float2uint_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f));
 }
+// Sub-bin of a key inside its (crossing) bin b: 64 equal slices of [b, b+1)/kappa.
+__device__ __forceinline__ int subbin(float s, int b) {
+  const float frac = __fsub_rn(__fmul_rn(s, kDecKappa), (float)b);
+  const int k = (int)__fmul_rn(frac, (float)kDecSub);
+  return k < 0 ? 0 : (k > kDecSub - 1 ? kDecSub - 1 : k);
+}
 // Mass relative to a reference score m (refinement path).
 __device__ __forceinline__ float wrel(float s, float m) {
   return exp2f(__fmul_rn(__fsub_rn(s, m), kLog2e));
@@ -338,6 +344,8 @@ __global__ void __launch_bounds__(kThreads) dec_merge_kernel(const MergeParams p
 struct CollectParams {
   const float* scores;
   const RowSel* rowsel;
+  unsigned long long* sub_m;  // [rows][kDecSub]: the crossing bin split 64 ways
+  uint32_t* sub_c;
   unsigned long long* cand;  // [rows][kDecCap]
   uint32_t* ncand;
   uint2* list;               // [groups][Lk_pad]
@@ -357,12 +365,11 @@ struct CollectParams {
 struct CollectSmem {
   RowSel rs[16];
   int wsum[kThreads / 32];
-  int is_last;
-  int big[16];                       // rows left for the block-wide paths
-  int nbig;
-  // last CTA
-  unsigned long long wc[kThreads / 32][kWarpCap];  // per-warp candidate sort
-  unsigned long long cand[kDecCap];                // block-wide sort
+};
+
+struct ResolveSmem {
+  unsigned long long wc[kWarpCap];  // warp-sorted candidates
+  unsigned long long cand[kDecCap]; // block-wide candidates
   unsigned long long tsum[kThreads];
   unsigned long long hm[256];
   uint32_t hc[256];
@@ -492,7 +499,7 @@ __device__ RowRes warp_walk(const unsigned long long* a, int n, const RowSel& rs
 
 // Block-wide walk for rows with more than kWarpCap candidates.
 template <class F>
-__device__ int walk_cut(CollectSmem& sm, int n, F&& fmass, double base, double scale, double T,
+__device__ int walk_cut(ResolveSmem& sm, int n, F&& fmass, double base, double scale, double T,
                         unsigned long long& cum_out) {
   const int tid = threadIdx.x;
   const int per = (n + kThreads - 1) / kThreads;
@@ -528,7 +535,7 @@ __device__ int walk_cut(CollectSmem& sm, int n, F&& fmass, double base, double s
 
 // Exact cut of one row by radix refinement over all its stored scores (masses
 // relative to the row max, composite (score, index) keys, 8-bit digits).  One CTA.
-__device__ void refine_row(CollectSmem& sm, const CollectParams& p, const float* srow,
+__device__ void refine_row(ResolveSmem& sm, const CollectParams& p, const float* srow,
                            RowRes& out) {
   const int tid = threadIdx.x;
   const int N = p.N;
@@ -631,7 +638,7 @@ __device__ void refine_row(CollectSmem& sm, const CollectParams& p, const float*
 // A normal row whose crossing bin holds more than kWarpCap keys: radix levels
 // over the candidates' composite keys (in shared memory) narrow the crossing down
 // to a few keys, which warp 0 sorts and walks.  Block-wide.
-__device__ RowRes resolve_many(CollectSmem& sm, const CollectParams& p, int row, RowSel rs,
+__device__ RowRes resolve_many(ResolveSmem& sm, const CollectParams& p, int row, RowSel rs,
                                int n) {
   const int tid = threadIdx.x;
   for (int a = tid; a < n; a += kThreads) sm.cand[a] = __ldcg(&p.cand[(int64_t)row * kDecCap + a]);
@@ -724,7 +731,7 @@ __device__ RowRes resolve_many(CollectSmem& sm, const CollectParams& p, int row,
     const unsigned long long ck = sm.cand[a];
     if (!member(ck)) continue;
     const int idx = atomicAdd(&sm.ncand, 1);
-    if (idx < kWarpCap) sm.wc[0][idx] = ck;
+    if (idx < kWarpCap) sm.wc[idx] = ck;
   }
   __syncthreads();
   RowRes rr;
@@ -734,21 +741,14 @@ __device__ RowRes resolve_many(CollectSmem& sm, const CollectParams& p, int row,
     RowSel r2 = rs;
     r2.above = rs.above + (double)base * rs.scale_b;
     r2.cnt_above = rs.cnt_above + cbase;
-    sort_desc_warp(sm.wc[0], m);
-    rr = warp_walk(sm.wc[0], m, r2);
+    sort_desc_warp(sm.wc, m);
+    rr = warp_walk(sm.wc, m, r2);
     // the walk's mass counts only the narrowed keys; add the candidates above them
   }
   __syncthreads();
   return rr;
 }
 
-__device__ void write_result(const CollectParams& p, int row, const RowRes& rr) {
-  p.rowres[row] = rr;
-  if (p.thr) p.thr[row] = rr.t;
-  if (p.jtie) p.jtie[row] = rr.jtie;
-  if (p.count) p.count[row] = rr.count;
-  if (p.mass) p.mass[row] = rr.mass;
-}
 
 __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -787,6 +787,10 @@ __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectPara
         const uint32_t idx = atomicAdd(&p.ncand[row0 + h], 1u);
         if (idx < (uint32_t)kDecCap)
           p.cand[(int64_t)(row0 + h) * kDecCap + idx] = comp_key(vs[e], j);
+        const int sb = subbin(vs[e], rs.bstar);
+        atomicAdd(&p.sub_m[(int64_t)(row0 + h) * kDecSub + sb],
+                  (unsigned long long)fixed21(wbin(vs[e], rs.bstar)));
+        atomicAdd(&p.sub_c[(int64_t)(row0 + h) * kDecSub + sb], 1u);
       }
     }
   }
@@ -814,91 +818,107 @@ __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectPara
     for (int w = 0; w < kThreads / 32; ++w) tot += sm.wsum[w];
     p.lcount[(int64_t)grp * p.nc + chunk] = tot;
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) sm.is_last = (atomicAdd(&p.counter[grp], 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!sm.is_last) return;
-  __threadfence();
+}
 
-  // ---- last CTA of the group
-  // list offsets: exclusive prefix of the chunk counts
-  {
-    const int nc = p.nc;
-    const int per = (nc + kThreads - 1) / kThreads;
-    const int c0 = tid * per, c1 = min(nc, c0 + per);
-    int segsum = 0;
-    for (int c = c0; c < c1; ++c) segsum += __ldcg(&p.lcount[(int64_t)grp * nc + c]);
-    int inc = segsum;
+// One CTA per retrieval row: the exact cut inside the crossing bin.
+__global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  ResolveSmem& sm = *reinterpret_cast<ResolveSmem*>(smem_raw);
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const RowSel rs = p.rowsel[row];
+  RowRes rr;
+  if (rs.mode == 1) {
+    rr.t = -INFINITY;
+    rr.jtie = p.N - 1;
+    rr.count = p.N;
+    rr.mass = 1.f;
+  } else {
+    const int n = (int)min(p.ncand[row], (uint32_t)kDecCap);
+    // crossing sub-bin (warp 0): sub-bins from the top, masses in fixed21 units
+    if (tid < 32 && rs.mode == 0 && n > 0) {
+      const unsigned long long m0 = p.sub_m[(int64_t)row * kDecSub + (kDecSub - 1 - 2 * lane)];
+      const unsigned long long m1 = p.sub_m[(int64_t)row * kDecSub + (kDecSub - 2 - 2 * lane)];
+      const uint32_t n0 = p.sub_c[(int64_t)row * kDecSub + (kDecSub - 1 - 2 * lane)];
+      const uint32_t n1 = p.sub_c[(int64_t)row * kDecSub + (kDecSub - 2 - 2 * lane)];
+      unsigned long long incl = m0 + m1;
+      uint32_t cincl = n0 + n1;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    __syncthreads();
-    if (lane == 31) sm.wsum[warp] = inc;
-    __syncthreads();
-    int run = inc - segsum;
-    for (int w = 0; w < warp; ++w) run += sm.wsum[w];
-    int32_t* lo = p.loff + (int64_t)grp * (nc + 1);
-    for (int c = c0; c < c1; ++c) {
-      lo[c] = run;
-      run += __ldcg(&p.lcount[(int64_t)grp * nc + c]);
-    }
-    if (tid == kThreads - 1) {
-      int tot = 0;
-      for (int w = 0; w < kThreads / 32; ++w) tot += sm.wsum[w];
-      lo[nc] = tot;
-    }
-  }
-  // rows: one warp each for the common case
-  if (tid == 0) sm.nbig = 0;
-  __syncthreads();
-  for (int h = warp; h < G; h += kThreads / 32) {
-    const RowSel rs = sm.rs[h];
-    const int row = row0 + h;
-    if (rs.mode == 1) {
-      if (lane == 0) {
-        RowRes rr;
-        rr.t = -INFINITY;
-        rr.jtie = p.N - 1;
-        rr.count = p.N;
-        rr.mass = 1.f;
-        write_result(p, row, rr);
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t lo = __shfl_up_sync(0xffffffffu, (uint32_t)incl, o);
+        const uint32_t hi = __shfl_up_sync(0xffffffffu, (uint32_t)(incl >> 32), o);
+        const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, o);
+        if (lane >= o) {
+          incl += ((unsigned long long)hi << 32) | lo;
+          cincl += cy;
+        }
       }
-      continue;
+      unsigned long long a = incl - m0 - m1;
+      uint32_t c = cincl - n0 - n1;
+      int my = 0x7FFFFFFF;
+      unsigned long long my_a = 0;
+      uint32_t my_c = 0, my_n = 0;
+      if (n0 && rs.above + (double)(a + m0) * rs.scale_b >= rs.T) {
+        my = 2 * lane; my_a = a; my_c = c; my_n = n0;
+      } else if (n1 && rs.above + (double)(a + m0 + m1) * rs.scale_b >= rs.T) {
+        my = 2 * lane + 1; my_a = a + m0; my_c = c + n0; my_n = n1;
+      }
+      int cut = my;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cut = min(cut, __shfl_xor_sync(0xffffffffu, cut, o));
+      if (cut == my && my != 0x7FFFFFFF) {
+        sm.s_acc = my_a;
+        sm.s_cnt = my_c;
+        sm.s_nin = my_n;
+        sm.s_k = kDecSub - 1 - cut;  // the sub-bin index
+      }
+      if (cut == 0x7FFFFFFF && lane == 0) sm.s_k = -1;
     }
-    const int n = (int)__ldcg(&p.ncand[row]);
-    if (rs.mode == 2 || n > kWarpCap || n == 0) {
-      if (lane == 0) sm.big[atomicAdd(&sm.nbig, 1)] = h;
-      continue;
-    }
-    unsigned long long* a = sm.wc[warp];
-    for (int i = lane; i < n; i += 32) a[i] = __ldcg(&p.cand[(int64_t)row * kDecCap + i]);
-    __syncwarp();
-    sort_desc_warp(a, n);
-    const RowRes rr = warp_walk(a, n, rs);
-    if (lane == 0) write_result(p, row, rr);
-    __syncwarp();
-  }
-  __syncthreads();
-  // rows left: many candidates (block sort) or refinement over all scores
-  const int nbig = sm.nbig;
-  for (int q = 0; q < nbig; ++q) {
-    const int h = sm.big[q];
-    const RowSel rs = sm.rs[h];
-    const int row = row0 + h;
-    RowRes rr;
-    const int n = (int)min(__ldcg(&p.ncand[row]), (uint32_t)kDecCap);
-    if (rs.mode == 0 && n > 0) {
+    __syncthreads();
+    const int ksub = (rs.mode == 0 && n > 0) ? sm.s_k : -1;
+    if (ksub >= 0 && sm.s_nin <= (uint32_t)kWarpCap) {
+      if (tid < 32) {
+        RowSel r2 = rs;
+        r2.above = rs.above + (double)sm.s_acc * rs.scale_b;
+        r2.cnt_above = rs.cnt_above + sm.s_cnt;
+        // the candidates of the crossing sub-bin, compacted by warp ballots
+        int m = 0;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+          const int i = i0 + lane;
+          unsigned long long ck = 0;
+          bool in = false;
+          if (i < n) {
+            ck = p.cand[(int64_t)row * kDecCap + i];
+            in = subbin(key_score((uint32_t)(ck >> kIdxBits)), rs.bstar) == ksub;
+          }
+          const unsigned ball = __ballot_sync(0xffffffffu, in);
+          if (in) sm.wc[m + __popc(ball & ((1u << lane) - 1u))] = ck;
+          m += __popc(ball);
+        }
+        __syncwarp();
+        sort_desc_warp(sm.wc, m);
+        rr = warp_walk(sm.wc, m, r2);
+      }
+    } else if (rs.mode == 0 && n > 0 && n <= kWarpCap) {
+      if (tid < 32) {
+        for (int i = lane; i < n; i += 32) sm.wc[i] = p.cand[(int64_t)row * kDecCap + i];
+        __syncwarp();
+        sort_desc_warp(sm.wc, n);
+        rr = warp_walk(sm.wc, n, rs);
+      }
+    } else if (rs.mode == 0 && n > 0) {
       rr = resolve_many(sm, p, row, rs, n);
     } else {
       refine_row(sm, p, p.scores + (int64_t)row * p.Lk_pad, rr);
     }
-    if (tid == 0) write_result(p, row, rr);
-    __syncthreads();
   }
-  if (tid == 0) p.counter[grp] = 0u;
+  if (tid == 0) {
+    p.rowres[row] = rr;
+    if (p.thr) p.thr[row] = rr.t;
+    if (p.jtie) p.jtie[row] = rr.jtie;
+    if (p.count) p.count[row] = rr.count;
+    if (p.mass) p.mass[row] = rr.mass;
+  }
 }
 
 }  // namespace
@@ -987,6 +1007,8 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     CollectParams cp;
     cp.scores = static_cast<const float*>(at(L.scores));
     cp.rowsel = static_cast<const RowSel*>(at(L.rowsel));
+    cp.sub_m = static_cast<unsigned long long*>(at(L.sub_m));
+    cp.sub_c = static_cast<uint32_t*>(at(L.sub_c));
     cp.cand = static_cast<unsigned long long*>(at(L.cand));
     cp.ncand = static_cast<uint32_t*>(at(L.ncand));
     cp.list = static_cast<uint2*>(at(L.list));
@@ -1010,14 +1032,23 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     if (cudaFuncSetAttribute(dec_collect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return RTP_ERR_CUDA;
-    TraceScope tr("dec_collect", s);
-    dec_collect_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(cp);
+    {
+      TraceScope tr("dec_collect", s);
+      dec_collect_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(cp);
+      if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+    }
+    const size_t rsmem = sizeof(ResolveSmem);
+    if (cudaFuncSetAttribute(dec_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)rsmem) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    TraceScope tr("dec_resolve", s);
+    dec_resolve_kernel<<<L.rows, kThreads, rsmem, s>>>(cp);
     if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
   }
   // 4. attention over the kept union
   DecodeLists dl;
   dl.list = static_cast<const uint2*>(at(L.list));
-  dl.loff = static_cast<const int32_t*>(at(L.loff));
+  dl.lcount = static_cast<const int32_t*>(at(L.lcount));
   dl.scores = static_cast<const float*>(at(L.scores));
   dl.rowres = static_cast<const RowRes*>(at(L.rowres));
   dl.part = static_cast<float*>(at(L.part));

@@ -6,6 +6,8 @@
 //
 // HBM-bound: each CTA stages 32 input rows (256 B each) and one 128x16 weight
 // in shared memory; 4 threads per row each produce 4 of the 16 outputs.
+#include <algorithm>
+
 #include "rtp_host.h"
 
 namespace rtp {
@@ -14,36 +16,46 @@ namespace {
 constexpr int kProjRows = 32;
 constexpr int kProjThreads = 128;
 
-struct ProjParams {
+struct ProjJob {
   const uint16_t* x;   // [B][L][heads][128]
   int64_t x_sb, x_sl;
   const uint16_t* W;   // [slots][128][16]
   uint16_t* out;       // [B][L][slots][16]
   int64_t o_sb, o_sl;
   int L;
-  int16_t head_of_slot[kMaxHeads];
+  int n_slots;
+};
+
+// Up to two projections (the query rows and the key rows) in one launch:
+// blockIdx.y < job[0].n_slots belongs to job 0, the rest to job 1.
+struct ProjParams {
+  ProjJob job[2];
+  int16_t head_of_slot[2][kMaxHeads];
 };
 
 __global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p) {
   __shared__ float sW[kD][kR];
   __shared__ float sX[kProjRows][kD + 1];
-  const int slot = blockIdx.y;
+  const int jb = blockIdx.y < p.job[0].n_slots ? 0 : 1;
+  const ProjJob& J = p.job[jb];
+  const int slot = blockIdx.y - (jb ? p.job[0].n_slots : 0);
   const int b = blockIdx.z;
   const int row0 = blockIdx.x * kProjRows;
+  if (row0 >= J.L) return;
   const int tid = threadIdx.x;
 
-  const uint16_t* W = p.W + (size_t)slot * kD * kR;
+  const uint16_t* W = J.W + (size_t)slot * kD * kR;
   for (int e = tid; e < kD * kR; e += kProjThreads)
     sW[e / kR][e % kR] = __uint_as_float((uint32_t)W[e] << 16);
 
-  const int head = p.head_of_slot[slot];
+  const int head = p.head_of_slot[jb][slot];
   // 32 rows x 16 chunks of 16 bytes
   for (int c = tid; c < kProjRows * 16; c += kProjThreads) {
     const int r = c / 16, ch = c % 16;
     const int row = row0 + r;
     uint4 v = make_uint4(0, 0, 0, 0);
-    if (row < p.L) {
-      const uint16_t* src = p.x + b * p.x_sb + (int64_t)row * p.x_sl + head * kD + ch * 8;
+    if (row < J.L) {
+      const uint16_t* src = J.x + b * J.x_sb + (int64_t)row * J.x_sl + head * kD + ch * 8;
       v = *reinterpret_cast<const uint4*>(src);
     }
     float* dst = &sX[r][ch * 8];
@@ -67,34 +79,26 @@ __global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p
     acc3 = fmaf(xv, w.w, acc3);
   }
   const int row = row0 + r;
-  if (row < p.L) {
+  if (row < J.L) {
     uint2 o;
     o.x = pack_bf16x2(acc0, acc1);
     o.y = pack_bf16x2(acc2, acc3);
-    uint16_t* dst = p.out + b * p.o_sb + (int64_t)row * p.o_sl + slot * kR + c0;
+    uint16_t* dst = J.out + b * J.o_sb + (int64_t)row * J.o_sl + slot * kR + c0;
     *reinterpret_cast<uint2*>(dst) = o;
   }
 }
 
-rtp_status launch_proj(const rtp_view& x, int L, int B, const void* W, int n_slots,
-                       const int16_t* head_of_slot, const rtp_view& out,
-                       cudaStream_t stream) {
-  if (L == 0 || B == 0 || n_slots == 0) return RTP_OK;
-  ProjParams p;
-  p.x = static_cast<const uint16_t*>(x.ptr);
-  p.x_sb = x.stride_b;
-  p.x_sl = x.stride_l;
-  p.W = static_cast<const uint16_t*>(W);
-  p.out = static_cast<uint16_t*>(out.ptr);
-  p.o_sb = out.stride_b;
-  p.o_sl = out.stride_l;
-  p.L = L;
-  for (int s = 0; s < n_slots; ++s) p.head_of_slot[s] = head_of_slot[s];
-  dim3 grid((L + kProjRows - 1) / kProjRows, n_slots, B);
-  if (grid.z > 65535 || grid.y > 65535) return RTP_ERR_UNSUPPORTED;
-  TraceScope tr("proj16", stream);
-  proj16_kernel<<<grid, kProjThreads, 0, stream>>>(p);
-  return check_cuda(cudaGetLastError());
+void set_job(ProjJob& J, const rtp_view& x, int L, const void* W, int n_slots,
+             const rtp_view& out) {
+  J.x = static_cast<const uint16_t*>(x.ptr);
+  J.x_sb = x.stride_b;
+  J.x_sl = x.stride_l;
+  J.W = static_cast<const uint16_t*>(W);
+  J.out = static_cast<uint16_t*>(out.ptr);
+  J.o_sb = out.stride_b;
+  J.o_sl = out.stride_l;
+  J.L = L;
+  J.n_slots = n_slots;
 }
 
 }  // namespace
@@ -119,15 +123,27 @@ extern "C" rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv
   if (do_q && Wq16 == nullptr) return RTP_ERR_INVALID_ARG;
   if (do_k && Wk16 == nullptr) return RTP_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!do_q && !do_k) return RTP_OK;
+  ProjParams p;
+  memset(&p, 0, sizeof(p));
+  int nj = 0, max_rows = 0;
   if (do_q) {
-    st = launch_proj(q, shape->Lq, shape->B, Wq16, hm.n_ret, hm.ret_q, q16, s);
-    if (st != RTP_OK) return st;
+    set_job(p.job[nj], q, shape->Lq, Wq16, hm.n_ret, q16);
+    for (int sl = 0; sl < hm.n_ret; ++sl) p.head_of_slot[nj][sl] = hm.ret_q[sl];
+    max_rows = std::max(max_rows, shape->Lq);
+    ++nj;
   }
   if (do_k) {
-    int16_t kv_of_slot[kMaxHeads];
+    set_job(p.job[nj], k, shape->Lk, Wk16, hm.H_k16, k16);
     for (int sl = 0; sl < hm.H_k16; ++sl)
-      kv_of_slot[sl] = k16_per_kv_head ? hm.rkv[sl] : (int16_t)(hm.ret_q[sl] / hm.G);
-    st = launch_proj(k, shape->Lk, shape->B, Wk16, hm.H_k16, kv_of_slot, k16, s);
+      p.head_of_slot[nj][sl] = k16_per_kv_head ? hm.rkv[sl] : (int16_t)(hm.ret_q[sl] / hm.G);
+    max_rows = std::max(max_rows, shape->Lk);
+    ++nj;
   }
+  dim3 grid((max_rows + kProjRows - 1) / kProjRows, p.job[0].n_slots + p.job[1].n_slots, shape->B);
+  if (grid.z > 65535 || grid.y > 65535) return RTP_ERR_UNSUPPORTED;
+  TraceScope tr("proj16", s);
+  proj16_kernel<<<grid, kProjThreads, 0, s>>>(p);
+  st = check_cuda(cudaGetLastError());
   return st;
 }

@@ -118,8 +118,10 @@ constexpr int kDecGLo = -1024;         // absolute bin of global bin 0
 constexpr int kDecCap = 4096;          // candidates a decode row resolves with one sort
 constexpr int kDecMaxSplits = 256;     // split-KV partials per (batch, kv head) in decode
 
+constexpr int kDecSub = 64;            // sub-bins of a row's crossing bin
+
 struct DecodeWs {   // retrieval decode
-  size_t scores, hist_m, hist_c, flags, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
+  size_t scores, hist_m, hist_c, flags, sub_m, sub_c, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
       part, mcount, total;
   int n_chunks, n_splits, Lk_pad, rows, groups;
 };
@@ -152,6 +154,8 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
   w.hist_m = take((size_t)w.rows * kDecGBins * 8);   // hist_m, hist_c, flags are one
   w.hist_c = take((size_t)w.rows * kDecGBins * 4);   // contiguous range (cleared per call)
   w.flags = take((size_t)w.rows * 4);
+  w.sub_m = take((size_t)w.rows * kDecSub * 8);       // also cleared per call
+  w.sub_c = take((size_t)w.rows * kDecSub * 4);
   w.rowsel = take((size_t)w.rows * sizeof(RowSel));
   w.rowres = take((size_t)w.rows * sizeof(RowRes));
   w.cand = take((size_t)w.rows * kDecCap * 8);
@@ -169,7 +173,7 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
 // Buffers the gathered decode attention reads (decode.cu).
 struct DecodeLists {
   const uint2* list;       // [groups][Lk_pad], chunk c's entries at c * kDecChunk
-  const int32_t* loff;     // [groups][n_chunks + 1] exclusive prefix of the chunk counts
+  const int32_t* lcount;   // [groups][n_chunks] entries per chunk
   const float* scores;
   const RowRes* rowres;
   float* part;

@@ -26,6 +26,7 @@
 #include <algorithm>
 
 #include "rtp_host.h"
+#include "tma.cuh"
 
 namespace rtp {
 namespace {
@@ -37,19 +38,35 @@ constexpr int kThreads = 256;
 constexpr double kFix21 = 1.0 / 2097152.0;  // 2^-21
 constexpr int kWarpCap = 512;               // candidates one warp sorts on its own
 
-// Absolute score bin floor(s * kappa), rounding toward -inf; clamped far outside
-// the histogram's range so that bin arithmetic never overflows.
-__device__ __forceinline__ int sbin(float s) {
-  const float x = fminf(fmaxf(__fmul_rn(s, kDecKappa), -1073741824.0f), 1073741824.0f);
-  return __float2int_rd(x);
+// Absolute score bin floor(s * kappa), rounding toward -inf.  kappa * s is
+// clamped to +-2^21 (far outside the histogram's range); adding 1.5 * 2^23 with
+// rounding toward -inf leaves floor(x) in the low mantissa bits, exactly, for
+// |x| < 2^22.  sbin_m returns that sum: the bin is bin_f / bin_i of it.
+__device__ __forceinline__ float sbin_m(float s) {
+  const float x = fminf(fmaxf(__fmul_rn(s, kDecKappa), -2097152.0f), 2097152.0f);
+  return __fadd_rd(x, 12582912.0f);
+}
+__device__ __forceinline__ float bin_f(float m) { return __fsub_rn(m, 12582912.0f); }
+__device__ __forceinline__ int bin_i(float m) { return __float_as_int(m) - 0x4B400000; }
+__device__ __forceinline__ int sbin(float s) { return bin_i(sbin_m(s)); }
+// 2^x for x <= 0 (no subnormal results matter here: x >= -0.37 in every use
+// that feeds a decision, and tiny results only need to stay tiny).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 // Mass of a key relative to the upper edge (b+1)/kappa of its bin: (0.78, 1].
-__device__ __forceinline__ float wbin(float s, int b) {
-  const float edge = __fmul_rn((float)(b + 1), 1.0f / kDecKappa);
-  return exp2f(__fmul_rn(__fsub_rn(s, edge), kLog2e));
+__device__ __forceinline__ float wbin_f(float s, float bf) {
+  const float edge = __fmul_rn(__fadd_rn(bf, 1.0f), 1.0f / kDecKappa);
+  return ex2_ftz(__fmul_rn(__fsub_rn(s, edge), kLog2e));
 }
+__device__ __forceinline__ float wbin(float s, int b) { return wbin_f(s, (float)b); }
+// trunc(w * 2^21) for w in [0, 1]: adding 2^23 with rounding toward zero leaves
+// the integer part in the low mantissa bits.
 __device__ __forceinline__ uint32_t fixed21(float w) {
-  return __float2uint_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f));
+  return __float_as_uint(__fadd_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f), 8388608.0f)) -
+         0x4B000000u;
 }
 // Sub-bin of a key inside its (crossing) bin b: 64 equal slices of [b, b+1)/kappa.
 __device__ __forceinline__ int subbin(float s, int b) {
@@ -70,11 +87,27 @@ __device__ __forceinline__ float key_score(uint32_t key) {
 }
 
 // ------------------------------------------------------------------ 1. score + histogram
+// Persistent, TMA-fed.  Work items are (kv group, 512 consecutive keys); a CTA
+// takes items blockIdx.x, blockIdx.x + gridDim.x, ...  One producer thread
+// streams each item's k16 rows as boxes of T keys x kw slots into a ring of
+// shared-memory stages; 8 consumer warps compute the scores,
+// then per item: the heads' max bins, the scores' store, a 256-bin window
+// histogram per head in shared memory and its flush into the row's absolute
+// histogram.  The producer keeps the ring full across those phases.
+//
+// The scores are a batched 16-element dot product per (key, head), which is
+// CUDA-core FMA work; the box is 128-byte swizzled when its rows are 128 bytes
+// or wider, so that the 32 lanes' 16-byte loads of 32 consecutive pairs hit
+// every bank once.
+constexpr int kSItem = 512;                      // keys per work item
+constexpr int kSStages = 4;
+constexpr int kSStageBytes = 16384;
+constexpr int kSConsumers = 256;                 // 8 warps
+constexpr int kSThreads = kSConsumers + 32;      // + the producer warp
+
 struct ScoreParams {
   const uint16_t* q16;
   int64_t q16_sb;
-  const uint16_t* k16;
-  int64_t k16_sb, k16_sl;
   float* scores;
   unsigned long long* hist_m;  // [rows][kDecGBins]
   uint32_t* hist_c;
@@ -82,136 +115,239 @@ struct ScoreParams {
   uint32_t* ncand;
   uint32_t* counter;
   uint32_t* mcount;
-  int N, Lk_pad, n_ret, n_rkv, G, per_kv;
+  DevStatus* status;
+  int N, Lk_pad, n_ret, n_rkv, G, lgG, per_kv, rows, groups;
+  int T;             // keys per box (a multiple of 16 dividing kSItem)
+  int kw;            // k16 slots per key in a box: G, or 1 when k16 is per kv head
+  int swz;           // 1: the box is 128-byte swizzled (rows of kw x 32 bytes, kw >= 4)
+  int batch_coord;   // 1, or 0 when every batch entry shares one k16 cache
+  int items_per_group, n_items;
 };
 
-__global__ void __launch_bounds__(kThreads) dec_score_kernel(const ScoreParams p) {
+struct ScoreSmemTail {
+  uint64_t full[kSStages];
+  uint64_t empty[kSStages];
+  int top[16];
+  int gave_up;
+};
+
+__host__ __device__ constexpr size_t score_smem_bytes(int G) {
+  return 1024 + (size_t)kSStages * kSStageBytes + (size_t)G * (kSItem + 4) * 4 +
+         (size_t)G * kDecWin * 8 + sizeof(ScoreSmemTail);
+}
+
+__global__ void __launch_bounds__(kSThreads, 2)
+    dec_score_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int G = p.G;
-  float* sc = reinterpret_cast<float*>(smem_raw);                        // [G][kDecChunk+4]
-  uint32_t* hm = reinterpret_cast<uint32_t*>(sc + G * (kDecChunk + 4));  // [G][kDecWin]
-  uint32_t* hc = hm + G * kDecWin;                                       // [G][kDecWin]
-  int* top = reinterpret_cast<int*>(hc + G * kDecWin);                   // [G]
+  // stages on a 1024-byte boundary (score_smem_bytes includes the slack)
+  unsigned char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  float* sc = reinterpret_cast<float*>(ring + kSStages * kSStageBytes);  // [G][kSItem+4]
+  uint32_t* hm = reinterpret_cast<uint32_t*>(sc + G * (kSItem + 4));     // [G][kDecWin]
+  uint32_t* hc = hm + G * kDecWin;
+  ScoreSmemTail* tl = reinterpret_cast<ScoreSmemTail*>(hc + G * kDecWin);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const int chunk = blockIdx.x;
-  const int grp = blockIdx.y;  // b * n_rkv + rk
-  const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
-  const int tid = threadIdx.x;
-  const int row0 = b * p.n_ret + rk * G;
-  if (chunk == 0) {  // the later kernels of this call count into these
-    if (tid < G) p.ncand[row0 + tid] = 0u;
-    if (tid == 0) {
-      p.counter[grp] = 0u;
-      p.mcount[grp] = 0u;
-    }
+  // the later kernels of this call count into these
+  for (int x = blockIdx.x * kSThreads + tid; x < p.rows; x += gridDim.x * kSThreads)
+    p.ncand[x] = 0u;
+  for (int x = blockIdx.x * kSThreads + tid; x < p.groups; x += gridDim.x * kSThreads) {
+    p.counter[x] = 0u;
+    p.mcount[x] = 0u;
   }
-  for (int x = tid; x < G * kDecWin; x += kThreads) {
+  for (int x = tid; x < G * kDecWin; x += kSThreads) {
     hm[x] = 0u;
     hc[x] = 0u;
   }
+  if (tid == 0) {
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&tl->full[s], 1);
+      mbar_init(&tl->empty[s], kSConsumers / 32);
+    }
+    tl->gave_up = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  volatile int* gave_up = &tl->gave_up;
+  const int box_bytes = p.T * p.kw * 32;
 
-  const int hh = tid % G;  // G divides 256: constant per thread
-  const int hr = rk * G + hh;
-  float q[kR];
-  {
-    const uint16_t* qp = p.q16 + b * p.q16_sb + (int64_t)hr * kR;
-    const uint4 a = *reinterpret_cast<const uint4*>(qp);
-    const uint4 c = *reinterpret_cast<const uint4*>(qp + 8);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      q[2 * i] = bf16_lo(w[i]);
-      q[2 * i + 1] = bf16_hi(w[i]);
+  if (warp == kSConsumers / 32) {  // ---------------- producer
+    if (lane == 0) {
+      int stage = 0, n_issued = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
+        const int grp = item / p.items_per_group, j0 = (item % p.items_per_group) * kSItem;
+        const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
+        const int nvalid = max(0, min(kSItem, p.N - j0));
+        const int nb = (nvalid + p.T - 1) / p.T;
+        const int slot0 = p.per_kv ? rk : rk * G;
+        // swizzled maps count 64-element (4-slot) quads in dim 1; others slots x 16 in dim 0
+        const int c0 = p.swz ? 0 : slot0 * kR, c1 = p.swz ? slot0 / 4 : 0;
+        for (int bx = 0; bx < nb; ++bx) {
+          if (!mbar_wait(&tl->empty[stage], ph ^ 1u, gave_up)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tl->full[stage], (uint32_t)box_bytes);
+          tma_load_4d(ring + stage * kSStageBytes, &kmap, c0, c1, j0 + bx * p.T,
+                      b * p.batch_coord, &tl->full[stage]);
+          ++n_issued;
+          if (++stage == kSStages) {
+            stage = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 20);
+      // every copy still in flight lands before the CTA may exit
+      for (int k = max(0, n_issued - kSStages); k < n_issued; ++k)
+        mbar_wait_drain(&tl->full[k % kSStages], (uint32_t)(k / kSStages) & 1u);
     }
+    return;
   }
-  const int slot = p.per_kv ? rk : hr;
-  const uint16_t* kb = p.k16 + b * p.k16_sb + (int64_t)slot * kR;
-  const int j0 = chunk * kDecChunk;
-  const int pairs = kDecChunk * G;
-  constexpr int kUnroll = 4;
-  for (int base = 0; base < pairs; base += kThreads * kUnroll) {
-    uint4 ka[kUnroll], kc[kUnroll];
-    int tok[kUnroll];
+
+  // ---------------- consumers (threads 0..255; named barrier 1)
+  const int hh = tid & (G - 1);         // G divides 256: constant per thread
+  const int hoff = p.per_kv ? 0 : hh;   // the head's k16 slot within the key's row
+  int stage = 0;
+  uint32_t ph = 0;
+  bool ok = true;
+  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    const int grp = item / p.items_per_group, j0 = (item % p.items_per_group) * kSItem;
+    const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
+    const int row0 = b * p.n_ret + rk * G;
+    const int nvalid = max(0, min(kSItem, p.N - j0));
+    const int nb = (nvalid + p.T - 1) / p.T;
+    float q[kR];  // q16 of this thread's head hh
+    {
+      const uint16_t* qp = p.q16 + b * p.q16_sb + (int64_t)(rk * G + hh) * kR;
+      const uint4 a = *reinterpret_cast<const uint4*>(qp);
+      const uint4 c = *reinterpret_cast<const uint4*>(qp + 8);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int pr = base + u * kThreads + tid;
-      tok[u] = pr / G;
-      const int j = j0 + tok[u];
-      if (pr < pairs && j < p.N) {
-        const uint16_t* src = kb + (int64_t)j * p.k16_sl;
-        ka[u] = __ldcs(reinterpret_cast<const uint4*>(src));
-        kc[u] = __ldcs(reinterpret_cast<const uint4*>(src + 8));
-      } else {
-        ka[u] = make_uint4(0, 0, 0, 0);
-        kc[u] = ka[u];
+      for (int i = 0; i < 8; ++i) {
+        q[2 * i] = bf16_lo(w[i]);
+        q[2 * i + 1] = bf16_hi(w[i]);
       }
     }
+    const int pairs = p.T * G;  // (key, head) pairs per box
+    float* scrow = sc + hh * (kSItem + 4);
+    for (int bx = 0; bx < nb; ++bx) {
+      ok = ok && mbar_wait_warp(&tl->full[stage], ph, gave_up);
+      if (ok) {
+        const unsigned char* buf = ring + stage * kSStageBytes;
+        const int lim = p.N - j0 - bx * p.T;  // keys of this box below N
+        // two pairs per pass, each dot as two chains (even / odd dims) summed at
+        // the end: a fixed order, four independent FMA chains
+        for (int pr = tid; pr < pairs; pr += 2 * kSConsumers) {
+          const bool second = pr + kSConsumers < pairs;
+          const int xk0 = pr >> p.lgG, xk1 = second ? (pr + kSConsumers) >> p.lgG : xk0;
+          uint4 kv[2][2];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int pr = base + u * kThreads + tid;
-      if (pr >= pairs) continue;
-      const uint32_t w[8] = {ka[u].x, ka[u].y, ka[u].z, ka[u].w,
-                             kc[u].x, kc[u].y, kc[u].z, kc[u].w};
-      float s = 0.f;
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t lin = (uint32_t)(((u ? xk1 : xk0) * p.kw + hoff) * 32);
+            const uint32_t o = p.swz ? swizzle128(lin) : lin;  // bytes 16..31 sit at o ^ 16
+            kv[u][0] = *reinterpret_cast<const uint4*>(buf + o);
+            kv[u][1] = *reinterpret_cast<const uint4*>(buf + (o ^ 16u));
+          }
+          float se[2] = {0.f, 0.f}, so[2] = {0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        s = fmaf(q[2 * c], bf16_lo(w[c]), s);
-        s = fmaf(q[2 * c + 1], bf16_hi(w[c]), s);
+          for (int c = 0; c < 8; ++c) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const uint4& kk = kv[u][c >> 2];
+              const uint32_t w =
+                  (c & 3) == 0 ? kk.x : (c & 3) == 1 ? kk.y : (c & 3) == 2 ? kk.z : kk.w;
+              se[u] = fmaf(q[2 * c], bf16_lo(w), se[u]);
+              so[u] = fmaf(q[2 * c + 1], bf16_hi(w), so[u]);
+            }
+          }
+          scrow[bx * p.T + xk0] = (xk0 < lim) ? __fadd_rn(se[0], so[0]) + 0.0f : -INFINITY;
+          if (second)
+            scrow[bx * p.T + xk1] = (xk1 < lim) ? __fadd_rn(se[1], so[1]) + 0.0f : -INFINITY;
+        }
       }
-      s = s + 0.0f;
-      const int j = j0 + tok[u];
-      sc[hh * (kDecChunk + 4) + tok[u]] = (j < p.N) ? s : -INFINITY;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tl->empty[stage]);
+      if (++stage == kSStages) {
+        stage = 0;
+        ph ^= 1u;
+      }
     }
-  }
-  __syncthreads();
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int h = warp; h < G; h += kThreads / 32) {
-    const float* row = sc + h * (kDecChunk + 4);
-    float mx = -INFINITY;
-    float* dst = p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0;
-    for (int x = lane * 4; x < kDecChunk; x += 128) {
-      const float4 v = *reinterpret_cast<const float4*>(row + x);
-      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
-      *reinterpret_cast<float4*>(dst + x) = v;
+    // keys of the item past the last box (past N): -inf
+    if (nb * p.T < kSItem)
+      for (int idx = tid; idx < G * kSItem; idx += kSConsumers) {
+        const int h = idx / kSItem, x = idx % kSItem;
+        if (x >= nb * p.T) sc[h * (kSItem + 4) + x] = -INFINITY;
+      }
+    named_bar(1, kSConsumers);
+    for (int h = warp; h < G; h += kSConsumers / 32) {  // max bin per head, scores' store
+      const float* row = sc + h * (kSItem + 4);
+      float mx = -INFINITY;
+      float* dst = p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0;
+      for (int x = lane * 4; x < kSItem; x += 128) {
+        const float4 v = *reinterpret_cast<const float4*>(row + x);
+        mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+        *reinterpret_cast<float4*>(dst + x) = v;
+      }
+      mx = warp_max(mx);
+      if (lane == 0) tl->top[h] = sbin(mx);
     }
-    mx = warp_max(mx);
-    if (lane == 0) top[h] = sbin(mx);
-  }
-  __syncthreads();
-  const int nvalid = min(kDecChunk, p.N - j0);
-  for (int idx = tid; idx < G * kDecChunk; idx += kThreads) {
-    const int h = idx / kDecChunk, x = idx % kDecChunk;
-    if (x >= nvalid) continue;
-    const float s = sc[h * (kDecChunk + 4) + x];
-    const int bb = sbin(s);
-    const int wi = top[h] - bb;  // 0 = the chunk's top bin
-    const uint32_t f = fixed21(wbin(s, bb));
-    if (wi < kDecWin) {
-      atomicAdd(&hm[h * kDecWin + wi], f);
-      atomicAdd(&hc[h * kDecWin + wi], 1u);
-    } else {  // far below this chunk's max: straight into the row histogram
-      int gb = bb - kDecGLo;
-      if (gb < 0) {
-        gb = 0;
+    named_bar(1, kSConsumers);
+    // a warp covers 32 / G keys x G heads: bins of different heads never collide
+    {
+      const int top = tl->top[hh];
+      uint32_t* whm = hm + hh * kDecWin;
+      uint32_t* whc = hc + hh * kDecWin;
+      const int row = row0 + hh;
+      const int xs = kSConsumers >> p.lgG;  // keys per pass
+      for (int x0 = tid >> p.lgG; x0 < nvalid; x0 += 4 * xs) {
+        float m[4], w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float sv = (x0 + u * xs < nvalid) ? scrow[x0 + u * xs] : -INFINITY;
+          m[u] = sbin_m(sv);
+          w[u] = sv;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (x0 + u * xs >= nvalid) break;
+          const int bi = bin_i(m[u]);
+          const int wi = top - bi;  // 0 = the item's top bin
+          const uint32_t f = fixed21(wbin_f(w[u], bin_f(m[u])));
+          if (wi < kDecWin) {
+            atomicAdd(&whm[wi], f);
+            atomicAdd(&whc[wi], 1u);
+          } else {  // far below this item's max: straight into the row histogram
+            int gb = bi - kDecGLo;
+            if (gb < 0) {
+              gb = 0;
+              atomicOr(&p.flags[row], 1u);
+            }
+            atomicAdd(&p.hist_m[(int64_t)row * kDecGBins + gb], (unsigned long long)f);
+            atomicAdd(&p.hist_c[(int64_t)row * kDecGBins + gb], 1u);
+          }
+        }
+      }
+    }
+    named_bar(1, kSConsumers);
+    for (int x = tid; x < G * kDecWin; x += kSConsumers) {  // flush the windows
+      const uint32_t c = hc[x];
+      if (c == 0) continue;
+      const int h = x / kDecWin, wi = x % kDecWin;
+      int gb = tl->top[h] - wi - kDecGLo;
+      if (gb < 0 || gb >= kDecGBins) {
+        gb = gb < 0 ? 0 : kDecGBins - 1;
         atomicOr(&p.flags[row0 + h], 1u);
       }
-      atomicAdd(&p.hist_m[(int64_t)(row0 + h) * kDecGBins + gb], (unsigned long long)f);
-      atomicAdd(&p.hist_c[(int64_t)(row0 + h) * kDecGBins + gb], 1u);
+      atomicAdd(&p.hist_m[(int64_t)(row0 + h) * kDecGBins + gb], (unsigned long long)hm[x]);
+      atomicAdd(&p.hist_c[(int64_t)(row0 + h) * kDecGBins + gb], c);
+      hm[x] = 0u;
+      hc[x] = 0u;
     }
   }
-  __syncthreads();
-  for (int x = tid; x < G * kDecWin; x += kThreads) {
-    const uint32_t c = hc[x];
-    if (c == 0) continue;
-    const int h = x / kDecWin, wi = x % kDecWin;
-    int gb = top[h] - wi - kDecGLo;
-    if (gb < 0 || gb >= kDecGBins) {
-      gb = gb < 0 ? 0 : kDecGBins - 1;
-      atomicOr(&p.flags[row0 + h], 1u);
-    }
-    atomicAdd(&p.hist_m[(int64_t)(row0 + h) * kDecGBins + gb], (unsigned long long)hm[x]);
-    atomicAdd(&p.hist_c[(int64_t)(row0 + h) * kDecGBins + gb], c);
-  }
+  if (!ok && tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 21);
 }
 
 // ------------------------------------------------------------------ 2. per-row merge
@@ -967,9 +1103,6 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     ScoreParams sp;
     sp.q16 = static_cast<const uint16_t*>(q16.ptr);
     sp.q16_sb = q16.stride_b;
-    sp.k16 = static_cast<const uint16_t*>(k16_cache.ptr);
-    sp.k16_sb = k16_cache.stride_b;
-    sp.k16_sl = k16_cache.stride_l;
     sp.scores = static_cast<float*>(at(L.scores));
     sp.hist_m = static_cast<unsigned long long*>(at(L.hist_m));
     sp.hist_c = static_cast<uint32_t*>(at(L.hist_c));
@@ -977,19 +1110,57 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     sp.ncand = static_cast<uint32_t*>(at(L.ncand));
     sp.counter = static_cast<uint32_t*>(at(L.counter));
     sp.mcount = static_cast<uint32_t*>(at(L.mcount));
+    sp.status = static_cast<DevStatus*>(ws);
     sp.N = N;
     sp.Lk_pad = L.Lk_pad;
     sp.n_ret = hm.n_ret;
     sp.n_rkv = hm.n_rkv;
     sp.G = hm.G;
+    sp.lgG = 0;
+    while ((1 << sp.lgG) < hm.G) ++sp.lgG;  // G is a power of two (it divides 256)
     sp.per_kv = k16_per_kv_head;
-    const size_t smem =
-        (size_t)hm.G * (kDecChunk + 4) * 4 + (size_t)hm.G * kDecWin * 8 + (size_t)hm.G * 4 + 16;
+    sp.rows = L.rows;
+    sp.groups = groups;
+    sp.kw = k16_per_kv_head ? 1 : hm.G;
+    sp.swz = sp.kw >= 4 ? 1 : 0;
+    sp.T = std::min(256, kSStageBytes / (sp.kw * kR * 2));  // divides kSItem
+    sp.batch_coord = (k16_cache.stride_b != 0 || shape->B == 1) ? 1 : 0;
+    sp.items_per_group = L.Lk_pad / kSItem;
+    sp.n_items = groups * sp.items_per_group;
+    // k16 as a 4-D tensor; keys past N read as 0.  Swizzled: {64 elements (4
+    // slots), slots / 4, keys 0..N-1, batch}; else {slots x 16, 1, keys, batch}.
+    CUtensorMap kmap;
+    const uint64_t sl_bytes = (uint64_t)k16_cache.stride_l * 2;
+    const uint64_t sb_bytes =
+        sp.batch_coord && k16_cache.stride_b != 0 ? (uint64_t)k16_cache.stride_b * 2 : sl_bytes * N;
+    const uint64_t nbatch = sp.batch_coord ? (uint64_t)shape->B : 1u;
+    const uint64_t row_el = (uint64_t)hm.H_k16 * kR;
+    uint64_t dims[4], strides[3];
+    uint32_t box[4];
+    if (sp.swz) {
+      dims[0] = 64; dims[1] = row_el / 64; dims[2] = (uint64_t)N; dims[3] = nbatch;
+      strides[0] = 128; strides[1] = sl_bytes; strides[2] = sb_bytes;
+      box[0] = 64; box[1] = (uint32_t)(sp.kw / 4); box[2] = (uint32_t)sp.T; box[3] = 1;
+    } else {
+      dims[0] = row_el; dims[1] = 1; dims[2] = (uint64_t)N; dims[3] = nbatch;
+      strides[0] = sl_bytes; strides[1] = sl_bytes; strides[2] = sb_bytes;
+      box[0] = (uint32_t)(sp.kw * kR); box[1] = 1; box[2] = (uint32_t)sp.T; box[3] = 1;
+    }
+    if (!tma_encode_bf16(&kmap, k16_cache.ptr, 4, dims, strides, box, sp.swz != 0))
+      return RTP_ERR_CUDA;
+    const size_t smem = score_smem_bytes(hm.G);
     if (cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return RTP_ERR_CUDA;
+    int dev = 0, n_sm = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dec_score_kernel, kSThreads,
+                                                      smem) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    const int grid = std::max(1, std::min(sp.n_items, std::max(1, per_sm) * n_sm));
     TraceScope tr("dec_score", s);
-    dec_score_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(sp);
+    dec_score_kernel<<<grid, kSThreads, smem, s>>>(kmap, sp);
     if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
   }
   {  // 2. per-row merge

@@ -1,0 +1,132 @@
+// tma.cuh -- mbarrier and TMA (cp.async.bulk.tensor) helpers for sm_100a.
+//
+// Every wait is bounded in time: once a wait has given up (which valid copies
+// never cause), the CTA's shared `gave_up` flag makes all later waits return at
+// once, so a failing kernel still terminates; the kernel records the failure in
+// the workspace status word.  No multicast forms are used.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "rtp_common.cuh"
+
+namespace rtp {
+
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: no valid copy takes this long
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// As above, letting the thread sleep up to `ns` nanoseconds for the phase.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete; false once this or
+// an earlier wait of the CTA gave up (after kWaitNs).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* gave_up) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (*gave_up) return false;
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+    if (globaltimer_ns() - t0 > kWaitNs) {
+      *gave_up = 1;
+      return false;
+    }
+  }
+}
+
+// Warp-wide wait: lane 0 polls, then every lane observes the completed phase
+// itself (which cannot advance again before this warp releases the stage).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* gave_up) {
+  const int lane = threadIdx.x & 31;
+  bool ok = true;
+  if (lane == 0) ok = mbar_wait(bar, parity, gave_up);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  if (ok && lane != 0) ok = mbar_wait(bar, parity, gave_up);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Same, ignoring the CTA's flag: used to drain copies in flight before exit.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+// 4-D tiled TMA load of one box into shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];\n" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Byte offset of `lin` inside a 1024-byte-aligned region written by TMA with
+// 128-byte swizzling: the 16-byte chunk index (bits 4..6) is XORed with the
+// 128-byte row index within each 1024-byte block (bits 7..9).
+__device__ __forceinline__ uint32_t swizzle128(uint32_t lin) {
+  return lin ^ (((lin >> 7) & 7u) << 4);
+}
+
+// Named barrier for a subset of the CTA's warps.
+__device__ __forceinline__ void named_bar(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Host: encode a bf16 tensor map of `rank` dims (innermost first; strides in
+// bytes for dims 1..rank-1), optionally with 128-byte swizzling.  Returns false
+// if the driver call is unavailable or rejects the map.
+bool tma_encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+
+}  // namespace rtp

@@ -109,6 +109,13 @@ def test_decode_per_kv_k16():
     run_decode(W["decode_128k_b8"], 6000, 2, 0.95, per_kv=True)
 
 
+@pytest.mark.parametrize("H", [4, 8, 16, 64])
+@pytest.mark.parametrize("per_kv", [False, True])
+def test_decode_head_groups(H, per_kv):
+    """G = H / 4 query heads per kv head in {1, 2, 4, 16}, k16 per query head or per kv head."""
+    run_decode(W["decode_128k_b8"].with_(H=H), 3000, 2, 0.9, per_kv=per_kv)
+
+
 def test_decode_128k_batch8_full():
     """The full 128K x batch-8 decode workload: every row of every head."""
     run_decode(W["decode_128k_b8"], 131072, 8, 0.95)

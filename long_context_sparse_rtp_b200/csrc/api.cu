@@ -146,7 +146,7 @@ extern "C" int rtp_trace_read(rtp_trace_entry* out, int max_entries) {
 
 namespace rtp {
 bool tma_encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128) {
+                     const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -158,6 +158,14 @@ bool tma_encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
   });
   if (encode == nullptr || rank < 1 || rank > 5) return false;
+  CUtensorMapSwizzle swz;
+  switch (swizzle_bytes) {
+    case 0: swz = CU_TENSOR_MAP_SWIZZLE_NONE; break;
+    case 32: swz = CU_TENSOR_MAP_SWIZZLE_32B; break;
+    case 64: swz = CU_TENSOR_MAP_SWIZZLE_64B; break;
+    case 128: swz = CU_TENSOR_MAP_SWIZZLE_128B; break;
+    default: return false;
+  }
   cuuint64_t d[5], st[4];
   cuuint32_t bx[5], es[5];
   for (int i = 0; i < rank; ++i) {
@@ -167,8 +175,7 @@ bool tma_encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
     if (i > 0) st[i - 1] = strides_bytes[i - 1];
   }
   return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }

@@ -1146,7 +1146,7 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
       strides[0] = sl_bytes; strides[1] = sl_bytes; strides[2] = sb_bytes;
       box[0] = (uint32_t)(sp.kw * kR); box[1] = 1; box[2] = (uint32_t)sp.T; box[3] = 1;
     }
-    if (!tma_encode_bf16(&kmap, k16_cache.ptr, 4, dims, strides, box, sp.swz != 0))
+    if (!tma_encode_bf16(&kmap, k16_cache.ptr, 4, dims, strides, box, sp.swz ? 128 : 0))
       return RTP_ERR_CUDA;
     const size_t smem = score_smem_bytes(hm.G);
     if (cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -3,47 +3,66 @@
 // Rule ("Dynamic Top-p Selection Mechanism", Eq. 5, paper-graph-ui summary of
 // arXiv 2605.16928): softmax the indexer scores of a query row, keep the
 // shortest prefix of the keys in (score desc, index asc) order whose mass
-// reaches p * Z.  The L x L score matrix is never stored: each CTA owns 64 query
-// rows of one retrieval head and streams that head's k16 tiles (L2-resident)
-// through several sweeps, recomputing Q16.K16^T on the tensor cores each time:
+// reaches p * Z.  The L x L score matrix is never stored.  A CTA owns 128 query
+// rows of one retrieval head and sweeps that head's k16 rows (L2-resident)
+// several times; every sweep recomputes the 128 x 128 score tiles
+// S = Q16 . K16^T on the tensor cores (one tcgen05.mma, M = N = 128, K = 16,
+// per tile, fp32 in TMEM) and one epilogue thread per query row reads its row
+// of each tile from TMEM, so all per-row state lives in that thread:
 //
-//   sweep 1  row max m                                   (1 compare / pair)
-//   sweep 2  Z = sum exp(s - m) and a 64-bin mass histogram of the scores in
+//   sweep 1  row max m                                    (1 compare / key)
+//   sweep 2  Z = sum exp(s - m) and a 32-bin mass histogram of the scores in
 //            [c0, m], c0 = m - ln(N / (1 - p)) - 1 (keys below c0 can never be
-//            kept: their total mass is < (1-p) Z)          (1 exp / pair)
+//            kept: their total mass is < (1-p) Z)           (1 exp / key)
 //   sweep 3+ radix refinement inside the crossing bin on the composite key
-//            (score key : 32 bits, 2^21-1-index : 21 bits), 6 bits per sweep,
-//            until the crossing bin holds <= 64 keys; those are collected,
-//            sorted and walked to the exact cut (a compare / pair).
+//            (score key : 32 bits, 2^21-1-index : 21 bits), 5 bits per sweep,
+//            until the crossing bin holds <= 32 keys; those are collected,
+//            sorted and walked to the exact cut.
 //
-// Masses are summed as 40-bit fixed point in 64-bit integers, so every sum is
-// exact and independent of the order atomics land in: the selection is
-// deterministic run to run.
+// Histogram masses are kept relative to the top edge e of their bin: a key adds
+// trunc(2^21 exp(s - e)) (a value in (0.7, 1] x 2^21) to its bin, so shared-memory
+// 32-bit atomics per tile group, flushed into 64-bit sums, are exact and
+// order-free; a bin's mass is its integer sum times exp(e - m) 2^-21, taken in
+// fp64 in a fixed order.  Z is a fixed-order fp32 tree per 32 keys summed in
+// fp64.  The selection is deterministic run to run.
+//
+// Warp roles: warps 0-3 epilogue (thread = query row = TMEM lane), warp 4 the
+// TMA producer (Q16 tile once, K16 tiles into a ring), warp 5 the MMA issuer
+// (owns the 256 TMEM columns: two 128-column accumulators).
+#include <cuda.h>
+
 #include "rtp_host.h"
+#include "tcgen05.cuh"
+#include "tma.cuh"
 
 namespace rtp {
 namespace {
 
-constexpr int kBM = 64;
-constexpr int kBN = 64;
-constexpr int kNB = 64;
-constexpr int kCap = 64;
-constexpr int kThreads = 128;
+constexpr int kBM = 128;         // query rows per CTA (MMA M, TMEM lanes)
+constexpr int kBN = 128;         // keys per tile (MMA N)
+constexpr int kStages = 4;       // K16 tile ring
+constexpr int kTileBytes = kBN * kR * 2;
+constexpr int kNB = 32;          // histogram bins (5-bit digits)
+constexpr int kDigit = 5;
+constexpr int kCap = 32;         // candidates collected per row
+constexpr int kGroup = 8;        // tiles per 32-bit bin-sum group: <= 1024 keys x 2^21 < 2^32
+constexpr int kMaxIter = 16;     // refine / collect sweeps (53 key bits / 5 + 1 suffice)
+constexpr int kEpi = 256;        // epilogue threads: two per query row (column halves)
+constexpr int kProdWarp = kEpi / 32, kMmaWarp = kEpi / 32 + 1;
+constexpr int kThreads = kEpi + 64;
 constexpr int kIdxBits = 21;
 constexpr unsigned long long kIdxMask = (1ull << kIdxBits) - 1;
 constexpr int kKeyBits = 32 + kIdxBits;  // 53
+constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 
 enum { ST_IDLE = 0, ST_REFINE = 1, ST_COLLECT = 2, ST_DONE = 3 };
 
 struct SelParams {
-  const uint16_t* q16;
-  int64_t q16_sb, q16_sl;
-  const uint16_t* k16;
-  int64_t k16_sb, k16_sl;
-  int Lq, Lk;
+  int Lq;
   int64_t q_pos0;
   int n_ret;
   float p;
+  int batch_coord_q, batch_coord_k;
   float* thr;
   int32_t* jtie;
   int32_t* count;
@@ -53,27 +72,44 @@ struct SelParams {
 };
 
 struct SelSmem {
-  uint16_t k16[2][kBN][kR];
-  unsigned long long hm[kBM][kNB];
-  uint32_t hc[kBM][kNB];
-  unsigned long long cand[kBM][kCap];
-  unsigned long long zf[kBM];
-  unsigned long long acc_above[kBM];
-  unsigned long long prefix[kBM];
-  double T[kBM];
-  float m[kBM], c0[kBM], scale[kBM];
-  uint32_t cnt_above[kBM];
-  int state[kBM], k0[kBM], pbits[kBM], ncand[kBM];
+  uint8_t ktile[kStages][kTileBytes];  // 1024-byte aligned (the struct is placed so)
+  uint8_t qtile[kBM * kR * 2];
+  union {
+    unsigned long long hw[kNB][kBM];   // per-row bin sums (fixed21 units), row fastest
+    unsigned long long cand[kCap][kBM];
+  } u;
+  uint32_t wacc[kNB][kBM];             // bin sums of the current tile group
+  uint32_t hc[kNB][kBM];               // bin counts
+  float tab[kNB][kBM];                 // exp(b / scale): level-0 bin b's edge factor
+  float mpart[2][kBM];
+  double zpart[2][kBM];
+  int ncnt[kBM];
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], qfull, ctl;
+  uint32_t tmem_base;
+  int go;
+  int gave_up;
 };
 
-__device__ __forceinline__ float canon(float s) { return s + 0.0f; }  // -0 -> +0
-
-__device__ __forceinline__ float mass_w(float s, float m) {
-  return exp2f(__fmul_rn(__fsub_rn(s, m), kLog2e));
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
-
+// exp(s - m) for s <= m.
+__device__ __forceinline__ float rel_w(float s, float m) {
+  return ex2_ftz(__fmul_rn(__fsub_rn(s, m), kLog2e));
+}
+// trunc(w * 2^21) for w in [0, 1]: adding 2^23 with rounding toward zero leaves
+// the integer part in the low mantissa bits.
+__device__ __forceinline__ uint32_t fixed21(float w) {
+  return __float_as_uint(__fadd_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f), 8388608.0f)) -
+         0x4B000000u;
+}
+// Level-0 bin of a score s <= m: floor((m - s) * scale), at most kNB - 1 (adding
+// 1.5 * 2^23 with rounding toward -inf leaves the floor in the low mantissa bits).
 __device__ __forceinline__ int bin0_of(float s, float m, float scale) {
-  const int b = (int)__fmul_rn(__fsub_rn(m, s), scale);
+  const float x = fminf(__fmul_rn(__fsub_rn(m, s), scale), 1048576.0f);
+  const int b = __float_as_int(__fadd_rd(x, 12582912.0f)) - 0x4B400000;
   return b < kNB - 1 ? b : kNB - 1;
 }
 
@@ -86,347 +122,447 @@ __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float(b);
 }
 
-__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int o) {
-  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, o);
-  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), o);
-  return ((unsigned long long)hi << 32) | lo;
-}
-
-struct SelCtx {
-  int b, hr, slot, m0, nrows, n_tiles, warp, lane, g, t;
-  int rA, rB;          // CTA-local rows owned by this thread (g, g+8 of the warp)
-  int64_t PA, PB;      // their positions
-  bool vA, vB;         // rows exist
-  int64_t warp_maxP;   // largest position among this warp's rows (-1: none)
-  uint32_t qa[4];      // q16 A fragment
-};
-
-// Stream the k16 tiles 0..n_tiles-1 and call body(kt, s) with this warp's
-// 16 x 64 score tile (s[nt][e]: row g (e<2) or g+8, key kt*64 + nt*8 + 2t + (e&1)).
-template <class Body>
-__device__ __forceinline__ void sweep(SelSmem& sm, const SelParams& p, const SelCtx& c,
-                                      bool warp_active, Body&& body) {
-  const int tid = threadIdx.x;
-  const uint16_t* kbase = p.k16 + c.b * p.k16_sb + c.slot * kR;
-  auto load = [&](int kt, int buf) {
-    const int key = tid >> 1, ch = tid & 1;
-    const int j = kt * kBN + key;
-    const bool ok = j < p.Lk;
-    const uint16_t* src = kbase + (int64_t)(ok ? j : 0) * p.k16_sl + ch * 8;
-    cp_async16(smem_u32(&sm.k16[buf][key][(ch ^ ((key >> 2) & 1)) * 8]), src, ok);
-  };
-  load(0, 0);
-  cp_async_commit();
-  for (int kt = 0; kt < c.n_tiles; ++kt) {
-    if (kt + 1 < c.n_tiles) {
-      load(kt + 1, (kt + 1) & 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (warp_active && (int64_t)kt * kBN <= c.warp_maxP) {
-      const int buf = kt & 1;
-      float s[8][4];
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        const int q = c.lane >> 3;
-        const int key = np * 16 + (c.lane & 7) + 8 * (q >> 1);
-        const int ch = q & 1;
-        uint32_t r[4];
-        ldmatrix_x4(r, smem_u32(&sm.k16[buf][key][(ch ^ ((key >> 2) & 1)) * 8]));
-        mma16816_zero(s[2 * np], c.qa, r[0], r[1]);
-        mma16816_zero(s[2 * np + 1], c.qa, r[2], r[3]);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s[nt][e] = canon(s[nt][e]);
-      body(kt, s);
-    }
-    __syncthreads();
-  }
-}
-
-// Crossing search over a descending histogram: the first bin where the running
-// mass reaches T.  Returns the bin; updates acc/cnt with the bins above it.
-__device__ __forceinline__ int crossing(const unsigned long long* hm, const uint32_t* hc, int nb,
-                                        double T, unsigned long long& acc, uint32_t& cnt,
+// Crossing search over one row's descending histogram (column r of hw / hc):
+// the first bin b where base + factor(b) * (inner + hw[b]) reaches T.  Returns
+// the bin; adds the bins above it to inner (same-factor histograms) or base
+// (factor per bin) and to cnt.
+template <class Factor>
+__device__ __forceinline__ int crossing(const SelSmem& sm, int r, int nb, double T, bool per_bin,
+                                        Factor&& factor, double& base,
+                                        unsigned long long& inner, uint32_t& cnt,
                                         uint32_t& n_in) {
   int last = -1;
   for (int b = 0; b < nb; ++b) {
-    if (hc[b] == 0) continue;
+    const uint32_t c = sm.hc[b][r];
+    if (c == 0) continue;
     last = b;
-    if ((double)(acc + hm[b]) >= T) {
-      n_in = hc[b];
+    const unsigned long long wb = sm.u.hw[b][r];
+    const double f = factor(b);
+    if (per_bin ? (base + f * (double)wb >= T) : (base + f * (double)(inner + wb) >= T)) {
+      n_in = c;
       return b;
     }
-    acc += hm[b];
-    cnt += hc[b];
+    if (per_bin)
+      base += f * (double)wb;
+    else
+      inner += wb;
+    cnt += c;
   }
   // rounding left T out of reach: keep everything, i.e. the lowest non-empty bin
   if (last >= 0) {
-    acc -= hm[last];
-    cnt -= hc[last];
-    n_in = hc[last];
+    if (per_bin)
+      base -= factor(last) * (double)sm.u.hw[last][r];
+    else
+      inner -= sm.u.hw[last][r];
+    cnt -= sm.hc[last][r];
+    n_in = sm.hc[last][r];
   }
   return last;
 }
 
-__global__ void __launch_bounds__(kThreads) topp_select_kernel(const SelParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw);
-  SelCtx c;
-  c.b = blockIdx.z;
-  c.hr = blockIdx.y;
-  c.slot = p.k16_slot[c.hr];
-  const int tile = gridDim.x - 1 - blockIdx.x;  // heavy (late) tiles first
-  c.m0 = tile * kBM;
-  c.nrows = min(kBM, p.Lq - c.m0);
-  const int tid = threadIdx.x;
-  c.warp = tid >> 5;
-  c.lane = tid & 31;
-  c.g = c.lane >> 2;
-  c.t = c.lane & 3;
-  c.rA = c.warp * 16 + c.g;
-  c.rB = c.rA + 8;
-  c.vA = c.rA < c.nrows;
-  c.vB = c.rB < c.nrows;
-  c.PA = p.q_pos0 + c.m0 + c.rA;
-  c.PB = p.q_pos0 + c.m0 + c.rB;
-  const int wlast = min(c.warp * 16 + 15, c.nrows - 1);
-  c.warp_maxP = (wlast >= c.warp * 16) ? p.q_pos0 + c.m0 + wlast : -1;
-  const int64_t Plast = p.q_pos0 + c.m0 + c.nrows - 1;
-  c.n_tiles = (int)((Plast + kBN) / kBN);
-
-  // q16 A fragment: rows g / g+8, dims 2t..2t+1 and 2t+8..2t+9
-  {
-    const uint16_t* qb = p.q16 + c.b * p.q16_sb + (int64_t)c.hr * kR;
-    auto ld = [&](int r, int d) -> uint32_t {
-      if (r >= c.nrows) return 0u;
-      return *reinterpret_cast<const uint32_t*>(qb + (int64_t)(c.m0 + r) * p.q16_sl + d);
-    };
-    c.qa[0] = ld(c.rA, 2 * c.t);
-    c.qa[1] = ld(c.rB, 2 * c.t);
-    c.qa[2] = ld(c.rA, 2 * c.t + 8);
-    c.qa[3] = ld(c.rB, 2 * c.t + 8);
+__device__ __forceinline__ void clear_row(SelSmem& sm, int r) {
+#pragma unroll 8
+  for (int b = 0; b < kNB; ++b) {
+    sm.u.hw[b][r] = 0ull;
+    sm.wacc[b][r] = 0u;
+    sm.hc[b][r] = 0u;
   }
+}
 
-  // ---------------------------------------------------------- sweep 1: max
-  {
-    float mx[2] = {-INFINITY, -INFINITY};
-    sweep(sm, p, c, true, [&](int kt, float (&s)[8][4]) {
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int64_t j = (int64_t)kt * kBN + nt * 8 + 2 * c.t + (e & 1);
-          const bool hi = e >= 2;
-          const bool ok = hi ? (c.vB && j <= c.PB) : (c.vA && j <= c.PA);
-          if (ok) mx[hi] = fmaxf(mx[hi], s[nt][e]);
-        }
-    });
-    mx[0] = quad_max(mx[0]);
-    mx[1] = quad_max(mx[1]);
-    if (c.t == 0) {
-      sm.m[c.rA] = mx[0];
-      sm.m[c.rB] = mx[1];
-    }
+// Moves the tile group's 32-bit bin sums into the 64-bit ones.
+__device__ __forceinline__ void flush_row(SelSmem& sm, int r) {
+#pragma unroll 8
+  for (int b = 0; b < kNB; ++b) {
+    sm.u.hw[b][r] += sm.wacc[b][r];
+    sm.wacc[b][r] = 0u;
   }
-  __syncthreads();
-  if (tid < kBM) {
-    const int r = tid;
-    if (r < c.nrows) {
-      const double N = (double)(p.q_pos0 + c.m0 + r + 1);
-      const float m = sm.m[r];
-      const float R = (float)(log(N / (1.0 - (double)p.p)) + 1.0);
-      sm.c0[r] = m - R;
-      sm.scale[r] = (float)kNB / R;
-      sm.state[r] = ST_REFINE;
+}
+
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float t[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) t[i] = fmaxf(v[i], v[i + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
+  return t[0];
+}
+
+// A refine / collect sweep's key that passed the score-interval prefilter:
+// the exact crossing-bin and prefix tests, then a candidate or a digit count.
+__device__ __noinline__ void refine_key(SelSmem& sm, int r, float s, int j, float m, float scale,
+                                        int k0, int pbits, unsigned long long prefix, int w,
+                                        float tk, bool collect) {
+  if (bin0_of(s, m, scale) != k0) return;
+  const unsigned long long ck = comp_key(s, j);
+  if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) return;
+  if (collect) {
+    const int slot_c = atomicAdd(&sm.ncnt[r], 1);
+    if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
+  } else {
+    const int digit = (int)((ck >> (kKeyBits - pbits - w)) & ((1ull << w) - 1));
+    const int bin = (1 << w) - 1 - digit;
+    atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(s, m), tk)));
+    atomicAdd(&sm.hc[bin][r], 1u);
+  }
+}
+
+// Score interval that holds every score of composite-key prefix `prefix`
+// (pbits bits) inside level-0 bin k0, widened by a relative margin.
+__device__ __forceinline__ void refine_range(float m, float scale, int k0, int pbits,
+                                             unsigned long long prefix, float& lo, float& hi) {
+  const float margin = 1e-5f * (fabsf(m) + (float)kNB / scale + 1.f);
+  lo = m - (float)(k0 + 1) / scale - margin;
+  hi = m - (float)k0 / scale + margin;
+  if (pbits > 0) {
+    uint32_t k_lo, k_hi;
+    if (pbits >= 32) {
+      k_lo = k_hi = (uint32_t)(prefix >> (pbits - 32));
     } else {
-      sm.state[r] = ST_IDLE;
+      k_lo = (uint32_t)(prefix << (32 - pbits));
+      k_hi = k_lo | ((1u << (32 - pbits)) - 1u);
     }
-    sm.acc_above[r] = 0;
-    sm.cnt_above[r] = 0;
-    sm.ncand[r] = 0;
-    sm.pbits[r] = 0;
-    sm.prefix[r] = 0;
-    for (int b = 0; b < kNB; ++b) {
-      sm.hm[r][b] = 0;
-      sm.hc[r][b] = 0;
-    }
+    float a = key_score(k_lo), c = key_score(k_hi);
+    if (a != a) a = -INFINITY;  // key ranges that reach NaN encodings
+    if (c != c) c = INFINITY;
+    lo = fmaxf(lo, a);
+    hi = fminf(hi, c);
   }
-  __syncthreads();
+}
 
-  // ---------------------------------------------------------- sweep 2: Z + level-0 histogram
-  {
-    const float mA = sm.m[c.rA], mB = sm.m[c.rB];
-    const float cA = sm.c0[c.rA], cB = sm.c0[c.rB];
-    const float sA = sm.scale[c.rA], sB = sm.scale[c.rB];
-    unsigned long long z[2] = {0ull, 0ull};
-    sweep(sm, p, c, true, [&](int kt, float (&s)[8][4]) {
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int64_t j = (int64_t)kt * kBN + nt * 8 + 2 * c.t + (e & 1);
-          const bool hi = e >= 2;
-          const bool ok = hi ? (c.vB && j <= c.PB) : (c.vA && j <= c.PA);
-          if (!ok) continue;
-          const float sv = s[nt][e];
-          const float m = hi ? mB : mA;
-          const unsigned long long f = mass_fixed40(mass_w(sv, m));
-          z[hi] += f;
-          if (sv >= (hi ? cB : cA)) {
-            const int r = hi ? c.rB : c.rA;
-            const int bin = bin0_of(sv, m, hi ? sB : sA);
-            atomicAdd(&sm.hm[r][bin], f);
-            atomicAdd(&sm.hc[r][bin], 1u);
-          }
-        }
-    });
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      z[h] += shfl_xor_u64(z[h], 1);
-      z[h] += shfl_xor_u64(z[h], 2);
-    }
-    if (c.t == 0) {
-      sm.zf[c.rA] = z[0];
-      sm.zf[c.rB] = z[1];
-    }
-  }
-  __syncthreads();
-  if (tid < c.nrows) {
-    const int r = tid;
-    const double T = (double)p.p * (double)sm.zf[r];
-    sm.T[r] = T;
-    unsigned long long acc = 0;
-    uint32_t cnt = 0, n_in = 0;
-    const int b = crossing(sm.hm[r], sm.hc[r], kNB, T, acc, cnt, n_in);
-    sm.acc_above[r] = acc;
-    sm.cnt_above[r] = cnt;
-    sm.k0[r] = b;
-    // composite-key prefix shared by every score this bin can hold
-    const float m = sm.m[r], scale = sm.scale[r];
-    const float hi_s = m - (float)b / scale, lo_s = m - (float)(b + 1) / scale;
-    const float margin = 1e-5f * (fabsf(m) + (float)kNB / scale + 1.f);
-    const unsigned long long kl = (unsigned long long)score_key(lo_s - margin) << kIdxBits;
-    const unsigned long long kh =
-        ((unsigned long long)score_key(hi_s + margin) << kIdxBits) | kIdxMask;
-    const int pb = (kl == kh) ? kKeyBits : (__clzll(kl ^ kh) - (64 - kKeyBits));
-    sm.pbits[r] = pb;
-    sm.prefix[r] = pb > 0 ? (kh >> (kKeyBits - pb)) : 0ull;
-    sm.state[r] = (n_in <= (uint32_t)kCap) ? ST_COLLECT : ST_REFINE;
-    for (int bb = 0; bb < kNB; ++bb) {
-      sm.hm[r][bb] = 0;
-      sm.hc[r][bb] = 0;
-    }
-  }
-  __syncthreads();
+__global__ void __launch_bounds__(kThreads, 2)
+    topp_select_kernel(const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap kmap, const SelParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelSmem& sm = *reinterpret_cast<SelSmem*>(smem_raw +
+                                             ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.z, hr = blockIdx.y;
+  const int slot = p.k16_slot[hr];
+  const int tile = gridDim.x - 1 - blockIdx.x;  // heavy (late) row blocks first
+  const int m0 = tile * kBM;
+  const int nrows = min(kBM, p.Lq - m0);
+  const int64_t Plast = p.q_pos0 + m0 + nrows - 1;
+  const int n_tiles = (int)((Plast + kBN) / kBN);
 
-  // ---------------------------------------------------------- sweeps 3+: refine / collect
-  for (int iter = 0; iter < 16; ++iter) {
-    const int active = __syncthreads_or(tid < kBM && (sm.state[tid] == ST_REFINE ||
-                                                      sm.state[tid] == ST_COLLECT));
-    if (!active) break;
-    int stA = sm.state[c.rA], stB = sm.state[c.rB];
-    const bool wact = __any_sync(0xffffffffu, (stA == ST_REFINE || stA == ST_COLLECT) ||
-                                                  (stB == ST_REFINE || stB == ST_COLLECT));
-    const float mA = sm.m[c.rA], mB = sm.m[c.rB];
-    const float cA = sm.c0[c.rA], cB = sm.c0[c.rB];
-    const float sA = sm.scale[c.rA], sB = sm.scale[c.rB];
-    const int kA = sm.k0[c.rA], kB = sm.k0[c.rB];
-    const int pbA = sm.pbits[c.rA], pbB = sm.pbits[c.rB];
-    const unsigned long long pxA = sm.prefix[c.rA], pxB = sm.prefix[c.rB];
-    sweep(sm, p, c, wact, [&](int kt, float (&s)[8][4]) {
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool hi = e >= 2;
-          const int st = hi ? stB : stA;
-          if (st != ST_REFINE && st != ST_COLLECT) continue;
-          const int64_t j = (int64_t)kt * kBN + nt * 8 + 2 * c.t + (e & 1);
-          if (j > (hi ? c.PB : c.PA)) continue;
-          const float sv = s[nt][e];
-          if (sv < (hi ? cB : cA)) continue;
-          const float m = hi ? mB : mA;
-          if (bin0_of(sv, m, hi ? sB : sA) != (hi ? kB : kA)) continue;
-          const unsigned long long ck = comp_key(sv, (int)j);
-          const int pb = hi ? pbB : pbA;
-          if (pb > 0 && (ck >> (kKeyBits - pb)) != (hi ? pxB : pxA)) continue;
-          const int r = hi ? c.rB : c.rA;
-          if (st == ST_COLLECT) {
-            const int idx = atomicAdd(&sm.ncand[r], 1);
-            if (idx < kCap) sm.cand[r][idx] = ck;
-          } else {
-            const int w = min(6, kKeyBits - pb);
-            const int digit = (int)((ck >> (kKeyBits - pb - w)) & ((1ull << w) - 1));
-            const int bin = (1 << w) - 1 - digit;
-            atomicAdd(&sm.hm[r][bin], mass_fixed40(mass_w(sv, m)));
-            atomicAdd(&sm.hc[r][bin], 1u);
-          }
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.tfull[i], 1);
+      mbar_init(&sm.tempty[i], kEpi / 32);
+    }
+    mbar_init(&sm.qfull, 1);
+    mbar_init(&sm.ctl, 1);
+    sm.gave_up = 0;
+    sm.go = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, 2 * kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* gave_up = &sm.gave_up;
+  volatile int* go = &sm.go;
+
+  if (warp == kProdWarp) {  // ------------------------------------- TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      int stage = 0, n_issued = 0;
+      uint32_t sph = 0;
+      mbar_arrive_expect_tx(&sm.qfull, (uint32_t)(kBM * kR * 2));
+      tma_load_4d(sm.qtile, &qmap, 0, hr, m0, b * p.batch_coord_q, &sm.qfull);
+      for (int sweep = 0; ok; ++sweep) {
+        if (sweep >= 2) {  // another sweep only if some row still needs one
+          ok = mbar_wait(&sm.ctl, (uint32_t)(sweep - 2) & 1u, gave_up);
+          if (!ok || *go == 0) break;
         }
-    });
-    __syncthreads();
-    if (tid < kBM) {
-      const int r = tid;
-      const int st = sm.state[r];
-      if (st == ST_COLLECT) {
-        int n = sm.ncand[r];
-        if (n > kCap) {
-          set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 11);
-          n = kCap;
-        }
-        unsigned long long* cd = sm.cand[r];
-        for (int a = 1; a < n; ++a) {  // insertion sort, descending
-          const unsigned long long x = cd[a];
-          int q = a - 1;
-          while (q >= 0 && cd[q] < x) {
-            cd[q + 1] = cd[q];
-            --q;
-          }
-          cd[q + 1] = x;
-        }
-        unsigned long long cum = sm.acc_above[r];
-        const double T = sm.T[r];
-        const float m = sm.m[r];
-        int take = n;
-        for (int a = 0; a < n; ++a) {
-          cum += mass_fixed40(mass_w(key_score((uint32_t)(cd[a] >> kIdxBits)), m));
-          if ((double)cum >= T) {
-            take = a + 1;
+        for (int kt = 0; kt < n_tiles; ++kt) {
+          if (!mbar_wait(&sm.empty[stage], sph ^ 1u, gave_up)) {
+            ok = false;
             break;
           }
-        }
-        const unsigned long long last = cd[take - 1];
-        const int i = c.m0 + r;
-        const int64_t o = ((int64_t)c.b * p.n_ret + c.hr) * p.Lq + i;
-        p.thr[o] = key_score((uint32_t)(last >> kIdxBits));
-        p.jtie[o] = (int32_t)(kIdxMask - (last & kIdxMask));
-        p.count[o] = (int32_t)(sm.cnt_above[r] + take);
-        if (p.mass) p.mass[o] = (float)((double)cum / (double)sm.zf[r]);
-        sm.state[r] = ST_DONE;
-      } else if (st == ST_REFINE) {
-        const int pb = sm.pbits[r];
-        const int w = min(6, kKeyBits - pb);
-        unsigned long long acc = sm.acc_above[r];
-        uint32_t cnt = sm.cnt_above[r], n_in = 0;
-        const int b = crossing(sm.hm[r], sm.hc[r], 1 << w, sm.T[r], acc, cnt, n_in);
-        sm.acc_above[r] = acc;
-        sm.cnt_above[r] = cnt;
-        const int digit = (1 << w) - 1 - b;
-        sm.prefix[r] = (sm.prefix[r] << w) | (unsigned long long)digit;
-        sm.pbits[r] = pb + w;
-        sm.state[r] = (n_in <= (uint32_t)kCap || pb + w >= kKeyBits) ? ST_COLLECT : ST_REFINE;
-        for (int bb = 0; bb < kNB; ++bb) {
-          sm.hm[r][bb] = 0;
-          sm.hc[r][bb] = 0;
+          mbar_arrive_expect_tx(&sm.full[stage], (uint32_t)kTileBytes);
+          tma_load_4d(sm.ktile[stage], &kmap, 0, slot, kt * kBN, b * p.batch_coord_k,
+                      &sm.full[stage]);
+          ++n_issued;
+          if (++stage == kStages) {
+            stage = 0;
+            sph ^= 1u;
+          }
         }
       }
-      sm.ncand[r] = 0;
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 12);
+      // every copy in flight lands before the CTA may exit
+      for (int k = max(0, n_issued - kStages); k < n_issued; ++k)
+        mbar_wait_drain(&sm.full[k % kStages], (uint32_t)(k / kStages) & 1u);
+      mbar_wait_drain(&sm.qfull, 0u);
     }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {  // ------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.qfull, 0u, gave_up);
+      const uint64_t adesc = sdesc_k_sw32(smem_u32(sm.qtile), 256);
+      int stage = 0;
+      uint32_t sph = 0, tcount = 0;
+      for (int sweep = 0; ok; ++sweep) {
+        if (sweep >= 2) {
+          ok = mbar_wait(&sm.ctl, (uint32_t)(sweep - 2) & 1u, gave_up);
+          if (!ok || *go == 0) break;
+        }
+        for (int kt = 0; kt < n_tiles; ++kt) {
+          const int buf = (int)(tcount & 1u);
+          if (!mbar_wait(&sm.full[stage], sph, gave_up) ||
+              !mbar_wait(&sm.tempty[buf], ((tcount >> 1) & 1u) ^ 1u, gave_up)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_bf16_ss(tmem + (uint32_t)(buf * kBN), adesc,
+                      sdesc_k_sw32(smem_u32(sm.ktile[stage]), 256), kIdesc, false);
+          mma_commit(&sm.empty[stage]);  // the K16 stage is free once the MMA has read it
+          mma_commit(&sm.tfull[buf]);    // the accumulator is ready
+          ++tcount;
+          if (++stage == kStages) {
+            stage = 0;
+            sph ^= 1u;
+          }
+        }
+      }
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 13);
+      if (tcount > 0)  // the last MMA is complete before TMEM is released
+        mbar_wait_drain(&sm.tfull[(tcount - 1) & 1u], ((tcount - 1) >> 1) & 1u);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue: two threads per row
+    // Thread (r, g) reads TMEM lane r, columns 64 g .. 64 g + 63 of every tile.
+    // Per-row decisions are computed identically by both from shared memory;
+    // g == 0 clears, flushes and writes the outputs.
+    const int r = tid & (kBM - 1), g = tid >> 7;
+    const bool valid = r < nrows;
+    const int64_t P = valid ? p.q_pos0 + m0 + r : -1;
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)(g * 64);
+    uint32_t tcount = 0;
+    bool ok = true;
+    auto ebar = [] { named_bar(1, kEpi); };
+    // one pass over the key tiles: body(j0, v) sees keys j0 .. j0 + 31 of this row;
+    // with a histogram, each tile group's 32-bit sums move to the 64-bit ones
+    auto sweep = [&](auto&& body, bool hist, bool row_hist) {
+      for (int kt = 0; kt < n_tiles; ++kt) {
+        const int buf = (int)(tcount & 1u);
+        ok = ok && mbar_wait_warp(&sm.tfull[buf], (tcount >> 1) & 1u, gave_up);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            float v[32];
+            tmem_ld32(lane_addr + (uint32_t)(buf * kBN + c * 32), v);
+            body(kt * kBN + g * 64 + c * 32, v);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+        ++tcount;
+        if (hist && ((kt & (kGroup - 1)) == kGroup - 1 || kt == n_tiles - 1)) {
+          ebar();
+          if (g == 0 && row_hist) flush_row(sm, r);
+          ebar();
+        }
+      }
+    };
+
+    // ---- sweep 1: row max
+    float m = -INFINITY;
+    sweep(
+        [&](int j0, float (&v)[32]) {
+          if ((int64_t)j0 + 31 > P) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if ((int64_t)(j0 + i) > P) v[i] = -INFINITY;
+          }
+          m = fmaxf(m, max32(v));
+        },
+        false, false);
+    sm.mpart[g][r] = m;
+    ebar();
+    m = fmaxf(sm.mpart[0][r], sm.mpart[1][r]);
+    float c0 = 0.f, scale = 0.f;
+    if (valid) {
+      const double N = (double)(P + 1);
+      const float R = (float)(log(N / (1.0 - (double)p.p)) + 1.0);
+      c0 = m - R;
+      scale = (float)kNB / R;
+    }
+    if (g == 0) {
+      clear_row(sm, r);
+      for (int bb = 0; bb < kNB; ++bb) sm.tab[bb][r] = expf((float)bb / scale);
+    }
+    ebar();
+
+    // ---- sweep 2: Z and the level-0 histogram over [c0, m]; a key in bin b adds
+    // trunc(2^21 exp(s - m) exp(b / scale)) = trunc(2^21 exp(s - edge_b))
+    double Zp = 0.0;
+    sweep(
+        [&](int j0, float (&v)[32]) {
+          if (!valid) return;
+          const bool full = (int64_t)j0 + 31 <= P;
+          float e[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const bool in = full || (int64_t)(j0 + i) <= P;
+            const float s = v[i];
+            e[i] = in ? rel_w(s, m) : 0.f;
+            if (in && s >= c0) {
+              const int bb = bin0_of(s, m, scale);
+              atomicAdd(&sm.wacc[bb][r], fixed21(__fmul_rn(e[i], sm.tab[bb][r])));
+              atomicAdd(&sm.hc[bb][r], 1u);
+            }
+          }
+#pragma unroll
+          for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) e[i] = __fadd_rn(e[i], e[i + w]);
+          Zp += (double)e[0];
+        },
+        true, valid);
+    sm.zpart[g][r] = Zp;
+    ebar();
+    const double Z = sm.zpart[0][r] + sm.zpart[1][r];
+    double T = 0.0, base = 0.0, fk = 0.0;  // fk: mass of one fixed21 unit of bin k0
+    unsigned long long inner = 0ull, prefix = 0ull;
+    uint32_t cnt_above = 0u;
+    int k0 = 0, pbits = 0, state = ST_IDLE;
+    float tk = 0.f;  // exp(k0 / scale)
+    if (valid) {
+      T = (double)p.p * Z;
+      uint32_t n_in = 0u;
+      auto f0 = [&](int bb) { return (1.0 / 2097152.0) / (double)sm.tab[bb][r]; };
+      k0 = crossing(sm, r, kNB, T, true, f0, base, inner, cnt_above, n_in);
+      tk = sm.tab[k0][r];
+      fk = f0(k0);
+      // composite-key prefix shared by every score the crossing bin can hold
+      const float hi_s = m - (float)k0 / scale, lo_s = m - (float)(k0 + 1) / scale;
+      const float margin = 1e-5f * (fabsf(m) + (float)kNB / scale + 1.f);
+      const unsigned long long kl = (unsigned long long)score_key(lo_s - margin) << kIdxBits;
+      const unsigned long long kh =
+          ((unsigned long long)score_key(hi_s + margin) << kIdxBits) | kIdxMask;
+      pbits = (kl == kh) ? kKeyBits : (__clzll(kl ^ kh) - (64 - kKeyBits));
+      prefix = pbits > 0 ? (kh >> (kKeyBits - pbits)) : 0ull;
+      state = (n_in <= (uint32_t)kCap) ? ST_COLLECT : ST_REFINE;
+    }
+    ebar();
+    if (g == 0) clear_row(sm, r);
+
+    // ---- sweeps 3+: refine the crossing bin 5 bits at a time, then collect
+    for (int iter = 0;; ++iter) {
+      const bool mine = state == ST_REFINE || state == ST_COLLECT;
+      if (g == 0) sm.ncnt[r] = 0;
+      bool any = bar_or(1, kEpi, mine);
+      if (any && iter >= kMaxIter) {
+        if (tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 14);
+        any = false;
+      }
+      if (tid == 0) {  // tell the producer and the MMA issuer whether to sweep again
+        *go = any ? 1 : 0;
+        mbar_arrive(&sm.ctl);
+      }
+      if (!any) break;
+      const int w = min(kDigit, kKeyBits - pbits);
+      const bool collect = state == ST_COLLECT;
+      float lo = 0.f, hi = -1.f;
+      if (mine) refine_range(m, scale, k0, pbits, prefix, lo, hi);
+      sweep(
+          [&](int j0, float (&v)[32]) {
+            if (!mine) return;
+            const bool full = (int64_t)j0 + 31 <= P;
+            uint32_t hits = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float s = v[i];
+              const bool h = s >= lo && s <= hi && (full || (int64_t)(j0 + i) <= P);
+              hits |= (h ? 1u : 0u) << i;
+            }
+            if (hits == 0u) return;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if ((hits >> i) & 1u)  // -0 -> +0: one composite key per score
+                refine_key(sm, r, v[i] + 0.0f, j0 + i, m, scale, k0, pbits, prefix, w, tk,
+                           collect);
+          },
+          true, state == ST_REFINE);
+      ebar();
+      if (state == ST_COLLECT) {
+        if (g == 0) {
+          int n = sm.ncnt[r];
+          if (n > kCap) {
+            set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 11);
+            n = kCap;
+          }
+          const int i = m0 + r;
+          const int64_t o = ((int64_t)b * p.n_ret + hr) * p.Lq + i;
+          if (n == 0) {  // cannot happen for a consistent histogram; keep every key
+            set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 15);
+            p.thr[o] = -INFINITY;
+            p.jtie[o] = (int32_t)P;
+            p.count[o] = (int32_t)(P + 1);
+            if (p.mass) p.mass[o] = 1.f;
+          } else {
+            for (int a = 1; a < n; ++a) {  // insertion sort, descending
+              const unsigned long long x = sm.u.cand[a][r];
+              int q = a - 1;
+              while (q >= 0 && sm.u.cand[q][r] < x) {
+                sm.u.cand[q + 1][r] = sm.u.cand[q][r];
+                --q;
+              }
+              sm.u.cand[q + 1][r] = x;
+            }
+            unsigned long long acc = inner;
+            double cum = base;
+            int take = n;
+            for (int a = 0; a < n; ++a) {
+              const float sa = key_score((uint32_t)(sm.u.cand[a][r] >> kIdxBits));
+              acc += fixed21(__fmul_rn(rel_w(sa, m), tk));
+              cum = base + fk * (double)acc;
+              if (cum >= T) {
+                take = a + 1;
+                break;
+              }
+            }
+            const unsigned long long last = sm.u.cand[take - 1][r];
+            p.thr[o] = key_score((uint32_t)(last >> kIdxBits));
+            p.jtie[o] = (int32_t)(kIdxMask - (last & kIdxMask));
+            p.count[o] = (int32_t)(cnt_above + (uint32_t)take);
+            if (p.mass) p.mass[o] = (float)(cum / Z);
+          }
+        }
+        state = ST_DONE;
+      } else if (state == ST_REFINE) {
+        uint32_t n_in = 0u;
+        auto fd = [&](int) { return fk; };
+        const int bsel = crossing(sm, r, 1 << w, T, false, fd, base, inner, cnt_above, n_in);
+        const int digit = (1 << w) - 1 - bsel;
+        prefix = (prefix << w) | (unsigned long long)digit;
+        pbits += w;
+        state = (n_in <= (uint32_t)kCap || pbits >= kKeyBits) ? ST_COLLECT : ST_REFINE;
+      }
+      ebar();
+      if (g == 0 && state == ST_REFINE) clear_row(sm, r);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * kBN);
   }
 }
 
@@ -475,14 +611,7 @@ extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_
   if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
   if ((st = check_view(k16, hm.H_k16, kR, true)) != RTP_OK) return st;
   SelParams prm;
-  prm.q16 = static_cast<const uint16_t*>(q16.ptr);
-  prm.q16_sb = q16.stride_b;
-  prm.q16_sl = q16.stride_l;
-  prm.k16 = static_cast<const uint16_t*>(k16.ptr);
-  prm.k16_sb = k16.stride_b;
-  prm.k16_sl = k16.stride_l;
   prm.Lq = shape->Lq;
-  prm.Lk = shape->Lk;
   prm.q_pos0 = shape->q_pos0;
   prm.n_ret = hm.n_ret;
   prm.p = p;
@@ -492,7 +621,32 @@ extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_
   prm.mass = mass;
   prm.status = static_cast<DevStatus*>(ws);
   for (int i = 0; i < hm.n_ret; ++i) prm.k16_slot[i] = hm.ret_k16[i];
-  const size_t smem = sizeof(SelSmem);
+  // q16 / k16 as 4-D tensors {16, slots, rows, batch}; 128-row boxes of one slot,
+  // 32-byte swizzled (the canonical K-major operand layout of the MMA)
+  prm.batch_coord_q = (q16.stride_b != 0 || shape->B == 1) ? 1 : 0;
+  prm.batch_coord_k = (k16.stride_b != 0 || shape->B == 1) ? 1 : 0;
+  CUtensorMap qmap, kmap;
+  {
+    const uint64_t sl = (uint64_t)q16.stride_l * 2;
+    const uint64_t sb = prm.batch_coord_q && q16.stride_b != 0 ? (uint64_t)q16.stride_b * 2
+                                                               : sl * (uint64_t)shape->Lq;
+    const uint64_t dims[4] = {16, (uint64_t)hm.n_ret, (uint64_t)shape->Lq,
+                              prm.batch_coord_q ? (uint64_t)shape->B : 1u};
+    const uint64_t strides[3] = {32, sl, sb};
+    const uint32_t box[4] = {16, 1, (uint32_t)kBM, 1};
+    if (!tma_encode_bf16(&qmap, q16.ptr, 4, dims, strides, box, 32)) return RTP_ERR_CUDA;
+  }
+  {
+    const uint64_t sl = (uint64_t)k16.stride_l * 2;
+    const uint64_t sb = prm.batch_coord_k && k16.stride_b != 0 ? (uint64_t)k16.stride_b * 2
+                                                               : sl * (uint64_t)shape->Lk;
+    const uint64_t dims[4] = {16, (uint64_t)hm.H_k16, (uint64_t)shape->Lk,
+                              prm.batch_coord_k ? (uint64_t)shape->B : 1u};
+    const uint64_t strides[3] = {32, sl, sb};
+    const uint32_t box[4] = {16, 1, (uint32_t)kBN, 1};
+    if (!tma_encode_bf16(&kmap, k16.ptr, 4, dims, strides, box, 32)) return RTP_ERR_CUDA;
+  }
+  const size_t smem = sizeof(SelSmem) + 1024;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(topp_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -503,6 +657,6 @@ extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_
   dim3 grid((shape->Lq + kBM - 1) / kBM, hm.n_ret, shape->B);
   if (grid.y > 65535 || grid.z > 65535) return RTP_ERR_UNSUPPORTED;
   TraceScope tr("topp_select", s);
-  topp_select_kernel<<<grid, kThreads, smem, s>>>(prm);
+  topp_select_kernel<<<grid, kThreads, smem, s>>>(qmap, kmap, prm);
   return check_cuda(cudaGetLastError());
 }

@@ -124,9 +124,9 @@ __device__ __forceinline__ void named_bar(int id, int threads) {
 }
 
 // Host: encode a bf16 tensor map of `rank` dims (innermost first; strides in
-// bytes for dims 1..rank-1), optionally with 128-byte swizzling.  Returns false
-// if the driver call is unavailable or rejects the map.
+// bytes for dims 1..rank-1) with 0, 32, 64 or 128-byte swizzling.  Returns
+// false if the driver call is unavailable or rejects the map.
 bool tma_encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box, bool swizzle128);
+                     const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
 
 }  // namespace rtp

@@ -47,6 +47,8 @@ constexpr int kDigit = 5;
 constexpr int kCap = 32;         // candidates collected per row
 constexpr int kGroup = 8;        // tiles per 32-bit bin-sum group: <= 1024 keys x 2^21 < 2^32
 constexpr int kMaxIter = 16;     // refine / collect sweeps (53 key bits / 5 + 1 suffice)
+constexpr int kQueue = 64;       // per-warp queue of refine hits (drained at 32)
+constexpr int kChunk = 16;       // keys per TMEM load and per unrolled body
 constexpr int kEpi = 256;        // epilogue threads: two per query row (column halves)
 constexpr int kProdWarp = kEpi / 32, kMmaWarp = kEpi / 32 + 1;
 constexpr int kThreads = kEpi + 64;
@@ -80,7 +82,13 @@ struct SelSmem {
   } u;
   uint32_t wacc[kNB][kBM];             // bin sums of the current tile group
   uint32_t hc[kNB][kBM];               // bin counts
-  float tab[kNB][kBM];                 // exp(b / scale): level-0 bin b's edge factor
+  union {
+    float tab[kNB][kBM];               // exp(b / scale): level-0 bin b's edge factor
+    struct {                           // refine sweeps: per-warp queues of prefilter hits
+      float s[kEpi / 32][kQueue];
+      uint32_t jl[kEpi / 32][kQueue];  // key index | owner lane << 21
+    } q;
+  } t;
   float mpart[2][kBM];
   double zpart[2][kBM];
   int ncnt[kBM];
@@ -178,32 +186,50 @@ __device__ __forceinline__ void flush_row(SelSmem& sm, int r) {
   }
 }
 
-__device__ __forceinline__ float max32(const float (&v)[32]) {
-  float t[16];
+__device__ __forceinline__ float max16(const float (&v)[kChunk]) {
+  float t[kChunk / 2];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) t[i] = fmaxf(v[i], v[i + 16]);
+  for (int i = 0; i < kChunk / 2; ++i) t[i] = fmaxf(v[i], v[i + kChunk / 2]);
 #pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
+  for (int w = kChunk / 4; w >= 1; w >>= 1)
 #pragma unroll
     for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
   return t[0];
 }
 
-// A refine / collect sweep's key that passed the score-interval prefilter:
-// the exact crossing-bin and prefix tests, then a candidate or a digit count.
-__device__ __noinline__ void refine_key(SelSmem& sm, int r, float s, int j, float m, float scale,
+// Processes the first n (<= 32) queued prefilter hits of this warp, one per
+// lane: the exact crossing-bin and prefix tests of the owning row (whose state
+// is fetched from the owner lane), then a candidate or a digit count.  Called by
+// all 32 lanes.
+__device__ __noinline__ void drain_hits(SelSmem& sm, int wq, int n, int row0, float m, float scale,
                                         int k0, int pbits, unsigned long long prefix, int w,
-                                        float tk, bool collect) {
-  if (bin0_of(s, m, scale) != k0) return;
+                                        float tk, int collect) {
+  const int lane = threadIdx.x & 31;
+  const bool has = lane < n;
+  const float s = has ? sm.t.q.s[wq][lane] : 0.f;
+  const uint32_t jl = has ? sm.t.q.jl[wq][lane] : 0u;
+  const int owner = (int)(jl >> 21), j = (int)(jl & 0x1FFFFFu);
+  const float om = __shfl_sync(0xffffffffu, m, owner);
+  const float osc = __shfl_sync(0xffffffffu, scale, owner);
+  const int ok0 = __shfl_sync(0xffffffffu, k0, owner);
+  const int opb = __shfl_sync(0xffffffffu, pbits, owner);
+  const uint32_t opl = __shfl_sync(0xffffffffu, (uint32_t)prefix, owner);
+  const uint32_t oph = __shfl_sync(0xffffffffu, (uint32_t)(prefix >> 32), owner);
+  const int ow = __shfl_sync(0xffffffffu, w, owner);
+  const float otk = __shfl_sync(0xffffffffu, tk, owner);
+  const int ocol = __shfl_sync(0xffffffffu, collect, owner);
+  if (!has || bin0_of(s, om, osc) != ok0) return;
   const unsigned long long ck = comp_key(s, j);
-  if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) return;
-  if (collect) {
+  const unsigned long long opx = ((unsigned long long)oph << 32) | opl;
+  if (opb > 0 && (ck >> (kKeyBits - opb)) != opx) return;
+  const int r = row0 + owner;
+  if (ocol) {
     const int slot_c = atomicAdd(&sm.ncnt[r], 1);
     if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
   } else {
-    const int digit = (int)((ck >> (kKeyBits - pbits - w)) & ((1ull << w) - 1));
-    const int bin = (1 << w) - 1 - digit;
-    atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(s, m), tk)));
+    const int digit = (int)((ck >> (kKeyBits - opb - ow)) & ((1ull << ow) - 1));
+    const int bin = (1 << ow) - 1 - digit;
+    atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(s, om), otk)));
     atomicAdd(&sm.hc[bin][r], 1u);
   }
 }
@@ -353,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t tcount = 0;
     bool ok = true;
     auto ebar = [] { named_bar(1, kEpi); };
-    // one pass over the key tiles: body(j0, v) sees keys j0 .. j0 + 31 of this row;
+    // one pass over the key tiles: body(j0, v) sees keys j0 .. j0 + 15 of this row;
     // with a histogram, each tile group's 32-bit sums move to the 64-bit ones
     auto sweep = [&](auto&& body, bool hist, bool row_hist) {
       for (int kt = 0; kt < n_tiles; ++kt) {
@@ -362,10 +388,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         if (ok) {
 #pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            float v[32];
-            tmem_ld32(lane_addr + (uint32_t)(buf * kBN + c * 32), v);
-            body(kt * kBN + g * 64 + c * 32, v);
+          for (int c = 0; c < 4; ++c) {
+            float v[kChunk];
+            tmem_ld16(lane_addr + (uint32_t)(buf * kBN + c * kChunk), v);
+            body(kt * kBN + g * 64 + c * kChunk, v);
           }
         }
         tc_fence_before();
@@ -383,13 +409,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- sweep 1: row max
     float m = -INFINITY;
     sweep(
-        [&](int j0, float (&v)[32]) {
-          if ((int64_t)j0 + 31 > P) {
+        [&](int j0, float (&v)[kChunk]) {
+          if ((int64_t)j0 + kChunk - 1 > P) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
+            for (int i = 0; i < kChunk; ++i)
               if ((int64_t)(j0 + i) > P) v[i] = -INFINITY;
           }
-          m = fmaxf(m, max32(v));
+          m = fmaxf(m, max16(v));
         },
         false, false);
     sm.mpart[g][r] = m;
@@ -404,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     if (g == 0) {
       clear_row(sm, r);
-      for (int bb = 0; bb < kNB; ++bb) sm.tab[bb][r] = expf((float)bb / scale);
+      for (int bb = 0; bb < kNB; ++bb) sm.t.tab[bb][r] = expf((float)bb / scale);
     }
     ebar();
 
@@ -412,23 +438,23 @@ __global__ void __launch_bounds__(kThreads, 2)
     // trunc(2^21 exp(s - m) exp(b / scale)) = trunc(2^21 exp(s - edge_b))
     double Zp = 0.0;
     sweep(
-        [&](int j0, float (&v)[32]) {
+        [&](int j0, float (&v)[kChunk]) {
           if (!valid) return;
-          const bool full = (int64_t)j0 + 31 <= P;
-          float e[32];
+          const bool full = (int64_t)j0 + kChunk - 1 <= P;
+          float e[kChunk];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < kChunk; ++i) {
             const bool in = full || (int64_t)(j0 + i) <= P;
             const float s = v[i];
             e[i] = in ? rel_w(s, m) : 0.f;
-            if (in && s >= c0) {
+            if (in && s >= c0) {  // the few keys in [c0, m]
               const int bb = bin0_of(s, m, scale);
-              atomicAdd(&sm.wacc[bb][r], fixed21(__fmul_rn(e[i], sm.tab[bb][r])));
+              atomicAdd(&sm.wacc[bb][r], fixed21(__fmul_rn(e[i], sm.t.tab[bb][r])));
               atomicAdd(&sm.hc[bb][r], 1u);
             }
           }
 #pragma unroll
-          for (int w = 16; w >= 1; w >>= 1)
+          for (int w = kChunk / 2; w >= 1; w >>= 1)
 #pragma unroll
             for (int i = 0; i < w; ++i) e[i] = __fadd_rn(e[i], e[i + w]);
           Zp += (double)e[0];
@@ -445,9 +471,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (valid) {
       T = (double)p.p * Z;
       uint32_t n_in = 0u;
-      auto f0 = [&](int bb) { return (1.0 / 2097152.0) / (double)sm.tab[bb][r]; };
+      auto f0 = [&](int bb) { return (1.0 / 2097152.0) / (double)sm.t.tab[bb][r]; };
       k0 = crossing(sm, r, kNB, T, true, f0, base, inner, cnt_above, n_in);
-      tk = sm.tab[k0][r];
+      tk = sm.t.tab[k0][r];
       fk = f0(k0);
       // composite-key prefix shared by every score the crossing bin can hold
       const float hi_s = m - (float)k0 / scale, lo_s = m - (float)(k0 + 1) / scale;
@@ -480,25 +506,51 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool collect = state == ST_COLLECT;
       float lo = 0.f, hi = -1.f;
       if (mine) refine_range(m, scale, k0, pbits, prefix, lo, hi);
+      const int wq = warp, row0 = (warp & 3) * 32;
+      int qn = 0;  // entries in this warp's queue (warp-uniform)
       sweep(
-          [&](int j0, float (&v)[32]) {
-            if (!mine) return;
-            const bool full = (int64_t)j0 + 31 <= P;
+          [&](int j0, float (&v)[kChunk]) {
+            const bool full = (int64_t)j0 + kChunk - 1 <= P;
             uint32_t hits = 0u;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < kChunk; ++i) {
               const float s = v[i];
-              const bool h = s >= lo && s <= hi && (full || (int64_t)(j0 + i) <= P);
+              const bool h = mine && s >= lo && s <= hi && (full || (int64_t)(j0 + i) <= P);
               hits |= (h ? 1u : 0u) << i;
             }
-            if (hits == 0u) return;
+            if (__ballot_sync(0xffffffffu, hits != 0u) == 0u) return;
+            const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if ((hits >> i) & 1u)  // -0 -> +0: one composite key per score
-                refine_key(sm, r, v[i] + 0.0f, j0 + i, m, scale, k0, pbits, prefix, w, tk,
-                           collect);
+            for (int i = 0; i < kChunk; ++i) {
+              const bool h = (hits >> i) & 1u;
+              const uint32_t bal = __ballot_sync(0xffffffffu, h);
+              if (bal == 0u) continue;
+              if (h) {  // -0 -> +0: one composite key per score
+                const int pos = qn + __popc(bal & lt);
+                sm.t.q.s[wq][pos] = v[i] + 0.0f;
+                sm.t.q.jl[wq][pos] = (uint32_t)(j0 + i) | ((uint32_t)lane << 21);
+              }
+              qn += __popc(bal);
+              if (qn >= 32) {
+                __syncwarp();
+                drain_hits(sm, wq, 32, row0, m, scale, k0, pbits, prefix, w, tk, collect);
+                __syncwarp();
+                if (lane + 32 < qn) {
+                  sm.t.q.s[wq][lane] = sm.t.q.s[wq][lane + 32];
+                  sm.t.q.jl[wq][lane] = sm.t.q.jl[wq][lane + 32];
+                }
+                __syncwarp();
+                qn -= 32;
+              }
+            }
           },
           true, state == ST_REFINE);
+      if (qn > 0) {  // the last partial batch (row histograms flush below)
+        __syncwarp();
+        drain_hits(sm, wq, qn, row0, m, scale, k0, pbits, prefix, w, tk, collect);
+      }
+      ebar();
+      if (state == ST_REFINE && g == 0) flush_row(sm, r);
       ebar();
       if (state == ST_COLLECT) {
         if (g == 0) {

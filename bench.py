@@ -167,13 +167,44 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest rank's time (device tensor under nccl, host tensor under gloo)."""
     import torch
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own replica of the workload (weak scaling)."""
+    return seed + 1000 * rank
+
+
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, or None
+    when the summary is missing or the kernel's source has changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    traffic = src = sha = None
+    for ln in open(path):
+        if ln.startswith("traffic_bytes_per_launch:"):
+            traffic = int(ln.split(":")[1])
+        elif ln.startswith("source:"):
+            parts = ln.split()
+            src, sha = parts[1], parts[-1]
+    if traffic is None or src is None:
+        return None
+    fn = os.path.join(ROOT, src)
+    if not os.path.exists(fn):
+        return None
+    if hashlib.sha256(open(fn, "rb").read()).hexdigest()[:len(sha)] != sha:
+        return None
+    return traffic
 
 
 def trace_read():
@@ -200,7 +231,7 @@ def decode_state(rank: int):
     import torch
     from long_context_sparse_rtp_b200 import rtp_index_scores, synth
     w = synth.WORKLOADS[DECODE_WL]
-    w = w.with_(seed=w.seed + 1000 * rank)
+    w = w.with_(seed=rank_seed(w.seed, rank))
     inp = synth.make_inputs(w, "cuda")
     q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
     L = k.shape[1]
@@ -342,7 +373,7 @@ def bench_prefill(args, world, rank, pk):
     import torch
     from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
     w = synth.WORKLOADS[PREFILL_WL]
-    w = w.with_(seed=w.seed + 1000 * rank)
+    w = w.with_(seed=rank_seed(w.seed, rank))
     inp = synth.make_inputs(w, "cuda")
     q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
     flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
@@ -492,10 +523,7 @@ def main():
     score_bytes = dec["bytes"]["k16"]
     achieved = score_bytes / (score_ms / 1e3) / 1e9
     step_gbs = dec["bytes"]["total"] / (dec["ms_step"] / 1e3) / 1e9
-    traffic = None
-    prof = os.path.join(ROOT, "profiles", "dec_score_traffic.json")
-    if os.path.exists(prof):
-        traffic = json.load(open(prof)).get("bytes_per_launch")
+    traffic = profiled_traffic("dec_score_decode_128k_b8.md")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dec["ms_step"],

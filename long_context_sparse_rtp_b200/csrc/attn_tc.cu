@@ -1,0 +1,503 @@
+// attn_tc.cu -- causal prefill attention tiles on the 5th-generation tensor
+// cores, for the three head kinds:
+//
+//   DENSE  every key j <= P (baseline);
+//   LOCAL  keys j <= P with j < n_sink or j > P - window ("Local Head Attention
+//          Pattern" of the paper-graph-ui summary of arXiv 2605.16928); key
+//          tiles outside the sinks and the window are never visited;
+//   SPARSE keys j <= P kept by the row's top-p descriptor (thr, jtie) ("Dynamic
+//          Top-p Selection Mechanism"): each tile's 16-dim indexer scores are
+//          recomputed by the same tcgen05 MMA shape and operand placement the
+//          selection used (128 query rows x 128 keys, K = 16), so the kept set
+//          is reproduced bit for bit.
+//
+// One CTA = 128 query rows of one head, 128-key tiles.  Warp 4 loads Q once and
+// K/V (and K16) tiles into a 2-stage ring with TMA (128-byte swizzle); warp 5
+// issues S = Q K^T (8 MMAs, K = 16 each) into one of two TMEM score buffers and
+// O += P V into a TMEM accumulator; warps 0-3 hold one query row per thread:
+// read the scores with tcgen05.ld, mask, online softmax in the log2 domain,
+// write P (bf16) to shared memory for the PV MMA.  The running max is only
+// moved (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles
+// need no rescale.  P is rounded to bf16 once and the normaliser sums the
+// rounded values, so the output is an exact convex combination of them.
+#include <cuda.h>
+
+#include "rtp_host.h"
+#include "tcgen05.cuh"
+#include "tma.cuh"
+
+namespace rtp {
+namespace {
+
+constexpr int kBM = 128;                  // query rows per CTA (TMEM lanes)
+constexpr int kBN = 128;                  // keys per tile
+constexpr int kStages = 2;                // K/V ring
+constexpr int kHalf = 128 * 128;          // one 64-column half of a 128 x 128 bf16 tile: 16 KB
+constexpr int kTile = 2 * kHalf;          // 32 KB
+constexpr int kThreads = 192;
+constexpr float kRescale = 8.f;           // move the max when it grows by > 2^8
+constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD) | (1u << 16);  // V is MN-major
+
+enum { MODE_DENSE = 0, MODE_LOCAL = 1, MODE_SPARSE = 2 };
+
+struct AttnParams {
+  uint16_t* o; int64_t o_sb, o_sl;
+  float* lse;                // [B][H][Lq] or null
+  DevStatus* status;
+  const float* thr;          // [B][n_ret][Lq]
+  const int32_t* jtie;
+  int Lq, Lk, H, G, n_ret;
+  int64_t q_pos0;
+  int window, n_sink;
+  int bq, bk;                // batch coordinate multipliers (0 when a tensor is shared)
+  float scale_log2;          // softmax_scale * log2(e)
+  int16_t head[kMaxHeads];   // launch head index -> query head
+  int16_t slot[kMaxHeads];   // launch head index -> retrieval slot (SPARSE)
+  int16_t k16slot[kMaxHeads];// launch head index -> k16 slot (SPARSE)
+};
+
+struct TcSmem {                      // placed on a 1024-byte boundary
+  uint8_t q[kTile];                  // [2 halves of 64 dims][128 rows][128 B]
+  uint8_t k[kStages][kTile];
+  uint8_t v[kStages][kTile];         // rows = keys, 2 halves of 64 dims (MN-major B)
+  uint8_t p[kTile];                  // [2 halves of 64 keys][128 rows][128 B]
+  uint8_t q16[kBM * kR * 2];         // 32-byte rows, 32-byte swizzle
+  uint8_t k16[kStages][kBN * kR * 2];
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], s16_empty,
+      p_full, o_done;
+  uint32_t tmem_base;
+  int gave_up;
+};
+
+// The key-tile schedule of a row block: LOCAL visits the sink tiles, then the
+// window tiles; the other modes every tile up to the diagonal.
+struct Sched {
+  int n, sink_end, win_begin;
+  __device__ __forceinline__ int tile(int it) const {
+    return it < sink_end ? it : win_begin + (it - sink_end);
+  }
+};
+
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int MODE>
+__device__ __forceinline__ Sched make_sched(const AttnParams& p, int64_t P0, int64_t Plast) {
+  Sched s;
+  const int t_end = (int)(Plast / kBN);  // inclusive
+  if (MODE == MODE_LOCAL) {
+    int sink_end = (p.n_sink + kBN - 1) / kBN;
+    const int64_t wlo = P0 - p.window + 1;  // lowest window key of the block's first row
+    int win_begin = (int)((wlo > 0 ? wlo : 0) / kBN);
+    if (win_begin < sink_end) win_begin = sink_end;
+    sink_end = min(sink_end, t_end + 1);
+    s.sink_end = sink_end;
+    s.win_begin = win_begin;
+    s.n = sink_end + max(0, t_end - win_begin + 1);
+  } else {
+    s.sink_end = t_end + 1;
+    s.win_begin = t_end + 1;
+    s.n = t_end + 1;
+  }
+  return s;
+}
+
+// K-major operand descriptor: K step kk (16 elements) of a 128 x 128 tile.
+__device__ __forceinline__ uint64_t kdesc(const uint8_t* tile, int kk) {
+  return sdesc_sw128(smem_u32(tile) + (uint32_t)((kk >> 2) * kHalf + (kk & 3) * 32), 16, 1024);
+}
+// MN-major V descriptor: K step kk (16 keys = 2 KB of rows), 64-dim halves kHalf apart.
+__device__ __forceinline__ uint64_t vdesc(const uint8_t* tile, int kk) {
+  return sdesc_sw128(smem_u32(tile) + (uint32_t)(kk * 2048), kHalf, 1024);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap qmap,
+                   const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap,
+                   const __grid_constant__ CUtensorMap q16map,
+                   const __grid_constant__ CUtensorMap k16map, const AttnParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw +
+                                          ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hidx = blockIdx.y;
+  const int h = p.head[hidx];
+  const int kvh = h / p.G;
+  const int b = blockIdx.z;
+  const int rb = gridDim.x - 1 - blockIdx.x;  // heavy (late) row blocks first
+  const int m0 = rb * kBM;
+  const int nrows = min(kBM, p.Lq - m0);
+  const int64_t P0 = p.q_pos0 + m0;
+  const int64_t Plast = P0 + nrows - 1;
+  const Sched sch = make_sched<MODE>(p, P0, Plast);
+  const bool sparse = MODE == MODE_SPARSE;
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_empty[i], 4);
+    }
+    mbar_init(&sm.s16_empty, 4);
+    mbar_init(&sm.p_full, 4);
+    mbar_init(&sm.o_done, 1);
+    sm.gave_up = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const uint32_t t_s = tmem, t_o = tmem + 256, t_s16 = tmem + 384;
+  volatile int* gave_up = &sm.gave_up;
+
+  if (warp == 4) {  // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t qbytes = kTile + (sparse ? kBM * kR * 2 : 0);
+      const uint32_t kvbytes = 2 * kTile + (sparse ? kBN * kR * 2 : 0);
+      mbar_arrive_expect_tx(&sm.q_full, qbytes);
+      tma_load_4d(sm.q, &qmap, 0, h, m0, b * p.bq, &sm.q_full);
+      tma_load_4d(sm.q + kHalf, &qmap, 64, h, m0, b * p.bq, &sm.q_full);
+      if (sparse) tma_load_4d(sm.q16, &q16map, 0, p.slot[hidx], m0, b * p.bq, &sm.q_full);
+      int n_issued = 0;
+      for (int it = 0; it < sch.n; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait(&sm.kv_empty[st], ((uint32_t)(it >> 1) & 1u) ^ 1u, gave_up)) {
+          ok = false;
+          break;
+        }
+        const int j0 = sch.tile(it) * kBN;
+        mbar_arrive_expect_tx(&sm.kv_full[st], kvbytes);
+        tma_load_4d(sm.k[st], &kmap, 0, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.k[st] + kHalf, &kmap, 64, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.v[st], &vmap, 0, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.v[st] + kHalf, &vmap, 64, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        if (sparse)
+          tma_load_4d(sm.k16[st], &k16map, 0, p.k16slot[hidx], j0, b * p.bk, &sm.kv_full[st]);
+        ++n_issued;
+      }
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 41);
+      for (int k = max(0, n_issued - kStages); k < n_issued; ++k)
+        mbar_wait_drain(&sm.kv_full[k & 1], (uint32_t)(k >> 1) & 1u);
+      mbar_wait_drain(&sm.q_full, 0u);
+    }
+    __syncwarp();
+  } else if (warp == 5) {  // ------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.q_full, 0u, gave_up);
+      uint32_t n_pv = 0;
+      // O += P V for tile `it` (its K/V stage is released when the MMAs are done)
+      auto pv = [&](int it) {
+        if (!mbar_wait(&sm.p_full, (uint32_t)it & 1u, gave_up)) return false;
+        tc_fence_after();
+        const int st = it & 1;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(t_o, kdesc(sm.p, kk), vdesc(sm.v[st], kk), kIdescPV, it > 0 || kk > 0);
+        mma_commit(&sm.o_done);
+        mma_commit(&sm.kv_empty[st]);
+        ++n_pv;
+        return true;
+      };
+      for (int it = 0; ok && it < sch.n; ++it) {
+        const int st = it & 1, sb = it & 1;
+        if (!mbar_wait(&sm.kv_full[st], (uint32_t)(it >> 1) & 1u, gave_up) ||
+            !mbar_wait(&sm.s_empty[sb], ((uint32_t)(it >> 1) & 1u) ^ 1u, gave_up) ||
+            (sparse && !mbar_wait(&sm.s16_empty, ((uint32_t)it & 1u) ^ 1u, gave_up))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(t_s + (uint32_t)(sb * kBN), kdesc(sm.q, kk), kdesc(sm.k[st], kk),
+                      kIdescQK, kk > 0);
+        if (sparse)
+          mma_bf16_ss(t_s16, sdesc_k_sw32(smem_u32(sm.q16), 256),
+                      sdesc_k_sw32(smem_u32(sm.k16[st]), 256), kIdescQK, false);
+        mma_commit(&sm.s_full[sb]);
+        if (it > 0 && !pv(it - 1)) ok = false;  // S(it) overlaps the softmax of tile it-1
+      }
+      if (ok && sch.n > 0 && !pv(sch.n - 1)) ok = false;
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 42);
+      if (n_pv > 0) mbar_wait_drain(&sm.o_done, (n_pv - 1) & 1u);
+    }
+    __syncwarp();
+  } else {  // ------------------------------------- softmax: thread = query row
+    const int r = tid;
+    const bool valid = r < nrows;
+    const int64_t P = P0 + r;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    float thr = INFINITY;
+    int64_t jt = -1;
+    if (sparse && valid) {
+      const int64_t ob = ((int64_t)b * p.n_ret + p.slot[hidx]) * p.Lq + m0 + r;
+      thr = p.thr[ob];
+      jt = p.jtie[ob];
+    }
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < sch.n; ++it) {
+      const int sb = it & 1;
+      const int64_t j0 = (int64_t)sch.tile(it) * kBN;
+      ok = ok && mbar_wait_warp(&sm.s_full[sb], (uint32_t)(it >> 1) & 1u, gave_up);
+      tc_fence_after();
+      bool full = false;
+      if (MODE == MODE_DENSE) full = j0 + kBN - 1 <= P;
+      if (MODE == MODE_LOCAL)
+        full = j0 + kBN - 1 <= P && (j0 > P - p.window || j0 + kBN - 1 < p.n_sink);
+      uint32_t keep[4] = {0u, 0u, 0u, 0u};
+      if (ok && sparse) {  // the indexer predicate: s16 > t, or s16 == t and j <= jtie
+        float t16[kBN];
+        tmem_ld128(t_s16 + lane_off, t16);
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) {
+          const float s16 = t16[i] + 0.0f;
+          const int64_t j = j0 + i;
+          const bool kp = j <= P && (s16 > thr || (s16 == thr && j <= jt));
+          keep[i >> 5] |= (kp ? 1u : 0u) << (i & 31);
+        }
+      }
+      // the tile's scores, masked and scaled into the log2 domain
+      float x[kBN];
+      if (ok) tmem_ld128(t_s + lane_off + (uint32_t)(sb * kBN), x);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {  // S (and S16) are in registers: the MMA may reuse the buffers
+        mbar_arrive(&sm.s_empty[sb]);
+        if (sparse) mbar_arrive(&sm.s16_empty);
+      }
+      if (full && ok) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) x[i] *= p.scale_log2;
+      } else {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) {
+          const int64_t j = j0 + i;
+          bool kp;
+          if (MODE == MODE_DENSE) kp = j <= P;
+          else if (MODE == MODE_LOCAL) kp = j <= P && (j < p.n_sink || j > P - p.window);
+          else kp = (keep[i >> 5] >> (i & 31)) & 1u;
+          x[i] = (ok && kp) ? x[i] * p.scale_log2 : -INFINITY;
+        }
+      }
+      float tm[8];  // tile max as a tree (independent chains)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tm[e] = x[e];
+#pragma unroll
+      for (int i = 8; i < kBN; ++i) tm[i & 7] = fmaxf(tm[i & 7], x[i]);
+      const float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
+                               fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
+      const float m_new = fmaxf(m_used, tmax);
+      const bool move = m_new > -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescale);
+      float alpha = 1.f;
+      if (move) {
+        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_new);
+        m_used = m_new;
+        l *= alpha;
+      }
+      // P and O are free once the previous tile's PV MMA is done
+      if (it > 0) ok = ok && mbar_wait_warp(&sm.o_done, (uint32_t)(it - 1) & 1u, gave_up);
+      tc_fence_after();
+      if (ok && it > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(t_o + lane_off + (uint32_t)(c * 32), o);
+        }
+        tmem_wait_st();
+      }
+      // P = 2^(x - m) rounded to bf16 once; row r of P keeps 16-byte chunk q of
+      // its 64-key half at chunk q ^ (r & 7)
+      uint8_t* prow = sm.p + (r >> 3) * 1024 + (r & 7) * 128;
+      const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
+      float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c16 = 0; c16 < 16; ++c16) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = c16 * 8 + 2 * e;
+          pk[e] = pack_bf16x2(ex2_ftz(x[i] - msafe), ex2_ftz(x[i + 1] - msafe));
+          lsum[e] += bf16_lo(pk[e]) + bf16_hi(pk[e]);
+        }
+        const int hf = c16 >> 3, qq = c16 & 7;
+        *reinterpret_cast<uint4*>(prow + hf * kHalf + ((qq ^ (r & 7)) << 4)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
+    }
+    // ---- epilogue: O / l from TMEM, bf16 rows to global
+    if (sch.n > 0) ok = ok && mbar_wait_warp(&sm.o_done, (uint32_t)(sch.n - 1) & 1u, gave_up);
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint16_t* orow = p.o + b * p.o_sb + (int64_t)(m0 + r) * p.o_sl + (int64_t)h * kD;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float o[32];
+      if (sch.n > 0) {
+        tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+      if (valid) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 w;
+          w.x = pack_bf16x2(o[q4 * 8 + 0] * inv, o[q4 * 8 + 1] * inv);
+          w.y = pack_bf16x2(o[q4 * 8 + 2] * inv, o[q4 * 8 + 3] * inv);
+          w.z = pack_bf16x2(o[q4 * 8 + 4] * inv, o[q4 * 8 + 5] * inv);
+          w.w = pack_bf16x2(o[q4 * 8 + 6] * inv, o[q4 * 8 + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = w;
+        }
+      }
+    }
+    if (valid && p.lse != nullptr)
+      p.lse[((int64_t)b * p.H + h) * p.Lq + m0 + r] =
+          l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    if (!ok && r == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 43);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// A bf16 [B][L][heads][width] view as a 4-D TMA map {width, heads, L, B} with
+// boxes of {box0, 1, 128, 1}; a batch stride of 0 (one tensor shared by every
+// batch entry) maps to a single batch coordinate.
+bool encode_view(CUtensorMap* map, const rtp_view& v, int width, int heads, int L, int B,
+                 int box0, int swizzle, int* batch_mult) {
+  const bool shared = v.stride_b == 0 && B > 1;
+  *batch_mult = shared ? 0 : 1;
+  const uint64_t sl = (uint64_t)v.stride_l * 2;
+  const uint64_t sb = !shared && v.stride_b != 0 ? (uint64_t)v.stride_b * 2 : sl * (uint64_t)L;
+  const uint64_t dims[4] = {(uint64_t)width, (uint64_t)heads, (uint64_t)L,
+                            shared ? 1u : (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)width * 2, sl, sb};
+  const uint32_t box[4] = {(uint32_t)box0, 1, 128, 1};
+  return tma_encode_bf16(map, v.ptr, 4, dims, strides, box, swizzle);
+}
+
+template <int MODE>
+rtp_status launch_tc(AttnParams& prm, int n_heads, const rtp_shape* shape, const rtp_view& q,
+                     const rtp_view& k, const rtp_view& v, const rtp_view* q16,
+                     const rtp_view* k16, int n_q16, int n_k16, cudaStream_t s) {
+  const int B = shape->B;
+  if (n_heads == 0 || B == 0 || prm.Lq == 0) return RTP_OK;
+  CUtensorMap qm, km, vm, q16m, k16m;
+  int bq = 1, bk = 1, bv = 1, b16q = 1, b16k = 1;
+  if (!encode_view(&qm, q, kD, shape->H, shape->Lq, B, 64, 128, &bq) ||
+      !encode_view(&km, k, kD, shape->Hkv, shape->Lk, B, 64, 128, &bk) ||
+      !encode_view(&vm, v, kD, shape->Hkv, shape->Lk, B, 64, 128, &bv))
+    return RTP_ERR_CUDA;
+  if (MODE == MODE_SPARSE) {
+    if (!encode_view(&q16m, *q16, kR, n_q16, shape->Lq, B, kR, 32, &b16q) ||
+        !encode_view(&k16m, *k16, kR, n_k16, shape->Lk, B, kR, 32, &b16k))
+      return RTP_ERR_CUDA;
+    if (b16q != bq || b16k != bk) return RTP_ERR_UNSUPPORTED;  // one batch rule per side
+  } else {
+    q16m = qm;
+    k16m = km;
+  }
+  if (bk != bv) return RTP_ERR_UNSUPPORTED;
+  prm.bq = bq;
+  prm.bk = bk;
+  const size_t smem = sizeof(TcSmem) + 1024;
+  if (cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  dim3 grid((prm.Lq + kBM - 1) / kBM, n_heads, B);
+  if (grid.y > 65535 || grid.z > 65535) return RTP_ERR_UNSUPPORTED;
+  static const char* kName[3] = {"attn_prefill_dense", "attn_prefill_local",
+                                 "attn_prefill_sparse"};
+  TraceScope tr(kName[MODE], s);
+  attn_tc_kernel<MODE><<<grid, kThreads, smem, s>>>(qm, km, vm, q16m, k16m, prm);
+  return check_cuda(cudaGetLastError());
+}
+
+void fill_common(AttnParams& prm, const rtp_shape* shape, const rtp_view& o, float* lse,
+                 float softmax_scale, void* ws) {
+  memset(&prm, 0, sizeof(prm));
+  prm.o = static_cast<uint16_t*>(o.ptr);
+  prm.o_sb = o.stride_b;
+  prm.o_sl = o.stride_l;
+  prm.lse = lse;
+  prm.status = static_cast<DevStatus*>(ws);
+  prm.Lq = shape->Lq;
+  prm.Lk = shape->Lk;
+  prm.H = shape->H;
+  prm.G = shape->H / shape->Hkv;
+  prm.q_pos0 = shape->q_pos0;
+  prm.scale_log2 = softmax_scale * kLog2e;
+}
+
+}  // namespace
+
+// Entry points used by the C ABI (decode dispatch lives in decode.cu).
+rtp_status prefill_local(const rtp_shape* shape, const HeadMap& hm, int window, int n_sink,
+                         const rtp_view& q, const rtp_view& k, const rtp_view& v,
+                         float scale, const rtp_view& o, float* lse, void* ws, cudaStream_t s) {
+  AttnParams prm;
+  fill_common(prm, shape, o, lse, scale, ws);
+  prm.window = window;
+  prm.n_sink = n_sink;
+  int n = 0;
+  for (int r = 0; r < hm.n_lkv; ++r)
+    for (int j = 0; j < hm.G; ++j) prm.head[n++] = (int16_t)(hm.lkv[r] * hm.G + j);
+  return launch_tc<MODE_LOCAL>(prm, n, shape, q, k, v, nullptr, nullptr, 0, 0, s);
+}
+
+rtp_status prefill_dense(const rtp_shape* shape, const rtp_view& q, const rtp_view& k,
+                         const rtp_view& v, float scale, const rtp_view& o, float* lse,
+                         void* ws, cudaStream_t s) {
+  AttnParams prm;
+  fill_common(prm, shape, o, lse, scale, ws);
+  for (int h = 0; h < shape->H; ++h) prm.head[h] = (int16_t)h;
+  return launch_tc<MODE_DENSE>(prm, shape->H, shape, q, k, v, nullptr, nullptr, 0, 0, s);
+}
+
+rtp_status prefill_sparse(const rtp_shape* shape, const HeadMap& hm, const rtp_view& q,
+                          const rtp_view& k, const rtp_view& v, const rtp_view& q16,
+                          const rtp_view& k16, const float* thr, const int32_t* jtie,
+                          float scale, const rtp_view& o, float* lse, void* ws, cudaStream_t s) {
+  AttnParams prm;
+  fill_common(prm, shape, o, lse, scale, ws);
+  prm.thr = thr;
+  prm.jtie = jtie;
+  prm.n_ret = hm.n_ret;
+  for (int hr = 0; hr < hm.n_ret; ++hr) {
+    prm.head[hr] = hm.ret_q[hr];
+    prm.slot[hr] = (int16_t)hr;
+    prm.k16slot[hr] = hm.ret_k16[hr];
+  }
+  return launch_tc<MODE_SPARSE>(prm, hm.n_ret, shape, q, k, v, &q16, &k16, hm.n_ret, hm.H_k16,
+                                s);
+}
+
+}  // namespace rtp

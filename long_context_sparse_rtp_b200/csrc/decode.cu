@@ -24,13 +24,13 @@
 namespace rtp {
 
 rtp_status prefill_local(const rtp_shape*, const HeadMap&, int, int, const rtp_view&,
-                         const rtp_view&, const rtp_view&, float, const rtp_view&, float*,
+                         const rtp_view&, const rtp_view&, float, const rtp_view&, float*, void*,
                          cudaStream_t);
 rtp_status prefill_dense(const rtp_shape*, const rtp_view&, const rtp_view&, const rtp_view&,
-                         float, const rtp_view&, float*, cudaStream_t);
+                         float, const rtp_view&, float*, void*, cudaStream_t);
 rtp_status prefill_sparse(const rtp_shape*, const HeadMap&, const rtp_view&, const rtp_view&,
                           const rtp_view&, const rtp_view&, const rtp_view&, const float*,
-                          const int32_t*, float, const rtp_view&, float*, cudaStream_t);
+                          const int32_t*, float, const rtp_view&, float*, void*, cudaStream_t);
 
 namespace {
 
@@ -565,7 +565,7 @@ extern "C" rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_r
     return decode_range(shape, hm.lkv, hm.n_lkv, window, n_sink, q, k, v, softmax_scale, o, lse,
                         ws, ws_bytes, s);
   }
-  return prefill_local(shape, hm, window, n_sink, q, k, v, softmax_scale, o, lse, s);
+  return prefill_local(shape, hm, window, n_sink, q, k, v, softmax_scale, o, lse, ws, s);
 }
 
 extern "C" rtp_status rtp_dense_attn(const rtp_shape* shape, rtp_view q, rtp_view k, rtp_view v,
@@ -591,7 +591,7 @@ extern "C" rtp_status rtp_dense_attn(const rtp_shape* shape, rtp_view q, rtp_vie
     return decode_range(shape, kvh, shape->Hkv, window, 0, q, k, v, softmax_scale, o, lse, ws,
                         ws_bytes, s);
   }
-  return prefill_dense(shape, q, k, v, softmax_scale, o, lse, s);
+  return prefill_dense(shape, q, k, v, softmax_scale, o, lse, ws, s);
 }
 
 extern "C" rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint8_t* kv_role,
@@ -617,7 +617,7 @@ extern "C" rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint
   if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
   if ((st = check_view(k16, hm.H_k16, kR, true)) != RTP_OK) return st;
   if (ws == nullptr || ws_bytes < kStatusBytes) return RTP_ERR_WORKSPACE_TOO_SMALL;
-  return prefill_sparse(shape, hm, q, k, v, q16, k16, thr, jtie, softmax_scale, o, lse,
+  return prefill_sparse(shape, hm, q, k, v, q16, k16, thr, jtie, softmax_scale, o, lse, ws,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 

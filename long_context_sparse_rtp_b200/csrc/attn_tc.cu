@@ -16,7 +16,8 @@
 // issues S = Q K^T (8 MMAs, K = 16 each) into one of two TMEM score buffers and
 // O += P V into a TMEM accumulator; warps 0-3 hold one query row per thread:
 // read the scores with tcgen05.ld, mask, online softmax in the log2 domain,
-// write P (bf16) to shared memory for the PV MMA.  The running max is only
+// write P (bf16, two per column) over the scores in TMEM, where the PV MMA
+// reads it as its A operand.  The running max is only
 // moved (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles
 // need no rescale.  P is rounded to bf16 once and the normaliser sums the
 // rounded values, so the output is an exact convex combination of them.
@@ -61,11 +62,12 @@ struct TcSmem {                      // placed on a 1024-byte boundary
   uint8_t q[kTile];                  // [2 halves of 64 dims][128 rows][128 B]
   uint8_t k[kStages][kTile];
   uint8_t v[kStages][kTile];         // rows = keys, 2 halves of 64 dims (MN-major B)
-  uint8_t p[kTile];                  // [2 halves of 64 keys][128 rows][128 B]
   uint8_t q16[kBM * kR * 2];         // 32-byte rows, 32-byte swizzle
   uint8_t k16[kStages][kBN * kR * 2];
-  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], s16_empty,
-      p_full, o_done;
+  // per-tile barriers with several arriving warps come in pairs by tile parity:
+  // a warp may run one tile ahead of another, never two
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], s16_empty[2],
+      p_full[2], o_done[2];
   uint32_t tmem_base;
   int gave_up;
 };
@@ -146,11 +148,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_empty[i], 4);
+      mbar_init(&sm.s_empty[i], 1);  // committed once the PV MMA reading P from it is done
+      mbar_init(&sm.o_done[i], 1);   // PV MMAs of tiles with this parity
+      mbar_init(&sm.s16_empty[i], 4);
+      mbar_init(&sm.p_full[i], 4);
     }
-    mbar_init(&sm.s16_empty, 4);
-    mbar_init(&sm.p_full, 4);
-    mbar_init(&sm.o_done, 1);
     sm.gave_up = 0;
     fence_mbar_init();
   }
@@ -201,24 +203,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       bool ok = mbar_wait(&sm.q_full, 0u, gave_up);
       uint32_t n_pv = 0;
-      // O += P V for tile `it` (its K/V stage is released when the MMAs are done)
+      // O += P V for tile `it`, P read from TMEM (its score buffer); the K/V stage
+      // and the score buffer are released when the MMAs are done
       auto pv = [&](int it) {
-        if (!mbar_wait(&sm.p_full, (uint32_t)it & 1u, gave_up)) return false;
+        if (!mbar_wait(&sm.p_full[it & 1], (uint32_t)(it >> 1) & 1u, gave_up)) return false;
         tc_fence_after();
-        const int st = it & 1;
+        const int st = it & 1, sb = it & 1;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ss(t_o, kdesc(sm.p, kk), vdesc(sm.v[st], kk), kIdescPV, it > 0 || kk > 0);
-        mma_commit(&sm.o_done);
+          mma_bf16_ts(t_o, t_s + (uint32_t)(sb * kBN + kk * 8), vdesc(sm.v[st], kk), kIdescPV,
+                      it > 0 || kk > 0);
+        mma_commit(&sm.o_done[it & 1]);
+        mma_commit(&sm.s_empty[sb]);
         mma_commit(&sm.kv_empty[st]);
         ++n_pv;
         return true;
       };
       for (int it = 0; ok && it < sch.n; ++it) {
         const int st = it & 1, sb = it & 1;
+        // S16 of tile it-1 must have been read before S16 of tile it overwrites it
         if (!mbar_wait(&sm.kv_full[st], (uint32_t)(it >> 1) & 1u, gave_up) ||
             !mbar_wait(&sm.s_empty[sb], ((uint32_t)(it >> 1) & 1u) ^ 1u, gave_up) ||
-            (sparse && !mbar_wait(&sm.s16_empty, ((uint32_t)it & 1u) ^ 1u, gave_up))) {
+            (sparse && it > 0 &&
+             !mbar_wait(&sm.s16_empty[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u, gave_up))) {
           ok = false;
           break;
         }
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && sch.n > 0 && !pv(sch.n - 1)) ok = false;
       if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 42);
-      if (n_pv > 0) mbar_wait_drain(&sm.o_done, (n_pv - 1) & 1u);
+      if (n_pv > 0) mbar_wait_drain(&sm.o_done[(n_pv - 1) & 1u], ((n_pv - 1) >> 1) & 1u);
     }
     __syncwarp();
   } else {  // ------------------------------------- softmax: thread = query row
@@ -261,39 +268,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (MODE == MODE_DENSE) full = j0 + kBN - 1 <= P;
       if (MODE == MODE_LOCAL)
         full = j0 + kBN - 1 <= P && (j0 > P - p.window || j0 + kBN - 1 < p.n_sink);
-      uint32_t keep[4] = {0u, 0u, 0u, 0u};
-      if (ok && sparse) {  // the indexer predicate: s16 > t, or s16 == t and j <= jtie
-        float t16[kBN];
-        tmem_ld128(t_s16 + lane_off, t16);
-#pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const float s16 = t16[i] + 0.0f;
-          const int64_t j = j0 + i;
-          const bool kp = j <= P && (s16 > thr || (s16 == thr && j <= jt));
-          keep[i >> 5] |= (kp ? 1u : 0u) << (i & 31);
-        }
-      }
       // the tile's scores, masked and scaled into the log2 domain
       float x[kBN];
-      if (ok) tmem_ld128(t_s + lane_off + (uint32_t)(sb * kBN), x);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {  // S (and S16) are in registers: the MMA may reuse the buffers
-        mbar_arrive(&sm.s_empty[sb]);
-        if (sparse) mbar_arrive(&sm.s16_empty);
-      }
-      if (full && ok) {
+      if (sparse) {
+        // the indexer predicate per 32-key chunk: s16 > t, or s16 == t and j <= jtie;
+        // key offsets i within the tile: i <= ptl (causal), i <= jtl (may keep a tie);
+        // -0 and +0 compare equal, so the scores need no canonical form here
+        auto clamp_off = [](int64_t d) {
+          return (int)(d < -1 ? -1 : (d > kBN - 1 ? kBN - 1 : d));
+        };
+        const int ptl = clamp_off(P - j0), jtl = clamp_off(jt - j0);
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) x[i] *= p.scale_log2;
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r16[32], rs[32];
+          if (ok) {
+            tmem_ld32_nowait(t_s16 + lane_off + (uint32_t)(c * 32), r16);
+            tmem_ld32_nowait(t_s + lane_off + (uint32_t)(sb * kBN + c * 32), rs);
+            tmem_wait_ld();
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            reg_fence(r16[i]);
+            reg_fence(rs[i]);
+            const int ii = c * 32 + i;
+            const float s16 = __uint_as_float(r16[i]);
+            // bitwise, not short-circuit: a select per key, no divergent branch
+            const bool kp = ok & ((s16 > thr) | ((s16 == thr) & (ii <= jtl))) & (ii <= ptl);
+            x[ii] = kp ? __uint_as_float(rs[i]) * p.scale_log2 : -INFINITY;
+          }
+        }
+        tc_fence_before();  // S16 is in registers: the MMA may reuse its buffer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s16_empty[it & 1]);
       } else {
+        if (ok) tmem_ld128(t_s + lane_off + (uint32_t)(sb * kBN), x);
+        if (full && ok) {
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const int64_t j = j0 + i;
-          bool kp;
-          if (MODE == MODE_DENSE) kp = j <= P;
-          else if (MODE == MODE_LOCAL) kp = j <= P && (j < p.n_sink || j > P - p.window);
-          else kp = (keep[i >> 5] >> (i & 31)) & 1u;
-          x[i] = (ok && kp) ? x[i] * p.scale_log2 : -INFINITY;
+          for (int i = 0; i < kBN; ++i) x[i] *= p.scale_log2;
+        } else {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) {
+            const int64_t j = j0 + i;
+            bool kp;
+            if (MODE == MODE_DENSE) kp = j <= P;
+            else kp = (j <= P) & ((j < p.n_sink) | (j > P - p.window));
+            x[i] = (ok & kp) ? x[i] * p.scale_log2 : -INFINITY;
+          }
         }
       }
       float tm[8];  // tile max as a tree (independent chains)
@@ -304,53 +324,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
                                fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
       const float m_new = fmaxf(m_used, tmax);
-      const bool move = m_new > -INFINITY && (m_used == -INFINITY || m_new > m_used + kRescale);
+      const bool first = m_used == -INFINITY && m_new > -INFINITY;  // O and l are still 0
+      const bool move = m_used > -INFINITY && m_new > m_used + kRescale;
       float alpha = 1.f;
+      if (first) m_used = m_new;
       if (move) {
-        alpha = (m_used == -INFINITY) ? 0.f : exp2f(m_used - m_new);
+        alpha = exp2f(m_used - m_new);
         m_used = m_new;
         l *= alpha;
       }
-      // P and O are free once the previous tile's PV MMA is done
-      if (it > 0) ok = ok && mbar_wait_warp(&sm.o_done, (uint32_t)(it - 1) & 1u, gave_up);
-      tc_fence_after();
-      if (ok && it > 0 && __any_sync(0xffffffffu, move)) {
+      // O is rescaled (rarely) once the previous tile's PV MMA is done
+      if (it > 0 && __any_sync(0xffffffffu, move)) {
+        ok = ok && mbar_wait_warp(&sm.o_done[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u,
+                                  gave_up);
+        tc_fence_after();
+        if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float o[32];
-          tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(t_o + lane_off + (uint32_t)(c * 32), o);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(t_o + lane_off + (uint32_t)(c * 32), o);
+          }
         }
-        tmem_wait_st();
       }
-      // P = 2^(x - m) rounded to bf16 once; row r of P keeps 16-byte chunk q of
-      // its 64-key half at chunk q ^ (r & 7)
-      uint8_t* prow = sm.p + (r >> 3) * 1024 + (r & 7) * 128;
+      // P = 2^(x - m) rounded to bf16 once, packed two per column over the scores
       const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
       float lsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c16 = 0; c16 < 16; ++c16) {
-        uint32_t pk[4];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = c16 * 8 + 2 * e;
+        for (int e = 0; e < 32; ++e) {
+          const int i = h2 * 64 + 2 * e;
           pk[e] = pack_bf16x2(ex2_ftz(x[i] - msafe), ex2_ftz(x[i + 1] - msafe));
-          lsum[e] += bf16_lo(pk[e]) + bf16_hi(pk[e]);
+          lsum[e & 3] += bf16_lo(pk[e]) + bf16_hi(pk[e]);
         }
-        const int hf = c16 >> 3, qq = c16 & 7;
-        *reinterpret_cast<uint4*>(prow + hf * kHalf + ((qq ^ (r & 7)) << 4)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (ok) tmem_st32u(t_s + lane_off + (uint32_t)(sb * kBN + h2 * 32), pk);
       }
+      tmem_wait_st();
       l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
-      fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full);
+      if (lane == 0) mbar_arrive(&sm.p_full[it & 1]);
     }
     // ---- epilogue: O / l from TMEM, bf16 rows to global
-    if (sch.n > 0) ok = ok && mbar_wait_warp(&sm.o_done, (uint32_t)(sch.n - 1) & 1u, gave_up);
+    if (sch.n > 0)
+      ok = ok && mbar_wait_warp(&sm.o_done[(sch.n - 1) & 1], (uint32_t)((sch.n - 1) >> 1) & 1u,
+                                gave_up);
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     uint16_t* orow = p.o + b * p.o_sb + (int64_t)(m0 + r) * p.o_sl + (int64_t)h * kD;

@@ -444,10 +444,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           float e[kChunk];
 #pragma unroll
           for (int i = 0; i < kChunk; ++i) {
-            const bool in = full || (int64_t)(j0 + i) <= P;
+            const bool in = full | ((int64_t)(j0 + i) <= P);
             const float s = v[i];
             e[i] = in ? rel_w(s, m) : 0.f;
-            if (in && s >= c0) {  // the few keys in [c0, m]
+            if (in & (s >= c0)) {  // the few keys in [c0, m]
               const int bb = bin0_of(s, m, scale);
               atomicAdd(&sm.wacc[bb][r], fixed21(__fmul_rn(e[i], sm.t.tab[bb][r])));
               atomicAdd(&sm.hc[bb][r], 1u);
@@ -515,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int i = 0; i < kChunk; ++i) {
               const float s = v[i];
-              const bool h = mine && s >= lo && s <= hi && (full || (int64_t)(j0 + i) <= P);
+              const bool h = mine & (s >= lo) & (s <= hi) & (full | ((int64_t)(j0 + i) <= P));
               hits |= (h ? 1u : 0u) << i;
             }
             if (__ballot_sync(0xffffffffu, hits != 0u) == 0u) return;

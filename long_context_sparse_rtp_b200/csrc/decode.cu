@@ -530,6 +530,10 @@ extern "C" size_t rtp_workspace_size(rtp_op op, const rtp_shape* shape, const ui
     case RTP_OP_SPARSE_DECODE:
       if (!have_roles) return kStatusBytes;
       return decode_ws_layout(shape, hm).total;
+    case RTP_OP_TOPP_SELECT: {
+      const size_t t = select_ws_layout().total;
+      return t > 0 ? t : kStatusBytes;
+    }
     case RTP_OP_LOCAL:
     case RTP_OP_DENSE: {
       if (shape->Lq != 1) return kStatusBytes;

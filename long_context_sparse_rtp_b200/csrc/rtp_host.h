@@ -120,6 +120,12 @@ constexpr int kDecMaxSplits = 256;     // split-KV partials per (batch, kv head)
 
 constexpr int kDecSub = 64;            // sub-bins of a row's crossing bin
 
+struct SelectWs {   // prefill top-p selection (select_prefill.cu)
+  size_t mask, lists, total;
+  int n_sm;
+};
+SelectWs select_ws_layout();
+
 struct DecodeWs {   // retrieval decode
   size_t scores, hist_m, hist_c, flags, sub_m, sub_c, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
       part, mcount, total;

@@ -57,9 +57,13 @@ constexpr unsigned long long kIdxMask = (1ull << kIdxBits) - 1;
 constexpr int kKeyBits = 32 + kIdxBits;  // 53
 constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 
-enum { ST_IDLE = 0, ST_REFINE = 1, ST_COLLECT = 2, ST_DONE = 3 };
+enum { ST_IDLE = 0, ST_REFINE = 1, ST_COLLECT = 2, ST_DONE = 3, ST_LIST = 4 };
+constexpr int kListCap = 1024;   // crossing-bin keys a row may park in its global list
 
 struct SelParams {
+  unsigned long long* lists;  // [slots][kBM][kListCap] crossing-bin keys, or null
+  uint32_t* slot_mask;        // [SMs]: bit b = slot 2 sm + b in use
+  int n_sm;
   int Lq;
   int64_t q_pos0;
   int n_ret;
@@ -96,6 +100,7 @@ struct SelSmem {
   uint32_t tmem_base;
   int go;
   int gave_up;
+  int slot;  // this CTA's candidate-list slot, -1 if none
 };
 
 __device__ __forceinline__ float ex2_ftz(float x) {
@@ -199,11 +204,12 @@ __device__ __forceinline__ float max16(const float (&v)[kChunk]) {
 
 // Processes the first n (<= 32) queued prefilter hits of this warp, one per
 // lane: the exact crossing-bin and prefix tests of the owning row (whose state
-// is fetched from the owner lane), then a candidate or a digit count.  Called by
-// all 32 lanes.
-__device__ __noinline__ void drain_hits(SelSmem& sm, int wq, int n, int row0, float m, float scale,
-                                        int k0, int pbits, unsigned long long prefix, int w,
-                                        float tk, int collect) {
+// is fetched from the owner lane), then a candidate (collect = 1), a key parked
+// in the row's global list (collect = 2) or a digit count (collect = 0).  Called
+// by all 32 lanes.
+__device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, int wq, int n,
+                                        int row0, float m, float scale, int k0, int pbits,
+                                        unsigned long long prefix, int w, float tk, int collect) {
   const int lane = threadIdx.x & 31;
   const bool has = lane < n;
   const float s = has ? sm.t.q.s[wq][lane] : 0.f;
@@ -223,7 +229,10 @@ __device__ __noinline__ void drain_hits(SelSmem& sm, int wq, int n, int row0, fl
   const unsigned long long opx = ((unsigned long long)oph << 32) | opl;
   if (opb > 0 && (ck >> (kKeyBits - opb)) != opx) return;
   const int r = row0 + owner;
-  if (ocol) {
+  if (ocol == 2) {  // park the key in the row's global list
+    const int slot_c = atomicAdd(&sm.ncnt[r], 1);
+    if (slot_c < kListCap) list[(size_t)r * kListCap + slot_c] = ck;
+  } else if (ocol) {
     const int slot_c = atomicAdd(&sm.ncnt[r], 1);
     if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
   } else {
@@ -286,6 +295,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     sm.gave_up = 0;
     sm.go = 0;
     fence_mbar_init();
+    // a candidate-list slot of this SM (at most two CTAs are resident per SM)
+    sm.slot = -1;
+    if (p.lists != nullptr) {
+      uint32_t smid;
+      asm volatile("mov.u32 %0, %%smid;\n" : "=r"(smid));
+      if ((int)smid < p.n_sm)
+        for (int b2 = 0; b2 < 2 && sm.slot < 0; ++b2)
+          if ((atomicOr(&p.slot_mask[smid], 1u << b2) & (1u << b2)) == 0u)
+            sm.slot = (int)smid * 2 + b2;
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, 2 * kBN);
@@ -467,7 +486,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     unsigned long long inner = 0ull, prefix = 0ull;
     uint32_t cnt_above = 0u;
     int k0 = 0, pbits = 0, state = ST_IDLE;
+    uint32_t n_cur = 0u;  // keys of the current crossing range
     float tk = 0.f;  // exp(k0 / scale)
+    unsigned long long* const lists =
+        sm.slot >= 0 ? p.lists + (size_t)sm.slot * kBM * kListCap : nullptr;
+    // a row whose crossing range holds <= kCap keys collects them; <= kListCap
+    // parks them in its global list once; more refines the range by a full sweep
+    auto next_state = [&](uint32_t n) {
+      if (n <= (uint32_t)kCap || pbits >= kKeyBits) return (int)ST_COLLECT;
+      return (lists != nullptr && n <= (uint32_t)kListCap) ? (int)ST_LIST : (int)ST_REFINE;
+    };
     if (valid) {
       T = (double)p.p * Z;
       uint32_t n_in = 0u;
@@ -483,14 +511,60 @@ __global__ void __launch_bounds__(kThreads, 2)
           ((unsigned long long)score_key(hi_s + margin) << kIdxBits) | kIdxMask;
       pbits = (kl == kh) ? kKeyBits : (__clzll(kl ^ kh) - (64 - kKeyBits));
       prefix = pbits > 0 ? (kh >> (kKeyBits - pbits)) : 0ull;
-      state = (n_in <= (uint32_t)kCap) ? ST_COLLECT : ST_REFINE;
+      n_cur = n_in;
+      state = next_state(n_in);
     }
     ebar();
     if (g == 0) clear_row(sm, r);
 
+    // sort the row's <= kCap candidates (smem) and walk them to the exact cut
+    auto finish_row = [&]() {
+      int n = sm.ncnt[r];
+      if (n > kCap) {
+        set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 11);
+        n = kCap;
+      }
+      const int i = m0 + r;
+      const int64_t o = ((int64_t)b * p.n_ret + hr) * p.Lq + i;
+      if (n == 0) {  // cannot happen for a consistent histogram; keep every key
+        set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 15);
+        p.thr[o] = -INFINITY;
+        p.jtie[o] = (int32_t)P;
+        p.count[o] = (int32_t)(P + 1);
+        if (p.mass) p.mass[o] = 1.f;
+        return;
+      }
+      for (int a = 1; a < n; ++a) {  // insertion sort, descending
+        const unsigned long long x = sm.u.cand[a][r];
+        int q = a - 1;
+        while (q >= 0 && sm.u.cand[q][r] < x) {
+          sm.u.cand[q + 1][r] = sm.u.cand[q][r];
+          --q;
+        }
+        sm.u.cand[q + 1][r] = x;
+      }
+      unsigned long long acc = inner;
+      double cum = base;
+      int take = n;
+      for (int a = 0; a < n; ++a) {
+        const float sa = key_score((uint32_t)(sm.u.cand[a][r] >> kIdxBits));
+        acc += fixed21(__fmul_rn(rel_w(sa, m), tk));
+        cum = base + fk * (double)acc;
+        if (cum >= T) {
+          take = a + 1;
+          break;
+        }
+      }
+      const unsigned long long last = sm.u.cand[take - 1][r];
+      p.thr[o] = key_score((uint32_t)(last >> kIdxBits));
+      p.jtie[o] = (int32_t)(kIdxMask - (last & kIdxMask));
+      p.count[o] = (int32_t)(cnt_above + (uint32_t)take);
+      if (p.mass) p.mass[o] = (float)(cum / Z);
+    };
+
     // ---- sweeps 3+: refine the crossing bin 5 bits at a time, then collect
     for (int iter = 0;; ++iter) {
-      const bool mine = state == ST_REFINE || state == ST_COLLECT;
+      const bool mine = state == ST_REFINE || state == ST_COLLECT || state == ST_LIST;
       if (g == 0) sm.ncnt[r] = 0;
       bool any = bar_or(1, kEpi, mine);
       if (any && iter >= kMaxIter) {
@@ -503,7 +577,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (!any) break;
       const int w = min(kDigit, kKeyBits - pbits);
-      const bool collect = state == ST_COLLECT;
+      const int collect = state == ST_COLLECT ? 1 : (state == ST_LIST ? 2 : 0);
       float lo = 0.f, hi = -1.f;
       if (mine) refine_range(m, scale, k0, pbits, prefix, lo, hi);
       const int wq = warp, row0 = (warp & 3) * 32;
@@ -533,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               qn += __popc(bal);
               if (qn >= 32) {
                 __syncwarp();
-                drain_hits(sm, wq, 32, row0, m, scale, k0, pbits, prefix, w, tk, collect);
+                drain_hits(sm, lists, wq, 32, row0, m, scale, k0, pbits, prefix, w, tk, collect);
                 __syncwarp();
                 if (lane + 32 < qn) {
                   sm.t.q.s[wq][lane] = sm.t.q.s[wq][lane + 32];
@@ -547,55 +621,15 @@ __global__ void __launch_bounds__(kThreads, 2)
           true, state == ST_REFINE);
       if (qn > 0) {  // the last partial batch (row histograms flush below)
         __syncwarp();
-        drain_hits(sm, wq, qn, row0, m, scale, k0, pbits, prefix, w, tk, collect);
+        drain_hits(sm, lists, wq, qn, row0, m, scale, k0, pbits, prefix, w, tk, collect);
       }
       ebar();
       if (state == ST_REFINE && g == 0) flush_row(sm, r);
       ebar();
+      // the list length of a row that parked its crossing range this sweep
+      const int nl = state == ST_LIST ? min(sm.ncnt[r], kListCap) : 0;
       if (state == ST_COLLECT) {
-        if (g == 0) {
-          int n = sm.ncnt[r];
-          if (n > kCap) {
-            set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 11);
-            n = kCap;
-          }
-          const int i = m0 + r;
-          const int64_t o = ((int64_t)b * p.n_ret + hr) * p.Lq + i;
-          if (n == 0) {  // cannot happen for a consistent histogram; keep every key
-            set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 15);
-            p.thr[o] = -INFINITY;
-            p.jtie[o] = (int32_t)P;
-            p.count[o] = (int32_t)(P + 1);
-            if (p.mass) p.mass[o] = 1.f;
-          } else {
-            for (int a = 1; a < n; ++a) {  // insertion sort, descending
-              const unsigned long long x = sm.u.cand[a][r];
-              int q = a - 1;
-              while (q >= 0 && sm.u.cand[q][r] < x) {
-                sm.u.cand[q + 1][r] = sm.u.cand[q][r];
-                --q;
-              }
-              sm.u.cand[q + 1][r] = x;
-            }
-            unsigned long long acc = inner;
-            double cum = base;
-            int take = n;
-            for (int a = 0; a < n; ++a) {
-              const float sa = key_score((uint32_t)(sm.u.cand[a][r] >> kIdxBits));
-              acc += fixed21(__fmul_rn(rel_w(sa, m), tk));
-              cum = base + fk * (double)acc;
-              if (cum >= T) {
-                take = a + 1;
-                break;
-              }
-            }
-            const unsigned long long last = sm.u.cand[take - 1][r];
-            p.thr[o] = key_score((uint32_t)(last >> kIdxBits));
-            p.jtie[o] = (int32_t)(kIdxMask - (last & kIdxMask));
-            p.count[o] = (int32_t)(cnt_above + (uint32_t)take);
-            if (p.mass) p.mass[o] = (float)(cum / Z);
-          }
-        }
+        if (g == 0) finish_row();
         state = ST_DONE;
       } else if (state == ST_REFINE) {
         uint32_t n_in = 0u;
@@ -604,14 +638,65 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int digit = (1 << w) - 1 - bsel;
         prefix = (prefix << w) | (unsigned long long)digit;
         pbits += w;
-        state = (n_in <= (uint32_t)kCap || pbits >= kKeyBits) ? ST_COLLECT : ST_REFINE;
+        n_cur = n_in;
+        state = next_state(n_in);
       }
       ebar();
       if (g == 0 && state == ST_REFINE) clear_row(sm, r);
+      // rows with a parked list: the remaining radix levels run over the list
+      const bool lst = state == ST_LIST;
+      const unsigned long long* my = lst ? lists + (size_t)r * kListCap : nullptr;
+      for (;;) {
+        const bool need = lst && n_cur > (uint32_t)kCap && pbits < kKeyBits;
+        if (!bar_or(1, kEpi, need)) break;
+        const int wl = min(kDigit, kKeyBits - pbits);
+        if (need) {
+          for (int e = g; e < nl; e += 2) {
+            const unsigned long long ck = my[e];
+            if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) continue;
+            const int digit = (int)((ck >> (kKeyBits - pbits - wl)) & ((1ull << wl) - 1));
+            const int bin = (1 << wl) - 1 - digit;
+            const float sc = key_score((uint32_t)(ck >> kIdxBits));
+            atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(sc, m), tk)));
+            atomicAdd(&sm.hc[bin][r], 1u);
+          }
+        }
+        ebar();
+        if (need && g == 0) flush_row(sm, r);
+        ebar();
+        if (need) {
+          uint32_t n_in = 0u;
+          auto fd = [&](int) { return fk; };
+          const int bsel = crossing(sm, r, 1 << wl, T, false, fd, base, inner, cnt_above, n_in);
+          prefix = (prefix << wl) | (unsigned long long)((1 << wl) - 1 - bsel);
+          pbits += wl;
+          n_cur = n_in;
+        }
+        ebar();
+        if (need && g == 0) clear_row(sm, r);
+      }
+      if (g == 0 && lst) sm.ncnt[r] = 0;
+      ebar();
+      if (lst)  // the final range's keys become the row's candidates
+        for (int e = g; e < nl; e += 2) {
+          const unsigned long long ck = my[e];
+          if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) continue;
+          const int slot_c = atomicAdd(&sm.ncnt[r], 1);
+          if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
+        }
+      ebar();
+      if (lst) {
+        if (g == 0) finish_row();
+        state = ST_DONE;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (tid == 0 && sm.slot >= 0) {  // the list slot is free again
+    __threadfence();
+    atomicAnd(&p.slot_mask[sm.slot >> 1], ~(1u << (sm.slot & 1)));
+  }
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 2 * kBN);
@@ -635,6 +720,26 @@ __global__ void topp_all_kernel(int n_ret, int Lq, int64_t q_pos0, int B, float*
 }  // namespace
 }  // namespace rtp
 
+namespace rtp {
+// Workspace of rtp_topp_select: the status word, one slot-occupancy word per SM
+// and two candidate-list slots per SM of kBM x kListCap composite keys.
+SelectWs select_ws_layout() {
+  SelectWs w{};
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n_sm <= 0) {
+    cudaGetLastError();
+    return w;  // total 0: lists off
+  }
+  w.n_sm = n_sm;
+  w.mask = kStatusBytes;
+  w.lists = w.mask + (((size_t)n_sm * 4 + 255) / 256) * 256;
+  w.total = w.lists + (size_t)2 * n_sm * kBM * kListCap * 8;
+  return w;
+}
+}  // namespace rtp
+
 using namespace rtp;
 
 extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_role,
@@ -654,6 +759,7 @@ extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_
   if (thr == nullptr || jtie == nullptr || count == nullptr) return RTP_ERR_INVALID_ARG;
   if (ws == nullptr || ws_bytes < kStatusBytes) return RTP_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const SelectWs wl = select_ws_layout();
   if (p >= 1.f) {
     TraceScope tr("topp_all", s);
     topp_all_kernel<<<592, 256, 0, s>>>(hm.n_ret, shape->Lq, shape->q_pos0, shape->B, thr,
@@ -663,6 +769,13 @@ extern "C" rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_
   if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
   if ((st = check_view(k16, hm.H_k16, kR, true)) != RTP_OK) return st;
   SelParams prm;
+  // with a full-size workspace, rows may park dense crossing bins in lists
+  const bool with_lists = wl.total > 0 && ws_bytes >= wl.total;
+  prm.lists = with_lists ? reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + wl.lists)
+                         : nullptr;
+  prm.slot_mask = with_lists ? reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + wl.mask)
+                             : nullptr;
+  prm.n_sm = wl.n_sm;
   prm.Lq = shape->Lq;
   prm.q_pos0 = shape->q_pos0;
   prm.n_ret = hm.n_ret;

@@ -118,8 +118,10 @@ RTP_API rtp_status rtp_workspace_init(void* ws, size_t ws_bytes, rtp_stream_t st
  * with fp32 accumulation and one round-to-nearest-even to bf16.  Shapes: q has
  * shape->Lq rows of H heads, k has shape->Lk rows of Hkv heads (either count may
  * be 0 to skip that half).  Wq16 [H_ret][128][16], Wk16 [H_k16][128][16] bf16,
- * contiguous.  Decode appends the new key by passing views offset to the new row.
- * No workspace.
+ * contiguous and 16-byte aligned (else RTP_ERR_ALIGNMENT).  The fp32 sum runs
+ * in one fixed order for every call, so a key's k16 is the same whether it is
+ * projected in a prefill or appended in a decode step.  Decode appends the new
+ * key by passing views offset to the new row.  No workspace.
  */
 RTP_API rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv_role,
                             int32_t k16_per_kv_head, rtp_view q, rtp_view k,

@@ -2,7 +2,8 @@
 //
 // q16 = W^Q q and k16 = W^K k per retrieval head ("Low-Dimensional Projection
 // Mechanism" of the paper-graph-ui summary of arXiv 2605.16928), fp32
-// accumulation in a fixed order (d = 0..127), one bf16 round-to-nearest-even.
+// accumulation in a fixed order (four interleaved chains over d, then a fixed
+// tree), one bf16 round-to-nearest-even.
 //
 // HBM-bound: each CTA stages 32 input rows (256 B each) and one 128x16 weight
 // in shared memory; 4 threads per row each produce 4 of the 16 outputs.
@@ -34,7 +35,7 @@ struct ProjParams {
 };
 
 __global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p) {
-  __shared__ float sW[kD][kR];
+  __shared__ __align__(16) float sW[kD][kR];
   __shared__ float sX[kProjRows][kD + 1];
   const int jb = blockIdx.y < p.job[0].n_slots ? 0 : 1;
   const ProjJob& J = p.job[jb];
@@ -43,21 +44,24 @@ __global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p
   const int row0 = blockIdx.x * kProjRows;
   if (row0 >= J.L) return;
   const int tid = threadIdx.x;
+  const int nrows = min(kProjRows, J.L - row0);
 
-  const uint16_t* W = J.W + (size_t)slot * kD * kR;
-  for (int e = tid; e < kD * kR; e += kProjThreads)
-    sW[e / kR][e % kR] = __uint_as_float((uint32_t)W[e] << 16);
-
+  // the weight: 256 chunks of 8 bf16, two per thread
+  const uint4* W = reinterpret_cast<const uint4*>(J.W + (size_t)slot * kD * kR);
+  for (int c = tid; c < kD * kR / 8; c += kProjThreads) {
+    const uint4 v = W[c];
+    float* dst = &sW[0][0] + c * 8;
+    dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x);
+    dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
+    dst[4] = bf16_lo(v.z); dst[5] = bf16_hi(v.z);
+    dst[6] = bf16_lo(v.w); dst[7] = bf16_hi(v.w);
+  }
   const int head = p.head_of_slot[jb][slot];
-  // 32 rows x 16 chunks of 16 bytes
-  for (int c = tid; c < kProjRows * 16; c += kProjThreads) {
+  // the rows: 16 chunks of 16 bytes each (rows past L are not read)
+  for (int c = tid; c < nrows * 16; c += kProjThreads) {
     const int r = c / 16, ch = c % 16;
-    const int row = row0 + r;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (row < J.L) {
-      const uint16_t* src = J.x + b * J.x_sb + (int64_t)row * J.x_sl + head * kD + ch * 8;
-      v = *reinterpret_cast<const uint4*>(src);
-    }
+    const uint16_t* src = J.x + b * J.x_sb + (int64_t)(row0 + r) * J.x_sl + head * kD + ch * 8;
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
     float* dst = &sX[r][ch * 8];
     dst[0] = bf16_lo(v.x); dst[1] = bf16_hi(v.x);
     dst[2] = bf16_lo(v.y); dst[3] = bf16_hi(v.y);
@@ -66,26 +70,38 @@ __global__ void __launch_bounds__(kProjThreads) proj16_kernel(const ProjParams p
   }
   __syncthreads();
 
+  // thread (r, c0): outputs c0..c0+3 of row r; each is four fp32 chains over
+  // d = q, q+4, q+8, ... (q = 0..3) summed as ((a0 + a1) + (a2 + a3)): a fixed
+  // order shared by every call, so a key's k16 is the same in prefill and decode
   const int r = tid / 4;
   const int c0 = (tid % 4) * 4;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  if (r >= nrows) return;
+  float acc[4][4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int o = 0; o < 4; ++o) acc[q][o] = 0.f;
 #pragma unroll 8
-  for (int d = 0; d < kD; ++d) {
-    const float xv = sX[r][d];
-    const float4 w = *reinterpret_cast<const float4*>(&sW[d][c0]);
-    acc0 = fmaf(xv, w.x, acc0);
-    acc1 = fmaf(xv, w.y, acc1);
-    acc2 = fmaf(xv, w.z, acc2);
-    acc3 = fmaf(xv, w.w, acc3);
+  for (int d = 0; d < kD; d += 4) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float xv = sX[r][d + q];
+      const float4 w = *reinterpret_cast<const float4*>(&sW[d + q][c0]);
+      acc[q][0] = fmaf(xv, w.x, acc[q][0]);
+      acc[q][1] = fmaf(xv, w.y, acc[q][1]);
+      acc[q][2] = fmaf(xv, w.z, acc[q][2]);
+      acc[q][3] = fmaf(xv, w.w, acc[q][3]);
+    }
   }
-  const int row = row0 + r;
-  if (row < J.L) {
-    uint2 o;
-    o.x = pack_bf16x2(acc0, acc1);
-    o.y = pack_bf16x2(acc2, acc3);
-    uint16_t* dst = J.out + b * J.o_sb + (int64_t)row * J.o_sl + slot * kR + c0;
-    *reinterpret_cast<uint2*>(dst) = o;
-  }
+  float out[4];
+#pragma unroll
+  for (int o = 0; o < 4; ++o)
+    out[o] = __fadd_rn(__fadd_rn(acc[0][o], acc[1][o]), __fadd_rn(acc[2][o], acc[3][o]));
+  uint2 ov;
+  ov.x = pack_bf16x2(out[0], out[1]);
+  ov.y = pack_bf16x2(out[2], out[3]);
+  uint16_t* dst = J.out + b * J.o_sb + (int64_t)(row0 + r) * J.o_sl + slot * kR + c0;
+  *reinterpret_cast<uint2*>(dst) = ov;
 }
 
 void set_job(ProjJob& J, const rtp_view& x, int L, const void* W, int n_slots,
@@ -122,6 +138,7 @@ extern "C" rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv
   if ((st = check_view(k16, hm.H_k16, kR, do_k)) != RTP_OK) return st;
   if (do_q && Wq16 == nullptr) return RTP_ERR_INVALID_ARG;
   if (do_k && Wk16 == nullptr) return RTP_ERR_INVALID_ARG;
+  if ((do_q && !aligned16(Wq16)) || (do_k && !aligned16(Wk16))) return RTP_ERR_ALIGNMENT;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!do_q && !do_k) return RTP_OK;
   ProjParams p;

@@ -339,6 +339,8 @@ def bench_decode(args, world, rank, local, pk):
     trace(False)
     res = decode_step(st, None, None)
     torch.cuda.synchronize()
+    from long_context_sparse_rtp_b200 import rtp_check_device
+    rtp_check_device()  # no kernel recorded an error during the timed steps
     union, compute_sel = union_size(st, res)
     B = st["q"].shape[0]
     nbytes = decode_bytes(st, union)
@@ -389,6 +391,8 @@ def bench_prefill(args, world, rank, pk):
     ms = max_over_ranks(ms, world)
     res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
     torch.cuda.synchronize()
+    from long_context_sparse_rtp_b200 import rtp_check_device
+    rtp_check_device()
     cnt = res["sel"]["count"].double()
     L = q.shape[1]
     sel_pairs = float(cnt.sum())

@@ -9,6 +9,7 @@ loudly if it is not built.
 """
 from .rtp import (  # noqa: F401
     RtpError,
+    rtp_check_device,
     rtp_dense_attn,
     rtp_get_device_status,
     rtp_index_scores,

@@ -626,8 +626,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       ebar();
       if (state == ST_REFINE && g == 0) flush_row(sm, r);
       ebar();
-      // the list length of a row that parked its crossing range this sweep
-      const int nl = state == ST_LIST ? min(sm.ncnt[r], kListCap) : 0;
+      // a row that parked its crossing range this sweep (a row that turns to
+      // ST_LIST below parks in the next sweep)
+      const bool lst = collect == 2 && mine;
+      const int nl = lst ? min(sm.ncnt[r], kListCap) : 0;
       if (state == ST_COLLECT) {
         if (g == 0) finish_row();
         state = ST_DONE;
@@ -642,9 +644,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         state = next_state(n_in);
       }
       ebar();
-      if (g == 0 && state == ST_REFINE) clear_row(sm, r);
+      if (g == 0 && (state == ST_REFINE || (state == ST_LIST && !lst))) clear_row(sm, r);
       // rows with a parked list: the remaining radix levels run over the list
-      const bool lst = state == ST_LIST;
       const unsigned long long* my = lst ? lists + (size_t)r * kListCap : nullptr;
       for (;;) {
         const bool need = lst && n_cur > (uint32_t)kCap && pbits < kKeyBits;

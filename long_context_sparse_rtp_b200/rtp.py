@@ -149,6 +149,23 @@ def rtp_get_device_status(ws: torch.Tensor, stream=None) -> int:
     return lib().rtp_get_device_status(_ptr(ws), _stream(stream))
 
 
+def rtp_check_device(device=None, stream=None) -> None:
+    """Reads (and clears) the device status word of every workspace the binding
+    holds for `device`; raises RtpError if a kernel recorded an error since the
+    last check (a bounded wait that ran out, or an internal consistency check).
+    Synchronises the stream."""
+    dev = str(torch.device(device if device is not None else "cuda"))
+    if dev == "cuda":
+        dev = f"cuda:{torch.cuda.current_device()}"
+    for (d, op), ws in list(_ws_cache.items()):
+        if d != dev:
+            continue
+        where = int(ws[4:8].view(torch.int32).item())
+        code = rtp_get_device_status(ws, stream)
+        if code != RTP_OK:
+            raise RtpError(f"device status of op {op} (site {where})", code)
+
+
 # --------------------------------------------------------------------- entry points
 def _n_ret(kv_role, G):
     return int(sum(int(x) for x in kv_role)) * G

@@ -80,28 +80,53 @@ def check_outputs(o_gpu: np.ndarray, o_orc: np.ndarray, what: str):
     return mx, mean
 
 
-def check_row_outputs(o_gpu, o_same_sel, o_e2e, same_count, same_sel, what,
-                      max_skip_count=0.01, max_skip_sel=0.05):
-    """Output parity of retrieval rows.
+def gpu_kept(s64, t_gpu, jtie_gpu, p):
+    """The GPU's kept set of one row as a bool mask over keys 0..P."""
+    j = np.arange(s64.size)
+    if p >= 1.0:
+        return np.ones(s64.size, bool)
+    return (s64 > t_gpu) | ((s64 == t_gpu) & (j <= jtie_gpu))
 
-    o_same_sel: the oracle run on the GPU's own q16/k16 (same kept sets up to
-    in-band keys); checked on every row where the kept-set sizes agree.
-    o_e2e: the oracle run end to end on its own projections; checked on the rows
-    whose oracle kept set does not change between the two projections (a 1-ulp
-    bf16 difference in q16/k16 can legitimately reorder near-tied keys, and in
-    a row with few kept keys that changes the output by O(1)).  The fraction of
-    rows skipped by either rule is bounded."""
+
+E2E_MASS = 1e-3
+
+
+def row_reference(q_bits, K_bits, V_bits, kept_gpu, sel_same, o_same, lse_same, sel_e2e, scale):
+    """References for one retrieval row.
+
+    (o_ref, lse_ref): the oracle's exact attention over the GPU's own kept set
+    (taken from the oracle run on the GPU's q16/k16 when its kept set is the
+    same, else attended directly) -- every row gets one.  e2e_ok: whether the
+    oracle run end to end (its own projections) may serve as a second reference:
+    its kept set differs from the GPU's by keys whose share of the attention
+    mass (over the union of both sets) is at most E2E_MASS.  Keys near the cut
+    carry little mass except in rows with few kept keys, where a legitimate
+    one-key difference changes the output by O(1)."""
+    if np.array_equal(kept_gpu, sel_same):
+        o_ref, lse_ref = o_same, lse_same
+    else:
+        o_ref, lse_ref = oracle.attend(q_bits, K_bits, V_bits, np.nonzero(kept_gpu)[0], scale)
+    sym = kept_gpu ^ sel_e2e
+    if not sym.any():
+        return o_ref, lse_ref, True
+    _, lse_sym = oracle.attend(q_bits, K_bits, V_bits, np.nonzero(sym)[0], scale)
+    _, lse_uni = oracle.attend(q_bits, K_bits, V_bits, np.nonzero(kept_gpu | sel_e2e)[0], scale)
+    return o_ref, lse_ref, bool(math.exp(lse_sym - lse_uni) <= E2E_MASS)
+
+
+def check_row_outputs(o_gpu, o_ref, o_e2e, e2e_ok, what, max_skip_e2e=0.05):
+    """Output parity of retrieval rows: every row against the oracle's attention
+    over the GPU's own kept set (o_ref); the rows whose end-to-end oracle kept
+    set carries the same mass up to E2E_MASS (e2e_ok) also against the oracle
+    run end to end on its own projections.  The share of rows left out of the
+    second check is bounded."""
     n = len(o_gpu)
-    same_count = np.asarray(same_count, bool)
-    same_sel = np.asarray(same_sel, bool)
-    assert (~same_count).sum() <= max(2, max_skip_count * n), (int((~same_count).sum()), n)
-    assert (~same_sel).sum() <= max(2, max_skip_sel * n), (int((~same_sel).sum()), n)
-    r1 = check_outputs(o_gpu[same_count], o_same_sel[same_count],
-                       what + " vs oracle on the GPU's q16/k16")
-    both = same_count & same_sel
-    r2 = check_outputs(o_gpu[both], o_e2e[both], what + " vs oracle end to end")
-    return dict(skip_count=int((~same_count).sum()), skip_sel=int((~same_sel).sum()),
-                max_abs=r1[0], mean_abs=r1[1], e2e_max_abs=r2[0], e2e_mean_abs=r2[1])
+    e2e_ok = np.asarray(e2e_ok, bool)
+    assert (~e2e_ok).sum() <= max(2, max_skip_e2e * n), (int((~e2e_ok).sum()), n)
+    r1 = check_outputs(o_gpu, o_ref, what + " vs oracle on the GPU's kept sets")
+    r2 = check_outputs(o_gpu[e2e_ok], o_e2e[e2e_ok], what + " vs oracle end to end")
+    return dict(skip_e2e=int((~e2e_ok).sum()), max_abs=r1[0], mean_abs=r1[1],
+                e2e_max_abs=r2[0], e2e_mean_abs=r2[1])
 
 
 def oracle_k16(k_bits, Wk_bits, w: synth.Workload, per_kv: bool = False):

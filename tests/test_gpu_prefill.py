@@ -17,6 +17,7 @@ import torch
 import oracle
 from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
 from rtp_check import (LSE_ABS, bits, check_outputs, check_row_outputs, check_row_selection, f64,
+                       gpu_kept, row_reference,
                        oracle_k16, oracle_q16, row_scores)
 
 pytestmark = pytest.mark.gpu
@@ -87,7 +88,7 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     k16o = oracle_k16(kb, Wkb, w, per_kv)
 
     n_band, o_ret_g, o_ret_a, o_ret_o, o_loc_g, o_loc_o = 0, [], [], [], [], []
-    same_count, same_sel = [], []
+    e2e_ok = []
     lse_err = 0.0
     for b in range(B):
         for x, i in enumerate(positions):
@@ -98,26 +99,27 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
             r2 = oracle.retrieval_rows(q1, kb1, vb1, q16_1, k16g1, rows, np.arange(len(ret)),
                                        np.array(k16slot), H=w.H, Hkv=w.Hkv, q_pos0=int(i), p=p,
                                        scale=SCALE, want_sel=True)
-            for s in range(len(ret)):
-                s64 = row_scores(q16s[b, x, s], k16g[b, :, k16slot[s]], int(i))
-                n_band += check_row_selection(
-                    s64, p, r2["t"][s], r2["sel"][s], float(sel["thr"][b, s, x]),
-                    int(sel["jtie"][b, s, x]), int(sel["count"][b, s, x]),
-                    float(sel["mass"][b, s, x]))
-                same_count.append(int(sel["count"][b, s, x]) == int(r2["count"][s]))
-            o_ret_a.append(r2["o"])
             # (iii) end to end with the oracle's own projections
             q16o = np.stack([oracle.project(qs[b, x, h][None], Wqb[s])[0][0]
                              for s, h in enumerate(ret)])[None, None]
             r3 = oracle.retrieval_rows(q1, kb1, vb1, q16o, k16o[b:b + 1], rows,
                                        np.arange(len(ret)), np.array(k16slot), H=w.H, Hkv=w.Hkv,
                                        q_pos0=int(i), p=p, scale=SCALE, want_sel=True)
-            same_sel.extend(np.array_equal(a, c) for a, c in zip(r2["sel"], r3["sel"]))
+            for s, h in enumerate(ret):
+                s64 = row_scores(q16s[b, x, s], k16g[b, :, k16slot[s]], int(i))
+                t_g, jt_g = float(sel["thr"][b, s, x]), int(sel["jtie"][b, s, x])
+                n_band += check_row_selection(s64, p, r2["t"][s], r2["sel"][s], t_g, jt_g,
+                                              int(sel["count"][b, s, x]),
+                                              float(sel["mass"][b, s, x]))
+                g = h // w.G
+                o_ref, lse_ref, ok = row_reference(
+                    qs[b, x, h], kb[b, :i + 1, g], vb[b, :i + 1, g], gpu_kept(s64, t_g, jt_g, p),
+                    r2["sel"][s], r2["o"][s], r2["lse"][s], r3["sel"][s], SCALE)
+                o_ret_a.append(o_ref)
+                e2e_ok.append(ok)
+                lse_err = max(lse_err, abs(float(lse[b, h, x]) - lse_ref))
             o_ret_o.append(r3["o"])
             o_ret_g.append(o[b, x, ret])
-            ok = np.array([int(sel["count"][b, s, x]) == int(r2["count"][s]) for s in range(len(ret))])
-            if ok.any():
-                lse_err = max(lse_err, float(np.abs(lse[b, ret, x] - r2["lse"])[ok].max()))
             if loc:
                 rl = oracle.local_rows(q1, kb1, vb1, np.array([(0, 0, h) for h in loc]), H=w.H,
                                        Hkv=w.Hkv, q_pos0=int(i), window=w.window,
@@ -125,8 +127,8 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
                 o_loc_o.append(rl["o"])
                 o_loc_g.append(o[b, x, loc])
                 lse_err = max(lse_err, float(np.abs(lse[b, loc, x] - rl["lse"]).max()))
-    stats = check_row_outputs(np.concatenate(o_ret_g), np.concatenate(o_ret_a),
-                              np.concatenate(o_ret_o), same_count, same_sel, "retrieval heads")
+    stats = check_row_outputs(np.concatenate(o_ret_g), np.stack(o_ret_a),
+                              np.concatenate(o_ret_o), e2e_ok, "retrieval heads")
     if loc:
         check_outputs(np.concatenate(o_loc_g), np.concatenate(o_loc_o), "local heads")
     assert lse_err <= LSE_ABS, lse_err

@@ -77,7 +77,8 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
         n_band += check_row_selection(s64, p, r2["t"][r], r2["sel"][r], float(sel["thr"][b, s]),
                                       int(sel["jtie"][b, s]), int(sel["count"][b, s]),
                                       float(sel["mass"][b, s]))
-        kept.append(gpu_kept(s64, float(sel["thr"][b, s]), int(sel["jtie"][b, s]), p))
+        kept.append(gpu_kept(q16g[b, 0, s], k16g[b, :, k16slot[s]], P, float(sel["thr"][b, s]),
+                             int(sel["jtie"][b, s]), int(sel["count"][b, s]), p))
     # (iii) end to end with the oracle's own projections
     q16o = np.zeros_like(q16g)
     for b in range(B):
@@ -87,17 +88,19 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
     r3 = oracle.retrieval_rows(qb, kb, vb, q16o, k16o, rows, slots, ks, H=w.H, Hkv=w.Hkv,
                                q_pos0=P, p=p, scale=SCALE, want_sel=True)
     og = np.stack([o[b, 0, h] for (b, _, h) in rows])
-    o_ref, lse_ref, e2e_ok = [], [], []
+    o_ref, lse_ref, ref_ok, e2e_ok = [], [], [], []
     for r, (b, _, h) in enumerate(rows):
         g = h // w.G
-        a, l_, ok = row_reference(qb[b, 0, h], kb[b, :P + 1, g], vb[b, :P + 1, g], kept[r],
-                                  r2["sel"][r], r2["o"][r], r2["lse"][r], r3["sel"][r], SCALE)
+        a, l_, ok, ok2 = row_reference(qb[b, 0, h], kb[b, :P + 1, g], vb[b, :P + 1, g], kept[r],
+                                       r2["sel"][r], r2["o"][r], r2["lse"][r], r3["sel"][r],
+                                       SCALE)
         o_ref.append(a)
         lse_ref.append(l_)
-        e2e_ok.append(ok)
-    check_row_outputs(og, np.stack(o_ref), r3["o"], e2e_ok, "retrieval decode")
+        ref_ok.append(ok)
+        e2e_ok.append(ok2)
+    check_row_outputs(og, np.stack(o_ref), ref_ok, r3["o"], e2e_ok, "retrieval decode")
     lg = np.array([lse[b, h, 0] for (b, _, h) in rows])
-    assert np.abs(lg - np.array(lse_ref)).max(initial=0.0) <= LSE_ABS
+    assert np.abs(lg - np.array(lse_ref))[np.array(ref_ok)].max(initial=0.0) <= LSE_ABS
     if loc:
         lrows = np.array([(b, 0, h) for b in range(B) for h in loc])
         rl = oracle.local_rows(qb, kb, vb, lrows, H=w.H, Hkv=w.Hkv, q_pos0=P, window=w.window,

@@ -88,7 +88,7 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     k16o = oracle_k16(kb, Wkb, w, per_kv)
 
     n_band, o_ret_g, o_ret_a, o_ret_o, o_loc_g, o_loc_o = 0, [], [], [], [], []
-    e2e_ok = []
+    ref_ok, e2e_ok = [], []
     lse_err = 0.0
     for b in range(B):
         for x, i in enumerate(positions):
@@ -112,12 +112,16 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
                                               int(sel["count"][b, s, x]),
                                               float(sel["mass"][b, s, x]))
                 g = h // w.G
-                o_ref, lse_ref, ok = row_reference(
-                    qs[b, x, h], kb[b, :i + 1, g], vb[b, :i + 1, g], gpu_kept(s64, t_g, jt_g, p),
-                    r2["sel"][s], r2["o"][s], r2["lse"][s], r3["sel"][s], SCALE)
+                kept = gpu_kept(q16s[b, x, s], k16g[b, :, k16slot[s]], int(i), t_g, jt_g,
+                                int(sel["count"][b, s, x]), p)
+                o_ref, lse_ref, ok, ok2 = row_reference(
+                    qs[b, x, h], kb[b, :i + 1, g], vb[b, :i + 1, g], kept, r2["sel"][s],
+                    r2["o"][s], r2["lse"][s], r3["sel"][s], SCALE)
                 o_ret_a.append(o_ref)
-                e2e_ok.append(ok)
-                lse_err = max(lse_err, abs(float(lse[b, h, x]) - lse_ref))
+                ref_ok.append(ok)
+                e2e_ok.append(ok2)
+                if ok:
+                    lse_err = max(lse_err, abs(float(lse[b, h, x]) - lse_ref))
             o_ret_o.append(r3["o"])
             o_ret_g.append(o[b, x, ret])
             if loc:
@@ -127,7 +131,7 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
                 o_loc_o.append(rl["o"])
                 o_loc_g.append(o[b, x, loc])
                 lse_err = max(lse_err, float(np.abs(lse[b, loc, x] - rl["lse"]).max()))
-    stats = check_row_outputs(np.concatenate(o_ret_g), np.stack(o_ret_a),
+    stats = check_row_outputs(np.concatenate(o_ret_g), np.stack(o_ret_a), ref_ok,
                               np.concatenate(o_ret_o), e2e_ok, "retrieval heads")
     if loc:
         check_outputs(np.concatenate(o_loc_g), np.concatenate(o_loc_o), "local heads")

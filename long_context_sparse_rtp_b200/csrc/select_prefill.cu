@@ -45,7 +45,7 @@ constexpr int kTileBytes = kBN * kR * 2;
 constexpr int kNB = 32;          // histogram bins (5-bit digits)
 constexpr int kDigit = 5;
 constexpr int kCap = 32;         // candidates collected per row
-constexpr int kGroup = 8;        // tiles per 32-bit bin-sum group: <= 1024 keys x 2^21 < 2^32
+constexpr int kGroup = 16;       // tiles per 32-bit bin-sum group: 16 x 64 keys x 2^21 < 2^32
 constexpr int kMaxIter = 16;     // refine / collect sweeps (53 key bits / 5 + 1 suffice)
 constexpr int kQueue = 64;       // per-warp queue of refine hits (drained at 32)
 constexpr int kChunk = 16;       // keys per TMEM load and per unrolled body
@@ -57,7 +57,9 @@ constexpr unsigned long long kIdxMask = (1ull << kIdxBits) - 1;
 constexpr int kKeyBits = 32 + kIdxBits;  // 53
 constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 
-enum { ST_IDLE = 0, ST_REFINE = 1, ST_COLLECT = 2, ST_DONE = 3, ST_LIST = 4 };
+// row states: REFINE1 = 32 uniform score sub-bins of the level-0 crossing bin,
+// REFINE = 5 composite-key bits, COLLECT / LIST = gather the crossing range's keys
+enum { ST_IDLE = 0, ST_REFINE1 = 1, ST_REFINE = 2, ST_COLLECT = 3, ST_DONE = 4, ST_LIST = 5 };
 constexpr int kListCap = 1024;   // crossing-bin keys a row may park in its global list
 
 struct SelParams {
@@ -81,11 +83,11 @@ struct SelSmem {
   uint8_t ktile[kStages][kTileBytes];  // 1024-byte aligned (the struct is placed so)
   uint8_t qtile[kBM * kR * 2];
   union {
-    unsigned long long hw[kNB][kBM];   // per-row bin sums (fixed21 units), row fastest
+    unsigned long long hw[kNB][kBM];   // per-row bin sums (units of 2^-21 of a bin edge), row fastest
     unsigned long long cand[kCap][kBM];
   } u;
-  uint32_t wacc[kNB][kBM];             // bin sums of the current tile group
-  uint32_t hc[kNB][kBM];               // bin counts
+  uint32_t wacc[2][kNB][kBM];          // bin sums of the current tile group, one copy per
+                                       // column half (the row's two threads)
   union {
     float tab[kNB][kBM];               // exp(b / scale): level-0 bin b's edge factor
     struct {                           // refine sweeps: per-warp queues of prefilter hits
@@ -96,6 +98,7 @@ struct SelSmem {
   float mpart[2][kBM];
   double zpart[2][kBM];
   int ncnt[kBM];
+  int nabove[kBM];                     // keys above the crossing range (exact)
   uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], qfull, ctl;
   uint32_t tmem_base;
   int go;
@@ -112,11 +115,10 @@ __device__ __forceinline__ float ex2_ftz(float x) {
 __device__ __forceinline__ float rel_w(float s, float m) {
   return ex2_ftz(__fmul_rn(__fsub_rn(s, m), kLog2e));
 }
-// trunc(w * 2^21) for w in [0, 1]: adding 2^23 with rounding toward zero leaves
-// the integer part in the low mantissa bits.
-__device__ __forceinline__ uint32_t fixed21(float w) {
-  return __float_as_uint(__fadd_rz(__fmul_rn(fminf(w, 1.0f), 2097152.0f), 8388608.0f)) -
-         0x4B000000u;
+// trunc(x) for x in [0, 2^21] (clamped): adding 2^23 with rounding toward zero
+// leaves the integer part in the low mantissa bits.
+__device__ __forceinline__ uint32_t fixed_u(float x) {
+  return __float_as_uint(__fadd_rz(fminf(x, 2097152.0f), 8388608.0f)) - 0x4B000000u;
 }
 // Level-0 bin of a score s <= m: floor((m - s) * scale), at most kNB - 1 (adding
 // 1.5 * 2^23 with rounding toward -inf leaves the floor in the low mantissa bits).
@@ -135,40 +137,38 @@ __device__ __forceinline__ float key_score(uint32_t key) {
   return __uint_as_float(b);
 }
 
-// Crossing search over one row's descending histogram (column r of hw / hc):
-// the first bin b where base + factor(b) * (inner + hw[b]) reaches T.  Returns
-// the bin; adds the bins above it to inner (same-factor histograms) or base
-// (factor per bin) and to cnt.
+// Crossing search over one row's descending histogram (column r of hw): the
+// first non-empty bin b where base + factor(b) * (inner + hw[b]) reaches T.
+// Returns the bin and its sum; adds the bins above it to inner (same-factor
+// histograms) or base (a factor per bin).  Every key adds a positive amount to
+// its bin, so a zero sum is an empty bin.
 template <class Factor>
 __device__ __forceinline__ int crossing(const SelSmem& sm, int r, int nb, double T, bool per_bin,
                                         Factor&& factor, double& base,
-                                        unsigned long long& inner, uint32_t& cnt,
-                                        uint32_t& n_in) {
+                                        unsigned long long& inner, unsigned long long& w_sel) {
   int last = -1;
   for (int b = 0; b < nb; ++b) {
-    const uint32_t c = sm.hc[b][r];
-    if (c == 0) continue;
-    last = b;
     const unsigned long long wb = sm.u.hw[b][r];
+    if (wb == 0ull) continue;
+    last = b;
     const double f = factor(b);
     if (per_bin ? (base + f * (double)wb >= T) : (base + f * (double)(inner + wb) >= T)) {
-      n_in = c;
+      w_sel = wb;
       return b;
     }
     if (per_bin)
       base += f * (double)wb;
     else
       inner += wb;
-    cnt += c;
   }
   // rounding left T out of reach: keep everything, i.e. the lowest non-empty bin
+  w_sel = 0ull;
   if (last >= 0) {
+    w_sel = sm.u.hw[last][r];
     if (per_bin)
-      base -= factor(last) * (double)sm.u.hw[last][r];
+      base -= factor(last) * (double)w_sel;
     else
-      inner -= sm.u.hw[last][r];
-    cnt -= sm.hc[last][r];
-    n_in = sm.hc[last][r];
+      inner -= w_sel;
   }
   return last;
 }
@@ -177,17 +177,18 @@ __device__ __forceinline__ void clear_row(SelSmem& sm, int r) {
 #pragma unroll 8
   for (int b = 0; b < kNB; ++b) {
     sm.u.hw[b][r] = 0ull;
-    sm.wacc[b][r] = 0u;
-    sm.hc[b][r] = 0u;
+    sm.wacc[0][b][r] = 0u;
+    sm.wacc[1][b][r] = 0u;
   }
 }
 
-// Moves the tile group's 32-bit bin sums into the 64-bit ones.
+// Moves the tile group's 32-bit bin sums (both copies) into the 64-bit ones.
 __device__ __forceinline__ void flush_row(SelSmem& sm, int r) {
 #pragma unroll 8
   for (int b = 0; b < kNB; ++b) {
-    sm.u.hw[b][r] += sm.wacc[b][r];
-    sm.wacc[b][r] = 0u;
+    sm.u.hw[b][r] += (unsigned long long)sm.wacc[0][b][r] + sm.wacc[1][b][r];
+    sm.wacc[0][b][r] = 0u;
+    sm.wacc[1][b][r] = 0u;
   }
 }
 
@@ -202,14 +203,46 @@ __device__ __forceinline__ float max16(const float (&v)[kChunk]) {
   return t[0];
 }
 
+// Level-1 sub-bin of a key of level-0 bin k0: the 32 uniform score sub-bins of
+// that bin.  (m - s) * 32 scale is exactly 32 times the product bin0_of floors,
+// so the sub-bins partition the bin.
+__device__ __forceinline__ int sub1_of(float s, float m, float scale32, int k0) {
+  const float x = fminf(__fmul_rn(__fsub_rn(m, s), scale32), 2097152.0f);
+  const int b = __float_as_int(__fadd_rd(x, 12582912.0f)) - 0x4B400000 - kNB * k0;
+  return min(max(b, 0), kNB - 1);
+}
+
+// Where a key stands against a row's crossing range (level-0 bin k0, level-1
+// sub-bin k1 if k1 >= 0, composite-key prefix of pbits bits): -1 below, 0
+// inside, 1 above.  The order is the one every histogram level used.
+__device__ __forceinline__ int classify(float s, unsigned long long ck, float m, float scale,
+                                        int k0, int k1, int pbits, unsigned long long prefix) {
+  const int b0 = bin0_of(s, m, scale);
+  if (b0 != k0) return b0 < k0 ? 1 : -1;
+  if (k1 >= 0) {
+    const int b1 = sub1_of(s, m, scale * (float)kNB, k0);
+    if (b1 != k1) return b1 < k1 ? 1 : -1;
+  }
+  if (pbits > 0) {
+    const unsigned long long px = ck >> (kKeyBits - pbits);
+    if (px != prefix) return px > prefix ? 1 : -1;
+  }
+  return 0;
+}
+
+enum { MODE_SUB1 = 0, MODE_DIGIT = 1, MODE_COLLECT = 2, MODE_PARK = 3 };
+
 // Processes the first n (<= 32) queued prefilter hits of this warp, one per
-// lane: the exact crossing-bin and prefix tests of the owning row (whose state
-// is fetched from the owner lane), then a candidate (collect = 1), a key parked
-// in the row's global list (collect = 2) or a digit count (collect = 0).  Called
-// by all 32 lanes.
+// lane, for the owning row (whose state is fetched from the owner lane):
+// MODE_SUB1 adds the key to its level-1 sub-bin, MODE_DIGIT to its digit bin
+// (the next w composite-key bits), MODE_COLLECT makes it a candidate,
+// MODE_PARK stores it in the row's global list; the last two count the keys
+// above the range.  Histogram sums go to this warp's column-half copy.
+// Called by all 32 lanes.
 __device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, int wq, int n,
-                                        int row0, float m, float scale, int k0, int pbits,
-                                        unsigned long long prefix, int w, float tk, int collect) {
+                                        int row0, int g, float m, float scale, int k0, int k1,
+                                        int pbits, unsigned long long prefix, int w, float tk,
+                                        int mode) {
   const int lane = threadIdx.x & 31;
   const bool has = lane < n;
   const float s = has ? sm.t.q.s[wq][lane] : 0.f;
@@ -218,38 +251,62 @@ __device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, i
   const float om = __shfl_sync(0xffffffffu, m, owner);
   const float osc = __shfl_sync(0xffffffffu, scale, owner);
   const int ok0 = __shfl_sync(0xffffffffu, k0, owner);
+  const int ok1 = __shfl_sync(0xffffffffu, k1, owner);
   const int opb = __shfl_sync(0xffffffffu, pbits, owner);
   const uint32_t opl = __shfl_sync(0xffffffffu, (uint32_t)prefix, owner);
   const uint32_t oph = __shfl_sync(0xffffffffu, (uint32_t)(prefix >> 32), owner);
   const int ow = __shfl_sync(0xffffffffu, w, owner);
   const float otk = __shfl_sync(0xffffffffu, tk, owner);
-  const int ocol = __shfl_sync(0xffffffffu, collect, owner);
-  if (!has || bin0_of(s, om, osc) != ok0) return;
-  const unsigned long long ck = comp_key(s, j);
-  const unsigned long long opx = ((unsigned long long)oph << 32) | opl;
-  if (opb > 0 && (ck >> (kKeyBits - opb)) != opx) return;
+  const int omode = __shfl_sync(0xffffffffu, mode, owner);
+  if (!has) return;
   const int r = row0 + owner;
-  if (ocol == 2) {  // park the key in the row's global list
-    const int slot_c = atomicAdd(&sm.ncnt[r], 1);
-    if (slot_c < kListCap) list[(size_t)r * kListCap + slot_c] = ck;
-  } else if (ocol) {
-    const int slot_c = atomicAdd(&sm.ncnt[r], 1);
-    if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
-  } else {
+  if (omode == MODE_SUB1) {
+    if (bin0_of(s, om, osc) != ok0) return;
+    const int b1 = sub1_of(s, om, osc * (float)kNB, ok0);
+    atomicAdd(&sm.wacc[g][b1][r], fixed_u(__fmul_rn(rel_w(s, om), otk)));
+    return;
+  }
+  const unsigned long long ck = comp_key(s, j);
+  const int c = classify(s, ck, om, osc, ok0, ok1, opb, ((unsigned long long)oph << 32) | opl);
+  if (omode == MODE_DIGIT) {
+    if (c != 0) return;
     const int digit = (int)((ck >> (kKeyBits - opb - ow)) & ((1ull << ow) - 1));
-    const int bin = (1 << ow) - 1 - digit;
-    atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(s, om), otk)));
-    atomicAdd(&sm.hc[bin][r], 1u);
+    atomicAdd(&sm.wacc[g][(1 << ow) - 1 - digit][r], fixed_u(__fmul_rn(rel_w(s, om), otk)));
+  } else if (c > 0) {
+    atomicAdd(&sm.nabove[r], 1);
+  } else if (c == 0) {
+    const int slot_c = atomicAdd(&sm.ncnt[r], 1);
+    if (omode == MODE_PARK) {
+      if (slot_c < kListCap) list[(size_t)r * kListCap + slot_c] = ck;
+    } else if (slot_c < kCap) {
+      sm.u.cand[slot_c][r] = ck;
+    }
   }
 }
 
-// Score interval that holds every score of composite-key prefix `prefix`
-// (pbits bits) inside level-0 bin k0, widened by a relative margin.
-__device__ __forceinline__ void refine_range(float m, float scale, int k0, int pbits,
-                                             unsigned long long prefix, float& lo, float& hi) {
-  const float margin = 1e-5f * (fabsf(m) + (float)kNB / scale + 1.f);
-  lo = m - (float)(k0 + 1) / scale - margin;
-  hi = m - (float)k0 / scale + margin;
+// The composite-key prefix shared by every score in [lo_s, hi_s] (widened by
+// the margin that covers the fp32 rounding of the bin edges).
+__device__ __forceinline__ void range_prefix(float lo_s, float hi_s, float margin, int& pbits,
+                                             unsigned long long& prefix) {
+  const unsigned long long kl = (unsigned long long)score_key(lo_s - margin) << kIdxBits;
+  const unsigned long long kh = ((unsigned long long)score_key(hi_s + margin) << kIdxBits) | kIdxMask;
+  pbits = (kl == kh) ? kKeyBits : (__clzll(kl ^ kh) - (64 - kKeyBits));
+  prefix = pbits > 0 ? (kh >> (kKeyBits - pbits)) : 0ull;
+}
+
+// Score interval that holds every key of a row's crossing range (level-0 bin
+// k0, level-1 sub-bin k1 if k1 >= 0, composite prefix), widened by the margin.
+__device__ __forceinline__ void refine_range(float m, float scale, float margin, int k0, int k1,
+                                             int pbits, unsigned long long prefix, float& lo,
+                                             float& hi) {
+  if (k1 >= 0) {
+    const float s32 = scale * (float)kNB;
+    lo = m - (float)(kNB * k0 + k1 + 1) / s32 - margin;
+    hi = m - (float)(kNB * k0 + k1) / s32 + margin;
+  } else {
+    lo = m - (float)(k0 + 1) / scale - margin;
+    hi = m - (float)k0 / scale + margin;
+  }
   if (pbits > 0) {
     uint32_t k_lo, k_hi;
     if (pbits >= 32) {
@@ -398,8 +455,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t tcount = 0;
     bool ok = true;
     auto ebar = [] { named_bar(1, kEpi); };
-    // one pass over the key tiles: body(j0, v) sees keys j0 .. j0 + 15 of this row;
-    // with a histogram, each tile group's 32-bit sums move to the 64-bit ones
+    // one pass over the key tiles: body(j0, v) sees keys j0 .. j0 + 15 of this row
+    // (keys past its causal limit read as -inf); with hist, each tile group's
+    // 32-bit bin sums move to the 64-bit ones (rows with row_hist)
     auto sweep = [&](auto&& body, bool hist, bool row_hist) {
       for (int kt = 0; kt < n_tiles; ++kt) {
         const int buf = (int)(tcount & 1u);
@@ -409,8 +467,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             float v[kChunk];
+            const int j0 = kt * kBN + g * 64 + c * kChunk;
             tmem_ld16(lane_addr + (uint32_t)(buf * kBN + c * kChunk), v);
-            body(kt * kBN + g * 64 + c * kChunk, v);
+            if ((int64_t)j0 + kChunk - 1 > P) {
+#pragma unroll
+              for (int i = 0; i < kChunk; ++i)
+                if ((int64_t)(j0 + i) > P) v[i] = -INFINITY;
+            }
+            body(j0, v);
           }
         }
         tc_fence_before();
@@ -427,29 +491,21 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // ---- sweep 1: row max
     float m = -INFINITY;
-    sweep(
-        [&](int j0, float (&v)[kChunk]) {
-          if ((int64_t)j0 + kChunk - 1 > P) {
-#pragma unroll
-            for (int i = 0; i < kChunk; ++i)
-              if ((int64_t)(j0 + i) > P) v[i] = -INFINITY;
-          }
-          m = fmaxf(m, max16(v));
-        },
-        false, false);
+    sweep([&](int, float (&v)[kChunk]) { m = fmaxf(m, max16(v)); }, false, false);
     sm.mpart[g][r] = m;
     ebar();
     m = fmaxf(sm.mpart[0][r], sm.mpart[1][r]);
-    float c0 = 0.f, scale = 0.f;
+    float c0 = 0.f, scale = 1.f, margin = 0.f;
     if (valid) {
       const double N = (double)(P + 1);
       const float R = (float)(log(N / (1.0 - (double)p.p)) + 1.0);
       c0 = m - R;
       scale = (float)kNB / R;
+      margin = 1e-5f * (fabsf(m) + R + 1.f);
     }
     if (g == 0) {
       clear_row(sm, r);
-      for (int bb = 0; bb < kNB; ++bb) sm.t.tab[bb][r] = expf((float)bb / scale);
+      for (int bb = 0; bb < kNB; ++bb) sm.t.tab[bb][r] = 2097152.0f * expf((float)bb / scale);
     }
     ebar();
 
@@ -457,20 +513,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     // trunc(2^21 exp(s - m) exp(b / scale)) = trunc(2^21 exp(s - edge_b))
     double Zp = 0.0;
     sweep(
-        [&](int j0, float (&v)[kChunk]) {
+        [&](int, float (&v)[kChunk]) {
           if (!valid) return;
-          const bool full = (int64_t)j0 + kChunk - 1 <= P;
           float e[kChunk];
 #pragma unroll
           for (int i = 0; i < kChunk; ++i) {
-            const bool in = full | ((int64_t)(j0 + i) <= P);
             const float s = v[i];
-            e[i] = in ? rel_w(s, m) : 0.f;
-            if (in & (s >= c0)) {  // the few keys in [c0, m]
-              const int bb = bin0_of(s, m, scale);
-              atomicAdd(&sm.wacc[bb][r], fixed21(__fmul_rn(e[i], sm.t.tab[bb][r])));
-              atomicAdd(&sm.hc[bb][r], 1u);
-            }
+            e[i] = rel_w(s, m);
+            const int bb = bin0_of(s, m, scale);
+            const uint32_t u = fixed_u(__fmul_rn(e[i], sm.t.tab[bb][r]));
+            sm.wacc[g][bb][r] += s >= c0 ? u : 0u;
           }
 #pragma unroll
           for (int w = kChunk / 2; w >= 1; w >>= 1)
@@ -482,37 +534,40 @@ __global__ void __launch_bounds__(kThreads, 2)
     sm.zpart[g][r] = Zp;
     ebar();
     const double Z = sm.zpart[0][r] + sm.zpart[1][r];
-    double T = 0.0, base = 0.0, fk = 0.0;  // fk: mass of one fixed21 unit of bin k0
+    double T = 0.0, base = 0.0, fk = 0.0;  // fk: mass of one unit of bin k0's sums
     unsigned long long inner = 0ull, prefix = 0ull;
-    uint32_t cnt_above = 0u;
-    int k0 = 0, pbits = 0, state = ST_IDLE;
-    uint32_t n_cur = 0u;  // keys of the current crossing range
-    float tk = 0.f;  // exp(k0 / scale)
+    int k0 = 0, k1 = -1, pbits = 0, state = ST_IDLE;
+    float tk = 0.f;    // 2^21 exp(k0 / scale)
+    float umin = 1.f;  // least amount one key of the current range adds
+    unsigned long long n_cur = 0ull;  // bound on the keys of the current range
     unsigned long long* const lists =
         sm.slot >= 0 ? p.lists + (size_t)sm.slot * kBM * kListCap : nullptr;
-    // a row whose crossing range holds <= kCap keys collects them; <= kListCap
-    // parks them in its global list once; more refines the range by a full sweep
-    auto next_state = [&](uint32_t n) {
-      if (n <= (uint32_t)kCap || pbits >= kKeyBits) return (int)ST_COLLECT;
-      return (lists != nullptr && n <= (uint32_t)kListCap) ? (int)ST_LIST : (int)ST_REFINE;
+    // upper bound on the keys of a range from its sum: every key adds >= umin
+    auto bound = [&](unsigned long long wsum) {
+      return (unsigned long long)((double)wsum / (double)umin);
+    };
+    // a range of <= kCap keys is collected, of <= kListCap parked once in the
+    // row's global list; a larger one is refined by another sweep
+    auto next_state = [&](unsigned long long n, bool at_level0) {
+      if (n <= (unsigned long long)kCap || pbits >= kKeyBits) return (int)ST_COLLECT;
+      if (lists != nullptr && n <= (unsigned long long)kListCap) return (int)ST_LIST;
+      return at_level0 ? (int)ST_REFINE1 : (int)ST_REFINE;
     };
     if (valid) {
       T = (double)p.p * Z;
-      uint32_t n_in = 0u;
-      auto f0 = [&](int bb) { return (1.0 / 2097152.0) / (double)sm.t.tab[bb][r]; };
-      k0 = crossing(sm, r, kNB, T, true, f0, base, inner, cnt_above, n_in);
+      unsigned long long wsel = 0ull;
+      auto f0 = [&](int bb) { return 1.0 / (double)sm.t.tab[bb][r]; };
+      k0 = crossing(sm, r, kNB, T, true, f0, base, inner, wsel);
+      if (k0 < 0) {  // cannot happen: the max key is in bin 0
+        set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 16);
+        k0 = 0;
+      }
       tk = sm.t.tab[k0][r];
       fk = f0(k0);
-      // composite-key prefix shared by every score the crossing bin can hold
-      const float hi_s = m - (float)k0 / scale, lo_s = m - (float)(k0 + 1) / scale;
-      const float margin = 1e-5f * (fabsf(m) + (float)kNB / scale + 1.f);
-      const unsigned long long kl = (unsigned long long)score_key(lo_s - margin) << kIdxBits;
-      const unsigned long long kh =
-          ((unsigned long long)score_key(hi_s + margin) << kIdxBits) | kIdxMask;
-      pbits = (kl == kh) ? kKeyBits : (__clzll(kl ^ kh) - (64 - kKeyBits));
-      prefix = pbits > 0 ? (kh >> (kKeyBits - pbits)) : 0ull;
-      n_cur = n_in;
-      state = next_state(n_in);
+      umin = fmaxf(2097152.0f * expf(-1.0f / scale) * (1.0f - 1.0f / 1024.0f) - 1.0f, 1.0f);
+      n_cur = bound(wsel);
+      range_prefix(m - (float)(k0 + 1) / scale, m - (float)k0 / scale, margin, pbits, prefix);
+      state = next_state(n_cur, true);
     }
     ebar();
     if (g == 0) clear_row(sm, r);
@@ -548,7 +603,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       int take = n;
       for (int a = 0; a < n; ++a) {
         const float sa = key_score((uint32_t)(sm.u.cand[a][r] >> kIdxBits));
-        acc += fixed21(__fmul_rn(rel_w(sa, m), tk));
+        acc += fixed_u(__fmul_rn(rel_w(sa, m), tk));
         cum = base + fk * (double)acc;
         if (cum >= T) {
           take = a + 1;
@@ -558,14 +613,19 @@ __global__ void __launch_bounds__(kThreads, 2)
       const unsigned long long last = sm.u.cand[take - 1][r];
       p.thr[o] = key_score((uint32_t)(last >> kIdxBits));
       p.jtie[o] = (int32_t)(kIdxMask - (last & kIdxMask));
-      p.count[o] = (int32_t)(cnt_above + (uint32_t)take);
+      p.count[o] = (int32_t)((int64_t)sm.nabove[r] + take);
       if (p.mass) p.mass[o] = (float)(cum / Z);
     };
 
-    // ---- sweeps 3+: refine the crossing bin 5 bits at a time, then collect
+    // ---- sweeps 3+: level-1 score sub-bins, then composite-key digits, until
+    // the crossing range is collected or parked
     for (int iter = 0;; ++iter) {
-      const bool mine = state == ST_REFINE || state == ST_COLLECT || state == ST_LIST;
-      if (g == 0) sm.ncnt[r] = 0;
+      const bool mine = state == ST_REFINE1 || state == ST_REFINE || state == ST_COLLECT ||
+                        state == ST_LIST;
+      if (g == 0) {
+        sm.ncnt[r] = 0;
+        sm.nabove[r] = 0;
+      }
       bool any = bar_or(1, kEpi, mine);
       if (any && iter >= kMaxIter) {
         if (tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 14);
@@ -576,79 +636,125 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&sm.ctl);
       }
       if (!any) break;
+      const int mode = state == ST_REFINE1  ? (int)MODE_SUB1
+                       : state == ST_REFINE ? (int)MODE_DIGIT
+                       : state == ST_COLLECT ? (int)MODE_COLLECT
+                                             : (int)MODE_PARK;
       const int w = min(kDigit, kKeyBits - pbits);
-      const int collect = state == ST_COLLECT ? 1 : (state == ST_LIST ? 2 : 0);
-      float lo = 0.f, hi = -1.f;
-      if (mine) refine_range(m, scale, k0, pbits, prefix, lo, hi);
+      float lo = INFINITY, hi = -INFINITY;
+      if (mine) refine_range(m, scale, margin, k0, k1, mode == MODE_SUB1 ? 0 : pbits, prefix, lo, hi);
+      // rows gathering their range count the keys above it: past hi here, the
+      // rest in drain_hits
+      const bool counting = mine && mode >= MODE_COLLECT;
+      const float hic = counting ? hi : INFINITY;
       const int wq = warp, row0 = (warp & 3) * 32;
       int qn = 0;  // entries in this warp's queue (warp-uniform)
+      uint32_t n_above = 0u;
+      auto drain = [&](int n) {
+        drain_hits(sm, lists, wq, n, row0, g, m, scale, k0, k1, pbits, prefix, w, tk, mode);
+      };
+      auto drain32 = [&]() {  // the queue's first 32 entries; the rest move down
+        __syncwarp();
+        drain(32);
+        __syncwarp();
+        if (lane + 32 < qn) {
+          sm.t.q.s[wq][lane] = sm.t.q.s[wq][lane + 32];
+          sm.t.q.jl[wq][lane] = sm.t.q.jl[wq][lane + 32];
+        }
+        __syncwarp();
+        qn -= 32;
+      };
       sweep(
           [&](int j0, float (&v)[kChunk]) {
-            const bool full = (int64_t)j0 + kChunk - 1 <= P;
             uint32_t hits = 0u;
 #pragma unroll
             for (int i = 0; i < kChunk; ++i) {
               const float s = v[i];
-              const bool h = mine & (s >= lo) & (s <= hi) & (full | ((int64_t)(j0 + i) <= P));
-              hits |= (h ? 1u : 0u) << i;
+              hits |= ((s >= lo) & (s <= hi) ? 1u : 0u) << i;
+              n_above += s > hic ? 1u : 0u;
             }
             if (__ballot_sync(0xffffffffu, hits != 0u) == 0u) return;
-            const uint32_t lt = (1u << lane) - 1u;
+            // -0 -> +0 below: one composite key per score
+            const int nh = __popc(hits);
+            int incl = nh;  // inclusive prefix sum of the lanes' hit counts
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-              const bool h = (hits >> i) & 1u;
-              const uint32_t bal = __ballot_sync(0xffffffffu, h);
-              if (bal == 0u) continue;
-              if (h) {  // -0 -> +0: one composite key per score
-                const int pos = qn + __popc(bal & lt);
-                sm.t.q.s[wq][pos] = v[i] + 0.0f;
-                sm.t.q.jl[wq][pos] = (uint32_t)(j0 + i) | ((uint32_t)lane << 21);
-              }
-              qn += __popc(bal);
-              if (qn >= 32) {
-                __syncwarp();
-                drain_hits(sm, lists, wq, 32, row0, m, scale, k0, pbits, prefix, w, tk, collect);
-                __syncwarp();
-                if (lane + 32 < qn) {
-                  sm.t.q.s[wq][lane] = sm.t.q.s[wq][lane + 32];
-                  sm.t.q.jl[wq][lane] = sm.t.q.jl[wq][lane + 32];
+            for (int o = 1; o < 32; o <<= 1) {
+              const int t = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += t;
+            }
+            const int total = __shfl_sync(0xffffffffu, incl, 31);
+            if (qn + total <= kQueue) {  // every lane writes its hits at once
+              int pos = qn + incl - nh;
+#pragma unroll
+              for (int i = 0; i < kChunk; ++i)
+                if ((hits >> i) & 1u) {
+                  sm.t.q.s[wq][pos] = v[i] + 0.0f;
+                  sm.t.q.jl[wq][pos] = (uint32_t)(j0 + i) | ((uint32_t)lane << 21);
+                  ++pos;
                 }
-                __syncwarp();
-                qn -= 32;
+              qn += total;
+              while (qn >= 32) drain32();
+            } else {  // a dense chunk: one key position at a time
+              const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+              for (int i = 0; i < kChunk; ++i) {
+                const bool h = (hits >> i) & 1u;
+                const uint32_t bal = __ballot_sync(0xffffffffu, h);
+                if (bal == 0u) continue;
+                if (h) {
+                  const int pos = qn + __popc(bal & lt);
+                  sm.t.q.s[wq][pos] = v[i] + 0.0f;
+                  sm.t.q.jl[wq][pos] = (uint32_t)(j0 + i) | ((uint32_t)lane << 21);
+                }
+                qn += __popc(bal);
+                if (qn >= 32) drain32();
               }
             }
           },
-          true, state == ST_REFINE);
-      if (qn > 0) {  // the last partial batch (row histograms flush below)
+          true, mine && mode <= MODE_DIGIT);
+      if (qn > 0) {  // the last partial batch
         __syncwarp();
-        drain_hits(sm, lists, wq, qn, row0, m, scale, k0, pbits, prefix, w, tk, collect);
+        drain(qn);
       }
+      if (counting) atomicAdd(&sm.nabove[r], (int)n_above);
       ebar();
-      if (state == ST_REFINE && g == 0) flush_row(sm, r);
+      if (g == 0 && mine && mode <= MODE_DIGIT) flush_row(sm, r);
       ebar();
-      // a row that parked its crossing range this sweep (a row that turns to
-      // ST_LIST below parks in the next sweep)
-      const bool lst = collect == 2 && mine;
+      // a row that parked its range this sweep (a row that turns to ST_LIST
+      // below parks in the next sweep)
+      const bool lst = mine && mode == MODE_PARK;
       const int nl = lst ? min(sm.ncnt[r], kListCap) : 0;
-      if (state == ST_COLLECT) {
+      auto fd = [&](int) { return fk; };
+      if (mine && mode == MODE_COLLECT) {
         if (g == 0) finish_row();
         state = ST_DONE;
-      } else if (state == ST_REFINE) {
-        uint32_t n_in = 0u;
-        auto fd = [&](int) { return fk; };
-        const int bsel = crossing(sm, r, 1 << w, T, false, fd, base, inner, cnt_above, n_in);
-        const int digit = (1 << w) - 1 - bsel;
-        prefix = (prefix << w) | (unsigned long long)digit;
+      } else if (mine && mode == MODE_SUB1) {
+        unsigned long long wsel = 0ull;
+        const int b1 = crossing(sm, r, kNB, T, false, fd, base, inner, wsel);
+        if (b1 < 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 17);
+        k1 = max(b1, 0);
+        const float s32 = scale * (float)kNB;
+        umin = fmaxf(2097152.0f * expf(-(float)(k1 + 1) / s32) * (1.0f - 1.0f / 1024.0f) - 1.0f,
+                     1.0f);
+        n_cur = bound(wsel);
+        range_prefix(m - (float)(kNB * k0 + k1 + 1) / s32, m - (float)(kNB * k0 + k1) / s32,
+                     margin, pbits, prefix);
+        state = next_state(n_cur, false);
+      } else if (mine && mode == MODE_DIGIT) {
+        unsigned long long wsel = 0ull;
+        const int bsel = crossing(sm, r, 1 << w, T, false, fd, base, inner, wsel);
+        if (bsel < 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 18);
+        prefix = (prefix << w) | (unsigned long long)((1 << w) - 1 - max(bsel, 0));
         pbits += w;
-        n_cur = n_in;
-        state = next_state(n_in);
+        n_cur = bound(wsel);
+        state = next_state(n_cur, false);
       }
       ebar();
       if (g == 0 && (state == ST_REFINE || (state == ST_LIST && !lst))) clear_row(sm, r);
-      // rows with a parked list: the remaining radix levels run over the list
+      // rows with a parked list: the remaining digit levels run over the list
       const unsigned long long* my = lst ? lists + (size_t)r * kListCap : nullptr;
       for (;;) {
-        const bool need = lst && n_cur > (uint32_t)kCap && pbits < kKeyBits;
+        const bool need = lst && n_cur > (unsigned long long)kCap && pbits < kKeyBits;
         if (!bar_or(1, kEpi, need)) break;
         const int wl = min(kDigit, kKeyBits - pbits);
         if (need) {
@@ -656,35 +762,40 @@ __global__ void __launch_bounds__(kThreads, 2)
             const unsigned long long ck = my[e];
             if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) continue;
             const int digit = (int)((ck >> (kKeyBits - pbits - wl)) & ((1ull << wl) - 1));
-            const int bin = (1 << wl) - 1 - digit;
             const float sc = key_score((uint32_t)(ck >> kIdxBits));
-            atomicAdd(&sm.wacc[bin][r], fixed21(__fmul_rn(rel_w(sc, m), tk)));
-            atomicAdd(&sm.hc[bin][r], 1u);
+            sm.wacc[g][(1 << wl) - 1 - digit][r] += fixed_u(__fmul_rn(rel_w(sc, m), tk));
           }
         }
         ebar();
         if (need && g == 0) flush_row(sm, r);
         ebar();
         if (need) {
-          uint32_t n_in = 0u;
-          auto fd = [&](int) { return fk; };
-          const int bsel = crossing(sm, r, 1 << wl, T, false, fd, base, inner, cnt_above, n_in);
-          prefix = (prefix << wl) | (unsigned long long)((1 << wl) - 1 - bsel);
+          unsigned long long wsel = 0ull;
+          const int bsel = crossing(sm, r, 1 << wl, T, false, fd, base, inner, wsel);
+          if (bsel < 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 19);
+          prefix = (prefix << wl) | (unsigned long long)((1 << wl) - 1 - max(bsel, 0));
           pbits += wl;
-          n_cur = n_in;
+          n_cur = bound(wsel);
         }
         ebar();
         if (need && g == 0) clear_row(sm, r);
       }
       if (g == 0 && lst) sm.ncnt[r] = 0;
       ebar();
-      if (lst)  // the final range's keys become the row's candidates
+      if (lst) {  // the final range's keys become the row's candidates
+        int above = 0;
         for (int e = g; e < nl; e += 2) {
           const unsigned long long ck = my[e];
-          if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) continue;
-          const int slot_c = atomicAdd(&sm.ncnt[r], 1);
-          if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
+          const unsigned long long px = pbits > 0 ? (ck >> (kKeyBits - pbits)) : 0ull;
+          if (px == prefix) {
+            const int slot_c = atomicAdd(&sm.ncnt[r], 1);
+            if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
+          } else if (px > prefix) {
+            ++above;
+          }
         }
+        atomicAdd(&sm.nabove[r], above);
+      }
       ebar();
       if (lst) {
         if (g == 0) finish_row();

@@ -86,10 +86,11 @@ struct SelSmem {
     unsigned long long hw[kNB][kBM];   // per-row bin sums (units of 2^-21 of a bin edge), row fastest
     unsigned long long cand[kCap][kBM];
   } u;
-  uint32_t wacc[2][kNB][kBM];          // bin sums of the current tile group, one copy per
-                                       // column half (the row's two threads)
+  uint32_t wacc[2][kNB + 1][kBM];      // bin sums of the current tile group, one copy per
+                                       // column half (the row's two threads); bin kNB
+                                       // collects the keys below c0 and is never read
   union {
-    float tab[kNB][kBM];               // exp(b / scale): level-0 bin b's edge factor
+    float tab[kNB + 1][kBM];           // 2^21 exp(b / scale): level-0 bin b's edge factor
     struct {                           // refine sweeps: per-warp queues of prefilter hits
       float s[kEpi / 32][kQueue];
       uint32_t jl[kEpi / 32][kQueue];  // key index | owner lane << 21
@@ -120,12 +121,15 @@ __device__ __forceinline__ float rel_w(float s, float m) {
 __device__ __forceinline__ uint32_t fixed_u(float x) {
   return __float_as_uint(__fadd_rz(fminf(x, 2097152.0f), 8388608.0f)) - 0x4B000000u;
 }
-// Level-0 bin of a score s <= m: floor((m - s) * scale), at most kNB - 1 (adding
-// 1.5 * 2^23 with rounding toward -inf leaves the floor in the low mantissa bits).
+// Level-0 bin of a score s <= m: floor((m - s) * scale), or kNB for a score at
+// or below c0 = m - kNB / scale (adding 1.5 * 2^23 with rounding toward -inf
+// leaves the floor in the low mantissa bits; larger or infinite products give
+// larger integers, clamped).  Keys below c0 + 1 are never kept, so the rounding
+// of that edge decides nothing.
 __device__ __forceinline__ int bin0_of(float s, float m, float scale) {
-  const float x = fminf(__fmul_rn(__fsub_rn(m, s), scale), 1048576.0f);
-  const int b = __float_as_int(__fadd_rd(x, 12582912.0f)) - 0x4B400000;
-  return b < kNB - 1 ? b : kNB - 1;
+  const int b = __float_as_int(__fadd_rd(__fmul_rn(__fsub_rn(m, s), scale), 12582912.0f)) -
+                0x4B400000;
+  return min(b, kNB);
 }
 
 __device__ __forceinline__ unsigned long long comp_key(float s, int j) {
@@ -237,12 +241,12 @@ enum { MODE_SUB1 = 0, MODE_DIGIT = 1, MODE_COLLECT = 2, MODE_PARK = 3 };
 // MODE_SUB1 adds the key to its level-1 sub-bin, MODE_DIGIT to its digit bin
 // (the next w composite-key bits), MODE_COLLECT makes it a candidate,
 // MODE_PARK stores it in the row's global list; the last two count the keys
-// above the range.  Histogram sums go to this warp's column-half copy.
+// above the range up to hic (the sweep counts those past it).  Histogram sums go to this warp's column-half copy.
 // Called by all 32 lanes.
 __device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, int wq, int n,
                                         int row0, int g, float m, float scale, int k0, int k1,
                                         int pbits, unsigned long long prefix, int w, float tk,
-                                        int mode) {
+                                        int mode, float hic) {
   const int lane = threadIdx.x & 31;
   const bool has = lane < n;
   const float s = has ? sm.t.q.s[wq][lane] : 0.f;
@@ -258,6 +262,7 @@ __device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, i
   const int ow = __shfl_sync(0xffffffffu, w, owner);
   const float otk = __shfl_sync(0xffffffffu, tk, owner);
   const int omode = __shfl_sync(0xffffffffu, mode, owner);
+  const float ohic = __shfl_sync(0xffffffffu, hic, owner);
   if (!has) return;
   const int r = row0 + owner;
   if (omode == MODE_SUB1) {
@@ -272,8 +277,8 @@ __device__ __noinline__ void drain_hits(SelSmem& sm, unsigned long long* list, i
     if (c != 0) return;
     const int digit = (int)((ck >> (kKeyBits - opb - ow)) & ((1ull << ow) - 1));
     atomicAdd(&sm.wacc[g][(1 << ow) - 1 - digit][r], fixed_u(__fmul_rn(rel_w(s, om), otk)));
-  } else if (c > 0) {
-    atomicAdd(&sm.nabove[r], 1);
+  } else if (c > 0) {  // keys past hic were counted by the sweep
+    if (s <= ohic) atomicAdd(&sm.nabove[r], 1);
   } else if (c == 0) {
     const int slot_c = atomicAdd(&sm.ncnt[r], 1);
     if (omode == MODE_PARK) {
@@ -495,17 +500,16 @@ __global__ void __launch_bounds__(kThreads, 2)
     sm.mpart[g][r] = m;
     ebar();
     m = fmaxf(sm.mpart[0][r], sm.mpart[1][r]);
-    float c0 = 0.f, scale = 1.f, margin = 0.f;
+    float scale = 1.f, margin = 0.f;
     if (valid) {
       const double N = (double)(P + 1);
       const float R = (float)(log(N / (1.0 - (double)p.p)) + 1.0);
-      c0 = m - R;
       scale = (float)kNB / R;
       margin = 1e-5f * (fabsf(m) + R + 1.f);
     }
     if (g == 0) {
       clear_row(sm, r);
-      for (int bb = 0; bb < kNB; ++bb) sm.t.tab[bb][r] = 2097152.0f * expf((float)bb / scale);
+      for (int bb = 0; bb <= kNB; ++bb) sm.t.tab[bb][r] = 2097152.0f * expf((float)bb / scale);
     }
     ebar();
 
@@ -516,14 +520,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         [&](int, float (&v)[kChunk]) {
           if (!valid) return;
           float e[kChunk];
+          int bb[kChunk];
 #pragma unroll
           for (int i = 0; i < kChunk; ++i) {
-            const float s = v[i];
-            e[i] = rel_w(s, m);
-            const int bb = bin0_of(s, m, scale);
-            const uint32_t u = fixed_u(__fmul_rn(e[i], sm.t.tab[bb][r]));
-            sm.wacc[g][bb][r] += s >= c0 ? u : 0u;
+            e[i] = rel_w(v[i], m);
+            bb[i] = bin0_of(v[i], m, scale);  // kNB: below c0, a bin never read
           }
+          float t[kChunk];  // every edge factor is read before the first store
+#pragma unroll
+          for (int i = 0; i < kChunk; ++i) t[i] = sm.t.tab[bb[i]][r];
+          // no-return atomics: the stores of one chunk need not wait for each other
+#pragma unroll
+          for (int i = 0; i < kChunk; ++i)
+            atomicAdd(&sm.wacc[g][bb[i]][r], fixed_u(__fmul_rn(e[i], t[i])));
 #pragma unroll
           for (int w = kChunk / 2; w >= 1; w >>= 1)
 #pragma unroll
@@ -647,11 +656,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       // rest in drain_hits
       const bool counting = mine && mode >= MODE_COLLECT;
       const float hic = counting ? hi : INFINITY;
+      // the prefilter |s - mid| <= half holds for every score in [lo, hi] (half
+      // is rounded up); keys past hi that pass it are told apart in drain_hits
+      float mid = 0.f, half = -1.f;
+      if (mine) {
+        mid = 0.5f * (lo + hi);
+        half = __fmul_ru(__fsub_ru(hi, lo), 0.5f * (1.0f + 1.0f / 1048576.0f)) +
+               fabsf(mid) * (1.0f / 4194304.0f) + 1e-30f;
+        if (!(fabsf(mid) < INFINITY) || !(half < INFINITY)) {  // unbounded range
+          mid = 0.f;
+          half = INFINITY;
+        }
+      }
       const int wq = warp, row0 = (warp & 3) * 32;
       int qn = 0;  // entries in this warp's queue (warp-uniform)
       uint32_t n_above = 0u;
       auto drain = [&](int n) {
-        drain_hits(sm, lists, wq, n, row0, g, m, scale, k0, k1, pbits, prefix, w, tk, mode);
+        drain_hits(sm, lists, wq, n, row0, g, m, scale, k0, k1, pbits, prefix, w, tk, mode, hic);
       };
       auto drain32 = [&]() {  // the queue's first 32 entries; the rest move down
         __syncwarp();
@@ -666,14 +687,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       };
       sweep(
           [&](int j0, float (&v)[kChunk]) {
-            uint32_t hits = 0u;
+            bool hit = false;
 #pragma unroll
             for (int i = 0; i < kChunk; ++i) {
-              const float s = v[i];
-              hits |= ((s >= lo) & (s <= hi) ? 1u : 0u) << i;
-              n_above += s > hic ? 1u : 0u;
+              hit |= fabsf(__fsub_rn(v[i], mid)) <= half;
+              n_above += v[i] > hic ? 1u : 0u;
             }
-            if (__ballot_sync(0xffffffffu, hits != 0u) == 0u) return;
+            if (__ballot_sync(0xffffffffu, hit) == 0u) return;
+            uint32_t hits = 0u;
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i)
+              hits |= (fabsf(__fsub_rn(v[i], mid)) <= half ? 1u : 0u) << i;
             // -0 -> +0 below: one composite key per score
             const int nh = __popc(hits);
             int incl = nh;  // inclusive prefix sum of the lanes' hit counts

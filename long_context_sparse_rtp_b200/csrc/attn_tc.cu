@@ -81,6 +81,15 @@ struct Sched {
   }
 };
 
+// The largest float below t (t = -inf stays -inf; no denormal flushing, so the
+// float below 0 is the negative least denormal and s > it iff s >= 0).
+__device__ __forceinline__ float float_below(float t) {
+  if (!(t > -INFINITY)) return t;
+  if (t == 0.f) return __uint_as_float(0x80000001u);
+  const uint32_t u = __float_as_uint(t);
+  return __uint_as_float(t > 0.f ? u - 1u : u + 1u);
+}
+
 __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -271,13 +280,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the tile's scores, masked and scaled into the log2 domain
       float x[kBN];
       if (sparse) {
-        // the indexer predicate per 32-key chunk: s16 > t, or s16 == t and j <= jtie;
-        // key offsets i within the tile: i <= ptl (causal), i <= jtl (may keep a tie);
-        // -0 and +0 compare equal, so the scores need no canonical form here
+        // the indexer predicate: s16 > t, or s16 == t and j <= jtie; causal j <= P.
+        // One compare per key against te = t, or the float below t where the tie
+        // index lies past the tile (every tie kept); the tile holding a lane's tie
+        // index and the diagonal tile take one more select per key
         auto clamp_off = [](int64_t d) {
           return (int)(d < -1 ? -1 : (d > kBN - 1 ? kBN - 1 : d));
         };
         const int ptl = clamp_off(P - j0), jtl = clamp_off(jt - j0);
+        const float te = !ok ? INFINITY : (jtl == kBN - 1 ? float_below(thr) : thr);
+        const bool mixed = __any_sync(0xffffffffu, (jtl >= 0) & (jtl < kBN - 1));
+        const bool diag = __any_sync(0xffffffffu, ptl < kBN - 1);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t r16[32], rs[32];
@@ -290,12 +303,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) {
             reg_fence(r16[i]);
             reg_fence(rs[i]);
-            const int ii = c * 32 + i;
-            const float s16 = __uint_as_float(r16[i]);
-            // bitwise, not short-circuit: a select per key, no divergent branch
-            const bool kp = ok & ((s16 > thr) | ((s16 == thr) & (ii <= jtl))) & (ii <= ptl);
-            x[ii] = kp ? __uint_as_float(rs[i]) * p.scale_log2 : -INFINITY;
+            x[c * 32 + i] = __uint_as_float(r16[i]) > te ? __uint_as_float(rs[i]) * p.scale_log2
+                                                          : -INFINITY;
           }
+          if (mixed) {  // ties up to the tie index (-0 and +0 compare equal)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const bool tie = ok & (__uint_as_float(r16[i]) == thr) & (c * 32 + i <= jtl);
+              x[c * 32 + i] = tie ? __uint_as_float(rs[i]) * p.scale_log2 : x[c * 32 + i];
+            }
+          }
+        }
+        if (diag) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i) x[i] = i <= ptl ? x[i] : -INFINITY;
         }
         tc_fence_before();  // S16 is in registers: the MMA may reuse its buffer
         __syncwarp();

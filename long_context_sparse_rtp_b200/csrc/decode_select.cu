@@ -26,6 +26,7 @@
 #include <algorithm>
 
 #include "rtp_host.h"
+#include "tcgen05.cuh"
 #include "tma.cuh"
 
 namespace rtp {
@@ -87,23 +88,33 @@ __device__ __forceinline__ float key_score(uint32_t key) {
 }
 
 // ------------------------------------------------------------------ 1. score + histogram
-// Persistent, TMA-fed.  Work items are (kv group, 512 consecutive keys); a CTA
-// takes items blockIdx.x, blockIdx.x + gridDim.x, ...  One producer thread
-// streams each item's k16 rows as boxes of T keys x kw slots into a ring of
-// shared-memory stages; 8 consumer warps compute the scores,
-// then per item: the heads' max bins, the scores' store, a 256-bin window
-// histogram per head in shared memory and its flush into the row's absolute
-// histogram.  The producer keeps the ring full across those phases.
-//
-// The scores are a batched 16-element dot product per (key, head), which is
-// CUDA-core FMA work; the box is 128-byte swizzled when its rows are 128 bytes
-// or wider, so that the 32 lanes' 16-byte loads of 32 consecutive pairs hit
-// every bank once.
-constexpr int kSItem = 512;                      // keys per work item
-constexpr int kSStages = 4;
-constexpr int kSStageBytes = 16384;
-constexpr int kSConsumers = 256;                 // 8 warps
-constexpr int kSThreads = kSConsumers + 32;      // + the producer warp
+// Persistent, TMA-fed, scores on the tensor cores.  Work items are (kv group,
+// 512 consecutive keys); a CTA takes a contiguous run of items.  Per 128-key
+// sub-tile the producer warp loads the group's kw k16 slots into a ring stage,
+// as [128 x 64] four-slot tiles (128-byte swizzled) when kw >= 4, else as kw
+// [128 x 16] tiles (32-byte swizzled), both the MMA's K-major layouts,
+// and writes the matching [16 x 16] query blocks: slot h's block holds q16 of
+// head h in row h (k16 per query head), or the G heads' q16 in rows 0..G-1 (one
+// k16 per kv head); every other row stays zero.  The MMA warp issues one
+// tcgen05.mma per slot (M = 128, N = 16, K = 16), accumulating
+// D[key][head] = q16_head . k16_(key, head's slot) in TMEM: the zero blocks add
+// exact zeros, so each score is the 16-term dot product of a single MMA, as in
+// the prefill selection.  The 8 consumer warps read D, then per item: the heads'
+// max bins, the scores' store, a 256-bin window histogram per head in shared
+// memory and its flush into the row's absolute histogram.  Producer and MMA run
+// ahead across items, bounded by the ring and by 8 TMEM accumulators.
+constexpr int kSItem = 512;                   // keys per work item
+constexpr int kSTile = 128;                   // keys per MMA (M)
+constexpr int kSN = 16;                       // MMA N: a group's heads, zero-padded
+constexpr int kSChunkA = kSTile * kR * 2;     // 4096 B: one slot of a sub-tile
+constexpr int kSChunkB = kSN * kR * 2;        // 512 B: one query block
+constexpr int kSBufs = 8;                     // TMEM accumulators, kSN columns each
+constexpr int kSConsumers = 256;              // 8 warps
+constexpr int kSProdWarp = kSConsumers / 32, kSMmaWarp = kSProdWarp + 1;
+constexpr int kSThreads = kSConsumers + 64;   // + the producer and MMA warps
+constexpr int kSRingBytes = 74 * 1024;
+constexpr int kSMaxStages = 8;
+constexpr uint32_t kSIdesc = idesc_bf16_f32(kSTile, kSN);
 
 struct ScoreParams {
   const uint16_t* q16;
@@ -117,32 +128,48 @@ struct ScoreParams {
   uint32_t* mcount;
   DevStatus* status;
   int N, Lk_pad, n_ret, n_rkv, G, lgG, per_kv, rows, groups;
-  int T;             // keys per box (a multiple of 16 dividing kSItem)
-  int kw;            // k16 slots per key in a box: G, or 1 when k16 is per kv head
-  int swz;           // 1: the box is 128-byte swizzled (rows of kw x 32 bytes, kw >= 4)
+  int kw;            // k16 slots per key of a group: G, or 1 when k16 is per kv head
+  int stages;        // ring stages (one sub-tile each)
+  int quad;          // 1: kw >= 4, the slots load as four-slot 128-byte-swizzled boxes
   int batch_coord;   // 1, or 0 when every batch entry shares one k16 cache
   int items_per_group, n_items;
 };
 
 struct ScoreSmemTail {
-  uint64_t full[kSStages];
-  uint64_t empty[kSStages];
+  uint64_t full[kSMaxStages];
+  uint64_t empty[kSMaxStages];
+  uint64_t tfull[kSBufs];
+  uint64_t tempty[kSBufs];
+  int bgrp[kSMaxStages];  // the group whose query blocks a stage holds (-1: none yet)
   int top[16];
+  uint32_t tmem_base;
   int gave_up;
 };
 
-__host__ __device__ constexpr size_t score_smem_bytes(int G) {
-  return 1024 + (size_t)kSStages * kSStageBytes + (size_t)G * (kSItem + 4) * 4 +
-         (size_t)G * kDecWin * 8 + sizeof(ScoreSmemTail);
+// A stage: kw slot tiles, then kw query blocks; 1024-byte multiples.
+__host__ __device__ constexpr int score_stage_bytes(int kw) {
+  return (kw * (kSChunkA + kSChunkB) + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr int score_stages(int kw) {
+  return kSRingBytes / score_stage_bytes(kw) < 2
+             ? 2
+             : (kSRingBytes / score_stage_bytes(kw) > kSMaxStages
+                    ? kSMaxStages
+                    : kSRingBytes / score_stage_bytes(kw));
+}
+__host__ __device__ constexpr size_t score_smem_bytes(int G, int kw) {
+  return 1024 + (size_t)score_stages(kw) * score_stage_bytes(kw) +
+         (size_t)G * (kSItem + 4) * 4 + (size_t)G * kDecWin * 8 + sizeof(ScoreSmemTail);
 }
 
 __global__ void __launch_bounds__(kSThreads, 2)
     dec_score_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int G = p.G;
+  const int G = p.G, kw = p.kw;
+  const int sbytes = score_stage_bytes(kw);
   // stages on a 1024-byte boundary (score_smem_bytes includes the slack)
   unsigned char* ring = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  float* sc = reinterpret_cast<float*>(ring + kSStages * kSStageBytes);  // [G][kSItem+4]
+  float* sc = reinterpret_cast<float*>(ring + p.stages * sbytes);         // [G][kSItem+4]
   uint32_t* hm = reinterpret_cast<uint32_t*>(sc + G * (kSItem + 4));     // [G][kDecWin]
   uint32_t* hc = hm + G * kDecWin;
   ScoreSmemTail* tl = reinterpret_cast<ScoreSmemTail*>(hc + G * kDecWin);
@@ -159,128 +186,183 @@ __global__ void __launch_bounds__(kSThreads, 2)
     hm[x] = 0u;
     hc[x] = 0u;
   }
+  // query blocks start zero: a group writes only its heads' rows
+  for (int s = 0; s < p.stages; ++s)
+    for (int x = tid; x < kw * kSChunkB / 16; x += kSThreads)
+      *reinterpret_cast<uint4*>(ring + s * sbytes + kw * kSChunkA + x * 16) = make_uint4(0, 0, 0, 0);
+  fence_async_smem();
   if (tid == 0) {
-    for (int s = 0; s < kSStages; ++s) {
+    for (int s = 0; s < p.stages; ++s) {
       mbar_init(&tl->full[s], 1);
-      mbar_init(&tl->empty[s], kSConsumers / 32);
+      mbar_init(&tl->empty[s], 1);
+      tl->bgrp[s] = -1;
+    }
+    for (int i = 0; i < kSBufs; ++i) {
+      mbar_init(&tl->tfull[i], 1);
+      mbar_init(&tl->tempty[i], 4);  // the four warps that read one accumulator
     }
     tl->gave_up = 0;
     fence_mbar_init();
   }
+  if (warp == kSMmaWarp) {
+    tmem_alloc(&tl->tmem_base, kSBufs * kSN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tl->tmem_base;
   volatile int* gave_up = &tl->gave_up;
-  const int box_bytes = p.T * p.kw * 32;
+  // a contiguous run of items per CTA: consecutive items share their kv group
+  const int per_cta = (p.n_items + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int it0 = (int)blockIdx.x * per_cta, it1 = min(it0 + per_cta, p.n_items);
 
-  if (warp == kSConsumers / 32) {  // ---------------- producer
+  if (warp == kSProdWarp) {  // ---------------- producer (the whole warp)
+    int stage = 0, n_issued = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int item = it0; ok && item < it1; ++item) {
+      const int grp = item / p.items_per_group, j0 = (item % p.items_per_group) * kSItem;
+      const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
+      const int nvalid = max(0, min(kSItem, p.N - j0));
+      const int nsub = (nvalid + kSTile - 1) / kSTile;
+      const int slot0 = p.per_kv ? rk : rk * G;
+      for (int st = 0; st < nsub; ++st) {
+        if (!mbar_wait_warp(&tl->empty[stage], ph ^ 1u, gave_up)) {
+          ok = false;
+          break;
+        }
+        unsigned char* sb = ring + stage * sbytes;
+        if (tl->bgrp[stage] != grp) {  // this stage's query blocks: the group's q16 rows
+          for (int e = lane; e < 2 * G; e += 32) {
+            const int h = e >> 1, c = e & 1;  // head, 16-byte half of its row
+            const uint4 v = *reinterpret_cast<const uint4*>(p.q16 + b * p.q16_sb +
+                                                            (int64_t)(rk * G + h) * kR + c * 8);
+            const int blk = p.per_kv ? 0 : h;
+            // 32-byte swizzle: the halves of rows 4..7 of every 8 swap
+            const int off = h * 32 + ((c ^ ((h >> 2) & 1)) << 4);
+            *reinterpret_cast<uint4*>(sb + kw * kSChunkA + blk * kSChunkB + off) = v;
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) tl->bgrp[stage] = grp;
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&tl->full[stage], (uint32_t)(kw * kSChunkA));
+          if (p.quad) {  // four slots (128-byte rows) per box
+            for (int qd = 0; qd < kw / 4; ++qd)
+              tma_load_4d(sb + qd * 4 * kSChunkA, &kmap, 0, slot0 / 4 + qd, j0 + st * kSTile,
+                          b * p.batch_coord, &tl->full[stage]);
+          } else {
+            for (int h = 0; h < kw; ++h)
+              tma_load_4d(sb + h * kSChunkA, &kmap, 0, slot0 + h, j0 + st * kSTile,
+                          b * p.batch_coord, &tl->full[stage]);
+          }
+        }
+        ++n_issued;
+        if (++stage == p.stages) {
+          stage = 0;
+          ph ^= 1u;
+        }
+      }
+    }
     if (lane == 0) {
-      int stage = 0, n_issued = 0;
-      uint32_t ph = 0;
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 20);
+      // every copy still in flight lands before the CTA may exit
+      for (int k = max(0, n_issued - p.stages); k < n_issued; ++k)
+        mbar_wait_drain(&tl->full[k % p.stages], (uint32_t)(k / p.stages) & 1u);
+    }
+    return;
+  }
+  if (warp == kSMmaWarp) {  // ---------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0, seq = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const int grp = item / p.items_per_group, j0 = (item % p.items_per_group) * kSItem;
-        const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
-        const int nvalid = max(0, min(kSItem, p.N - j0));
-        const int nb = (nvalid + p.T - 1) / p.T;
-        const int slot0 = p.per_kv ? rk : rk * G;
-        // swizzled maps count 64-element (4-slot) quads in dim 1; others slots x 16 in dim 0
-        const int c0 = p.swz ? 0 : slot0 * kR, c1 = p.swz ? slot0 / 4 : 0;
-        for (int bx = 0; bx < nb; ++bx) {
-          if (!mbar_wait(&tl->empty[stage], ph ^ 1u, gave_up)) {
+      for (int item = it0; ok && item < it1; ++item) {
+        const int j0 = (item % p.items_per_group) * kSItem;
+        const int nsub = (max(0, min(kSItem, p.N - j0)) + kSTile - 1) / kSTile;
+        for (int st = 0; st < nsub; ++st) {
+          const uint32_t buf = seq % kSBufs;
+          if (!mbar_wait(&tl->full[stage], ph, gave_up) ||
+              !mbar_wait(&tl->tempty[buf], ((seq / kSBufs) & 1u) ^ 1u, gave_up)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tl->full[stage], (uint32_t)box_bytes);
-          tma_load_4d(ring + stage * kSStageBytes, &kmap, c0, c1, j0 + bx * p.T,
-                      b * p.batch_coord, &tl->full[stage]);
-          ++n_issued;
-          if (++stage == kSStages) {
+          tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * sbytes);
+          for (int h = 0; h < kw; ++h) {
+            // slot h: its own 32-byte-swizzled tile, or the 16-element K step h % 4
+            // of a 128-byte-swizzled four-slot tile
+            const uint64_t adesc =
+                p.quad ? sdesc_sw128(sa + (uint32_t)((h >> 2) * 4 * kSChunkA + (h & 3) * 32), 16,
+                                     1024)
+                       : sdesc_k_sw32(sa + (uint32_t)(h * kSChunkA), 256);
+            mma_bf16_ss(tmem + buf * kSN, adesc,
+                        sdesc_k_sw32(sa + (uint32_t)(kw * kSChunkA + h * kSChunkB), 256), kSIdesc,
+                        h > 0);
+          }
+          mma_commit(&tl->empty[stage]);  // the stage is free once the MMAs have read it
+          mma_commit(&tl->tfull[buf]);    // the accumulator is ready
+          ++seq;
+          if (++stage == p.stages) {
             stage = 0;
             ph ^= 1u;
           }
         }
       }
-      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 20);
-      // every copy still in flight lands before the CTA may exit
-      for (int k = max(0, n_issued - kSStages); k < n_issued; ++k)
-        mbar_wait_drain(&tl->full[k % kSStages], (uint32_t)(k / kSStages) & 1u);
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 22);
+      if (seq > 0)  // the last MMAs are complete before TMEM is released
+        mbar_wait_drain(&tl->tfull[(seq - 1) % kSBufs], ((seq - 1) / kSBufs) & 1u);
     }
+    __syncwarp();
+    tc_fence_before();
+    named_bar(2, kSConsumers + 32);  // the consumers are done with TMEM
+    tc_fence_after();
+    tmem_dealloc(tmem, kSBufs * kSN);
     return;
   }
 
   // ---------------- consumers (threads 0..255; named barrier 1)
-  const int hh = tid & (G - 1);         // G divides 256: constant per thread
-  const int hoff = p.per_kv ? 0 : hh;   // the head's k16 slot within the key's row
-  int stage = 0;
-  uint32_t ph = 0;
+  const int hh = tid & (G - 1);  // G divides 256: constant per thread
+  uint32_t sub_base = 0;         // sub-tiles of the earlier items (the MMA's sequence)
   bool ok = true;
-  for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+  for (int item = it0; item < it1; ++item) {
     const int grp = item / p.items_per_group, j0 = (item % p.items_per_group) * kSItem;
     const int b = grp / p.n_rkv, rk = grp % p.n_rkv;
     const int row0 = b * p.n_ret + rk * G;
     const int nvalid = max(0, min(kSItem, p.N - j0));
-    const int nb = (nvalid + p.T - 1) / p.T;
-    float q[kR];  // q16 of this thread's head hh
-    {
-      const uint16_t* qp = p.q16 + b * p.q16_sb + (int64_t)(rk * G + hh) * kR;
-      const uint4 a = *reinterpret_cast<const uint4*>(qp);
-      const uint4 c = *reinterpret_cast<const uint4*>(qp + 8);
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        q[2 * i] = bf16_lo(w[i]);
-        q[2 * i + 1] = bf16_hi(w[i]);
-      }
-    }
-    const int pairs = p.T * G;  // (key, head) pairs per box
+    const int nsub = (nvalid + kSTile - 1) / kSTile;
     float* scrow = sc + hh * (kSItem + 4);
-    for (int bx = 0; bx < nb; ++bx) {
-      ok = ok && mbar_wait_warp(&tl->full[stage], ph, gave_up);
-      if (ok) {
-        const unsigned char* buf = ring + stage * kSStageBytes;
-        const int lim = p.N - j0 - bx * p.T;  // keys of this box below N
-        // two pairs per pass, each dot as two chains (even / odd dims) summed at
-        // the end: a fixed order, four independent FMA chains
-        for (int pr = tid; pr < pairs; pr += 2 * kSConsumers) {
-          const bool second = pr + kSConsumers < pairs;
-          const int xk0 = pr >> p.lgG, xk1 = second ? (pr + kSConsumers) >> p.lgG : xk0;
-          uint4 kv[2][2];
+    // the item's scores: warps 0-3 read sub-tiles 0 and 1, warps 4-7 sub-tiles 2
+    // and 3, each its TMEM lane quarter (one key per lane, the heads in columns);
+    // keys past N read as -inf
+#pragma unroll 1
+    for (int u = 0; u < 2; ++u) {
+      const int st = (warp >> 2) * 2 + u;
+      const int x = st * kSTile + (warp & 3) * 32 + lane;
+      float d[kSN];
+      if (st < nsub) {
+        const uint32_t seq = sub_base + (uint32_t)st, buf = seq % kSBufs;
+        ok = ok && mbar_wait_warp(&tl->tfull[buf], (seq / kSBufs) & 1u, gave_up);
+        tc_fence_after();
+        if (ok) {
+          tmem_ld16(tmem + ((uint32_t)((warp & 3) * 32) << 16) + buf * kSN, d);
+        } else {
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t lin = (uint32_t)(((u ? xk1 : xk0) * p.kw + hoff) * 32);
-            const uint32_t o = p.swz ? swizzle128(lin) : lin;  // bytes 16..31 sit at o ^ 16
-            kv[u][0] = *reinterpret_cast<const uint4*>(buf + o);
-            kv[u][1] = *reinterpret_cast<const uint4*>(buf + (o ^ 16u));
-          }
-          float se[2] = {0.f, 0.f}, so[2] = {0.f, 0.f};
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const uint4& kk = kv[u][c >> 2];
-              const uint32_t w =
-                  (c & 3) == 0 ? kk.x : (c & 3) == 1 ? kk.y : (c & 3) == 2 ? kk.z : kk.w;
-              se[u] = fmaf(q[2 * c], bf16_lo(w), se[u]);
-              so[u] = fmaf(q[2 * c + 1], bf16_hi(w), so[u]);
-            }
-          }
-          scrow[bx * p.T + xk0] = (xk0 < lim) ? __fadd_rn(se[0], so[0]) + 0.0f : -INFINITY;
-          if (second)
-            scrow[bx * p.T + xk1] = (xk1 < lim) ? __fadd_rn(se[1], so[1]) + 0.0f : -INFINITY;
+          for (int h = 0; h < kSN; ++h) d[h] = 0.f;
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tl->tempty[buf]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tl->empty[stage]);
-      if (++stage == kSStages) {
-        stage = 0;
-        ph ^= 1u;
-      }
+      const bool in = st < nsub && x < nvalid;
+#pragma unroll
+      for (int h = 0; h < kSN; ++h)
+        if (h < G) sc[h * (kSItem + 4) + x] = in ? d[h] + 0.0f : -INFINITY;  // -0 -> +0
     }
-    // keys of the item past the last box (past N): -inf
-    if (nb * p.T < kSItem)
-      for (int idx = tid; idx < G * kSItem; idx += kSConsumers) {
-        const int h = idx / kSItem, x = idx % kSItem;
-        if (x >= nb * p.T) sc[h * (kSItem + 4) + x] = -INFINITY;
-      }
+    sub_base += (uint32_t)nsub;
     named_bar(1, kSConsumers);
     for (int h = warp; h < G; h += kSConsumers / 32) {  // max bin per head, scores' store
       const float* row = sc + h * (kSItem + 4);
@@ -348,6 +430,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
   }
   if (!ok && tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 21);
+  tc_fence_before();
+  named_bar(2, kSConsumers + 32);  // TMEM may be released
 }
 
 // ------------------------------------------------------------------ 2. per-row merge
@@ -1122,43 +1206,45 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     sp.rows = L.rows;
     sp.groups = groups;
     sp.kw = k16_per_kv_head ? 1 : hm.G;
-    sp.swz = sp.kw >= 4 ? 1 : 0;
-    sp.T = std::min(256, kSStageBytes / (sp.kw * kR * 2));  // divides kSItem
+    sp.stages = score_stages(sp.kw);
+    sp.quad = sp.kw >= 4 ? 1 : 0;  // kw >= 4: group slots start at a multiple of 4
     sp.batch_coord = (k16_cache.stride_b != 0 || shape->B == 1) ? 1 : 0;
     sp.items_per_group = L.Lk_pad / kSItem;
     sp.n_items = groups * sp.items_per_group;
-    // k16 as a 4-D tensor; keys past N read as 0.  Swizzled: {64 elements (4
-    // slots), slots / 4, keys 0..N-1, batch}; else {slots x 16, 1, keys, batch}.
+    // k16 as a 4-D tensor {16 x slots per box, slot boxes, keys 0..N-1, batch}
+    // (keys past N read as 0); boxes of 128 keys x one slot (32-byte swizzled) or
+    // x four slots (128-byte swizzled)
     CUtensorMap kmap;
     const uint64_t sl_bytes = (uint64_t)k16_cache.stride_l * 2;
     const uint64_t sb_bytes =
         sp.batch_coord && k16_cache.stride_b != 0 ? (uint64_t)k16_cache.stride_b * 2 : sl_bytes * N;
     const uint64_t nbatch = sp.batch_coord ? (uint64_t)shape->B : 1u;
-    const uint64_t row_el = (uint64_t)hm.H_k16 * kR;
-    uint64_t dims[4], strides[3];
-    uint32_t box[4];
-    if (sp.swz) {
-      dims[0] = 64; dims[1] = row_el / 64; dims[2] = (uint64_t)N; dims[3] = nbatch;
-      strides[0] = 128; strides[1] = sl_bytes; strides[2] = sb_bytes;
-      box[0] = 64; box[1] = (uint32_t)(sp.kw / 4); box[2] = (uint32_t)sp.T; box[3] = 1;
-    } else {
-      dims[0] = row_el; dims[1] = 1; dims[2] = (uint64_t)N; dims[3] = nbatch;
-      strides[0] = sl_bytes; strides[1] = sl_bytes; strides[2] = sb_bytes;
-      box[0] = (uint32_t)(sp.kw * kR); box[1] = 1; box[2] = (uint32_t)sp.T; box[3] = 1;
-    }
-    if (!tma_encode_bf16(&kmap, k16_cache.ptr, 4, dims, strides, box, sp.swz ? 128 : 0))
+    const uint64_t dims[4] = {sp.quad ? 64u : 16u,
+                              (uint64_t)hm.H_k16 / (sp.quad ? 4u : 1u), (uint64_t)N, nbatch};
+    const uint64_t strides[3] = {sp.quad ? 128u : 32u, sl_bytes, sb_bytes};
+    const uint32_t box[4] = {sp.quad ? 64u : 16u, 1, (uint32_t)kSTile, 1};
+    if (!tma_encode_bf16(&kmap, k16_cache.ptr, 4, dims, strides, box, sp.quad ? 128 : 32))
       return RTP_ERR_CUDA;
-    const size_t smem = score_smem_bytes(hm.G);
+    const size_t smem = score_smem_bytes(hm.G, sp.kw);
+    // the whole carveout as shared memory: two CTAs per SM for kw <= 8
     if (cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+                             (int)smem) != cudaSuccess ||
+        cudaFuncSetAttribute(dec_score_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return RTP_ERR_CUDA;
-    int dev = 0, n_sm = 0, per_sm = 0;
+    // CTAs per SM: two by the launch bounds, fewer if shared memory says so (the
+    // occupancy query counts a TMEM-allocating kernel as one per SM; two CTAs
+    // hold 2 x 128 of the 512 TMEM columns)
+    int dev = 0, n_sm = 0, smem_sm = 0, smem_res = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dec_score_kernel, kSThreads,
-                                                      smem) != cudaSuccess)
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+            cudaSuccess)
       return RTP_ERR_CUDA;
-    const int grid = std::max(1, std::min(sp.n_items, std::max(1, per_sm) * n_sm));
+    const int per_sm = std::max(1, std::min(2, smem_sm / ((int)smem + smem_res)));
+    const int grid = std::max(1, std::min(sp.n_items, per_sm * n_sm));
     TraceScope tr("dec_score", s);
     dec_score_kernel<<<grid, kSThreads, smem, s>>>(kmap, sp);
     if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;

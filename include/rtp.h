@@ -195,19 +195,19 @@ RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role
  * For callers that cannot hand the library a workspace: code that runs under a
  * memory allocator it does not own (a host framework's fixed pool, a plugin
  * interface that passes only inputs and outputs) or in a phase where device
- * allocation is not allowed.  The split-KV partials and merge counters live in
+ * allocation is not allowed.  The split-KV partials live in
  * one file-scope device array of RTP_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU
  * which loads the library holds until the process exits.
  *  - Same arguments and results as rtp_local_attn for one decode token, minus
  *    the workspace.  Shapes whose partials exceed the array return
  *    RTP_ERR_SCRATCH_LIMIT before anything is enqueued (the need is about
- *    8320 bytes per (batch entry, local kv head, split), with
+ *    8448 bytes per (batch entry, local kv head, split), with
  *    min(ceil(296 / (B * local_kv_heads)), ceil(n_keys / 64)) splits; n_keys
  *    is the number of sink and window keys, at most window + n_sink).
  *  - The first call on a device looks the array's device address up
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    outside any stream capture.
- *  - Every call reuses the same array and clears the counters it needs; calls
+ *  - Every call reuses the same array; calls
  *    that overlap on the GPU (other streams, other threads) race on it and
  *    must be serialised by the caller.
  *  - Never calls cudaMalloc, cudaFree or any allocating routine.

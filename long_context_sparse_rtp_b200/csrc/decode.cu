@@ -3,19 +3,15 @@
 //
 // Retrieval decode for one query token per batch entry ("Dynamic Top-p
 // Selection Mechanism" and the decode flow of the paper-graph-ui summary of
-// arXiv 2605.16928), per kv group of G query heads:
-//   1. score     stream the k16 cache once (HBM-bound), s = q16 . k16 in fp32,
-//                scores kept in the workspace (L2-resident), chunk maxima;
-//   2. histogram Z and a 256-bin mass histogram above c0 = m - ln(N/(1-p)) - 1,
-//                40-bit fixed-point sums (exact, order-free); the last CTA of a
-//                row (arrival counter) finds the crossing bin, collects the keys
-//                in it, sorts them and walks to the exact cut (t, jtie);
-//   3. compact   one ordered list per kv group of the union of kept keys with a
-//                per-head bit mask (the kv-level "memory sparsity" set);
-//   4. attend    split-KV over the list: gathered K/V rows staged in shared
-//                memory with 16-byte cp.async, tensor-core QK^T / PV with the
-//                G heads as mma rows, per-head masks, online softmax; the last
-//                CTA of a group merges the splits.
+// arXiv 2605.16928), per kv group of G query heads: the scores, the exact cut
+// and the kept-key union list come from decode_select.cu; this file holds the
+// attention over that list and over sink + window ranges:
+//   attend   split-KV over the list (or the range): gathered K/V rows staged in
+//            shared memory with 16-byte cp.async, tensor-core QK^T / PV with the
+//            G heads as mma rows, per-head masks, online softmax, one partial
+//            (m, l, o) per split;
+//   merge    a second kernel, one CTA per (batch, kv group, head), combines the
+//            splits in split order.
 #include <algorithm>
 #include <mutex>
 
@@ -53,7 +49,6 @@ struct DecAttnParams {
   // range mode
   int64_t P; int n_sink_eff; int64_t win_lo; int64_t n_keys; int keys_per_split;
   float* part;                            // [B*groups][n_splits][16][2+128]
-  uint32_t* mcount;                       // [B*groups]
   int16_t kvh[kMaxHeads];                 // group -> kv head
 };
 
@@ -73,7 +68,6 @@ struct DecSmem {
   int etok[kRound];        // list mode: resolved tokens and head masks of this round
   uint32_t emask[kRound];
   float lsum[16], mmax[16];
-  int is_last;
   int wsc[kDecThreads / 32];
   int loffs[1];  // list mode: n_chunks + 1 entries (dynamic tail)
 };
@@ -343,7 +337,7 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
     wo[warp][g + 8][col + 1] = oacc[d][3];
   }
   __syncthreads();
-  float* part = p.part + ((int64_t)gg * p.n_splits + split) * 16 * (2 + kD);
+  float* part = p.part + ((int64_t)gg * p.n_splits + split) * 16 * kPartRow;
   for (int x = tid; x < 16 * kD; x += kDecThreads) {
     const int r = x / kD, d = x % kD;
     float M = -INFINITY;
@@ -356,81 +350,72 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
         l += f * sm.wl[w][r];
       }
     }
-    part[r * (2 + kD) + 2 + d] = o;
+    part[r * kPartRow + 4 + d] = o;
     if (d == 0) {
-      part[r * (2 + kD)] = M;
-      part[r * (2 + kD) + 1] = l;
+      part[r * kPartRow] = M;
+      part[r * kPartRow + 1] = l;
     }
   }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) sm.is_last = (atomicAdd(&p.mcount[gg], 1u) == (uint32_t)p.n_splits - 1);
-  __syncthreads();
-  if (!sm.is_last) return;
-  __threadfence();
+}
 
-  // ---- last CTA of the group: merge splits in a fixed order.  Every global load
-  // below is independent of the others, so they are all issued before use.
-  const float* pg = p.part + (int64_t)gg * p.n_splits * 16 * (2 + kD);
+// Merge of one (batch, kv group, head)'s split partials by one warp: lane i
+// owns dimensions 4i .. 4i + 3 and sums the splits in split order; the mass l is
+// a per-lane sum in split order followed by a fixed butterfly, so the result
+// does not depend on which split finished last.  Launched after the split
+// kernel on the same stream.
+__global__ void __launch_bounds__(32) dec_split_merge_kernel(const DecAttnParams p) {
+  __shared__ float fs[kMaxSplits];
+  const int gg = blockIdx.x, r = blockIdx.y;  // b * groups + group, head of the group
+  const int b = gg / p.groups, grp = gg % p.groups;
+  const int lane = threadIdx.x;
+  const int64_t sstride = 16 * kPartRow;  // floats between consecutive splits
+  const float* pg = p.part + (int64_t)gg * p.n_splits * sstride + (int64_t)r * kPartRow;
   const int ns = min(p.n_splits, kMaxSplits);
-  float* pm = reinterpret_cast<float*>(&sm.k[0][0][0]);  // [ns][16] split maxima
-  float* pl = pm + kMaxSplits * 16;                      // [ns][16] split sums
-  float* fs = pl + kMaxSplits * 16;                      // [ns][16] split weights
-  static_assert(3 * kMaxSplits * 16 * sizeof(float) <= 2 * kTile * kD * 2 * sizeof(uint16_t),
-                "merge scratch must fit in the K/V staging buffers");
-  for (int x = tid; x < ns * G; x += kDecThreads) {
-    const int sp = x / G, r = x % G;
-    pm[sp * 16 + r] = __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD));
-    pl[sp * 16 + r] = __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD) + 1);
+  float M = -INFINITY;
+  for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, __ldcg(pg + sp * sstride));
+  M = warp_max(M);
+  float l = 0.f;
+  for (int sp = lane; sp < ns; sp += 32) {
+    const float ms = __ldcg(pg + sp * sstride), ls = __ldcg(pg + sp * sstride + 1);
+    const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    fs[sp] = f;
+    l += f * ls;
   }
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, pm[sp * 16 + tid]);
-    float l = 0.f;
-    for (int sp = 0; sp < ns; ++sp) {
-      const float ms = pm[sp * 16 + tid];
-      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-      fs[sp * 16 + tid] = f;
-      l += f * pl[sp * 16 + tid];
-    }
-    sm.mmax[tid] = M;
-    sm.lsum[tid] = l;
-  }
-  __syncthreads();
-  {
-    const int d = tid;  // one dimension per thread, every head
-    float acc[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) acc[r] = 0.f;
-    int sp = 0;
-    for (; sp + 4 <= ns; sp += 4) {
-      float v[4][16];
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  __syncwarp();
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* po = pg + 4 + 4 * lane;
+  int sp = 0;
+  for (; sp + 8 <= ns; sp += 8) {  // eight independent 16-byte loads in flight
+    float4 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(po + (sp + u) * sstride));
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-          v[u][r] = r < G ? __ldcg(pg + ((int64_t)(sp + u) * 16 + r) * (2 + kD) + 2 + d) : 0.f;
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] += fs[(sp + u) * 16 + r] * v[u][r];
-    }
-    for (; sp < ns; ++sp)
-#pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r < G) acc[r] += fs[sp * 16 + r] * __ldcg(pg + ((int64_t)sp * 16 + r) * (2 + kD) + 2 + d);
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      if (r >= G) break;
-      const float l = sm.lsum[r];
-      const int h = kvh * G + r;
-      p.o[b * p.o_sb + (int64_t)h * kD + d] = f32_to_bf16_bits(l > 0.f ? acc[r] / l : 0.f);
-      if (d == 0 && p.lse != nullptr)
-        p.lse[b * p.lse_sb + h] = l > 0.f ? (sm.mmax[r] + log2f(l)) * kLn2 : -INFINITY;
+    for (int u = 0; u < 8; ++u) {
+      const float f = fs[sp + u];
+      acc.x += f * v[u].x;
+      acc.y += f * v[u].y;
+      acc.z += f * v[u].z;
+      acc.w += f * v[u].w;
     }
   }
-  if (tid == 0) p.mcount[gg] = 0;
+  for (; sp < ns; ++sp) {
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(po + sp * sstride));
+    const float f = fs[sp];
+    acc.x += f * v.x;
+    acc.y += f * v.y;
+    acc.z += f * v.z;
+    acc.w += f * v.w;
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  const int h = p.kvh[grp] * p.G + r;
+  uint2 w;
+  w.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  w.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(p.o + b * p.o_sb + (int64_t)h * kD + 4 * lane) = w;
+  if (lane == 0 && p.lse != nullptr)
+    p.lse[b * p.lse_sb + h] = l > 0.f ? (M + log2f(l)) * kLn2 : -INFINITY;
 }
 
 template <bool LIST>
@@ -441,8 +426,14 @@ rtp_status launch_dec_attn(const DecAttnParams& prm, int B, cudaStream_t s) {
     return RTP_ERR_CUDA;
   dim3 grid(prm.n_splits, B * prm.groups);
   if (grid.y > 65535) return RTP_ERR_UNSUPPORTED;
-  TraceScope tr(LIST ? "dec_attn_list" : "dec_attn_range", s);
-  dec_attn_kernel<LIST><<<grid, kDecThreads, smem, s>>>(prm);
+  {
+    TraceScope tr(LIST ? "dec_attn_list" : "dec_attn_range", s);
+    dec_attn_kernel<LIST><<<grid, kDecThreads, smem, s>>>(prm);
+  }
+  rtp_status st = check_cuda(cudaGetLastError());
+  if (st != RTP_OK) return st;
+  TraceScope tr(LIST ? "dec_merge_list" : "dec_merge_range", s);
+  dec_split_merge_kernel<<<dim3(B * prm.groups, prm.G), 32, 0, s>>>(prm);
   return check_cuda(cudaGetLastError());
 }
 
@@ -483,11 +474,7 @@ rtp_status decode_range(const rtp_shape* shape, const int16_t* kv_heads, int n_g
   prm.n_keys = n_keys;
   prm.keys_per_split = L.keys_per_split;
   prm.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part);
-  prm.mcount = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.mcount);
   for (int i = 0; i < n_groups; ++i) prm.kvh[i] = kv_heads[i];
-  if (cudaMemsetAsync(prm.mcount, 0, (size_t)shape->B * n_groups * sizeof(uint32_t), s) !=
-      cudaSuccess)
-    return RTP_ERR_CUDA;
   return launch_dec_attn<false>(prm, shape->B, s);
 }
 
@@ -509,7 +496,6 @@ rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, cons
   prm.rowres = lists.rowres;
   prm.n_ret = hm.n_ret;
   prm.part = lists.part;
-  prm.mcount = lists.mcount;
   for (int i = 0; i < hm.n_rkv; ++i) prm.kvh[i] = hm.rkv[i];
   return launch_dec_attn<true>(prm, shape->B, s);
 }

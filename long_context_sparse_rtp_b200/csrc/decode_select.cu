@@ -125,7 +125,6 @@ struct ScoreParams {
   uint32_t* flags;             // [rows]: 1 = a score fell outside the histogram range
   uint32_t* ncand;
   uint32_t* counter;
-  uint32_t* mcount;
   DevStatus* status;
   int N, Lk_pad, n_ret, n_rkv, G, lgG, per_kv, rows, groups;
   int kw;            // k16 slots per key of a group: G, or 1 when k16 is per kv head
@@ -178,10 +177,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
   // the later kernels of this call count into these
   for (int x = blockIdx.x * kSThreads + tid; x < p.rows; x += gridDim.x * kSThreads)
     p.ncand[x] = 0u;
-  for (int x = blockIdx.x * kSThreads + tid; x < p.groups; x += gridDim.x * kSThreads) {
+  for (int x = blockIdx.x * kSThreads + tid; x < p.groups; x += gridDim.x * kSThreads)
     p.counter[x] = 0u;
-    p.mcount[x] = 0u;
-  }
   for (int x = tid; x < G * kDecWin; x += kSThreads) {
     hm[x] = 0u;
     hc[x] = 0u;
@@ -1193,7 +1190,6 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     sp.flags = static_cast<uint32_t*>(at(L.flags));
     sp.ncand = static_cast<uint32_t*>(at(L.ncand));
     sp.counter = static_cast<uint32_t*>(at(L.counter));
-    sp.mcount = static_cast<uint32_t*>(at(L.mcount));
     sp.status = static_cast<DevStatus*>(ws);
     sp.N = N;
     sp.Lk_pad = L.Lk_pad;
@@ -1309,7 +1305,6 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
   dl.scores = static_cast<const float*>(at(L.scores));
   dl.rowres = static_cast<const RowRes*>(at(L.rowres));
   dl.part = static_cast<float*>(at(L.part));
-  dl.mcount = static_cast<uint32_t*>(at(L.mcount));
   dl.Lk_pad = L.Lk_pad;
   dl.n_chunks = nc;
   dl.n_splits = decode_list_splits(groups, nc);

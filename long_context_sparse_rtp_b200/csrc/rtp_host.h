@@ -117,6 +117,7 @@ constexpr int kDecGBins = 2048;        // absolute bins per row: scores in [-256
 constexpr int kDecGLo = -1024;         // absolute bin of global bin 0
 constexpr int kDecCap = 4096;          // candidates a decode row resolves with one sort
 constexpr int kDecMaxSplits = 256;     // split-KV partials per (batch, kv head) in decode
+constexpr int kPartRow = kD + 4;       // a partial row: m, l, two pad floats, o[kD] (16-byte rows)
 
 constexpr int kDecSub = 64;            // sub-bins of a row's crossing bin
 
@@ -128,7 +129,7 @@ SelectWs select_ws_layout();
 
 struct DecodeWs {   // retrieval decode
   size_t scores, hist_m, hist_c, flags, sub_m, sub_c, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
-      part, mcount, total;
+      part, total;
   int n_chunks, n_splits, Lk_pad, rows, groups;
 };
 
@@ -170,8 +171,7 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
   w.list = take(groups * w.Lk_pad * 8);
   w.lcount = take(groups * nc * 4);
   w.loff = take(groups * (nc + 1) * 4);
-  w.part = take(groups * w.n_splits * 16 * (2 + kD) * 4);
-  w.mcount = take(groups * 4);
+  w.part = take(groups * w.n_splits * 16 * kPartRow * 4);
   w.total = off;
   return w;
 }
@@ -183,7 +183,6 @@ struct DecodeLists {
   const float* scores;
   const RowRes* rowres;
   float* part;
-  uint32_t* mcount;
   int Lk_pad, n_chunks, n_splits;
 };
 
@@ -193,7 +192,7 @@ rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, cons
                                  cudaStream_t s);
 
 struct AttnDecodeWs {  // local / dense decode (range mode)
-  size_t part, mcount, total;
+  size_t part, total;
   int n_splits, keys_per_split;
 };
 
@@ -215,9 +214,7 @@ inline AttnDecodeWs range_decode_ws_layout(int64_t n_keys, int groups) {
   // count then also fits every smaller key count
   size_t off = kStatusBytes;
   w.part = off;
-  off = align_up(off + (size_t)groups * want * 16 * (2 + kD) * 4, 256);
-  w.mcount = off;
-  off = align_up(off + (size_t)groups * 4, 256);
+  off = align_up(off + (size_t)groups * want * 16 * kPartRow * 4, 256);
   w.total = off;
   return w;
 }

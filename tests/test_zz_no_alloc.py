@@ -29,7 +29,7 @@ def _args(inp, q_pos0):
 
 def test_rejects_shapes_beyond_the_scratch_array():
     """Host-side check, nothing enqueued: 400 batch entries x 3 local kv heads
-    need at least one 8320-byte partial each, ~10 MB, more than the 8 MiB array."""
+    need at least one 8448-byte partial each, ~10 MB, more than the 8 MiB array."""
     build.build()
     L = rtp.lib()
     shape = rtp.Shape(400, 1, 9000, 32, 4, 128, 8999)

@@ -1094,35 +1094,36 @@ __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectPara
     __syncthreads();
     const int ksub = (rs.mode == 0 && n > 0) ? sm.s_k : -1;
     if (ksub >= 0 && sm.s_nin <= (uint32_t)kWarpCap) {
-      if (tid < 32) {
-        RowSel r2 = rs;
-        r2.above = rs.above + (double)sm.s_acc * rs.scale_b;
-        r2.cnt_above = rs.cnt_above + sm.s_cnt;
-        // the candidates of the crossing sub-bin, compacted by warp ballots
-        int m = 0;
-        for (int i0 = 0; i0 < n; i0 += 32) {
-          const int i = i0 + lane;
-          unsigned long long ck = 0;
-          bool in = false;
-          if (i < n) {
-            ck = p.cand[(int64_t)row * kDecCap + i];
-            in = subbin(key_score((uint32_t)(ck >> kIdxBits)), rs.bstar) == ksub;
-          }
-          const unsigned ball = __ballot_sync(0xffffffffu, in);
-          if (in) sm.wc[m + __popc(ball & ((1u << lane) - 1u))] = ck;
-          m += __popc(ball);
+      RowSel r2 = rs;
+      r2.above = rs.above + (double)sm.s_acc * rs.scale_b;
+      r2.cnt_above = rs.cnt_above + sm.s_cnt;
+      // the candidates of the crossing sub-bin, compacted by the block in order
+      const unsigned long long* src = p.cand + (int64_t)row * kDecCap;
+      int m = 0;
+      for (int i0 = 0; i0 < n; i0 += kThreads) {
+        const int i = i0 + tid;
+        unsigned long long ck = 0;
+        bool in = false;
+        if (i < n) {
+          ck = __ldcg(src + i);
+          in = subbin(key_score((uint32_t)(ck >> kIdxBits)), rs.bstar) == ksub;
         }
-        __syncwarp();
-        sort_desc_warp(sm.wc, m);
-        rr = warp_walk(sm.wc, m, r2);
+        const unsigned ball = __ballot_sync(0xffffffffu, in);
+        if (lane == 0) sm.hc[tid >> 5] = __popc(ball);
+        __syncthreads();
+        int off = m;
+        for (int w2 = 0; w2 < (tid >> 5); ++w2) off += (int)sm.hc[w2];
+        if (in) sm.wc[off + __popc(ball & ((1u << lane) - 1u))] = ck;
+        for (int w2 = 0; w2 < kThreads / 32; ++w2) m += (int)sm.hc[w2];
+        __syncthreads();
       }
+      sort_desc_block(sm.wc, m);
+      if (tid < 32) rr = warp_walk(sm.wc, m, r2);
     } else if (rs.mode == 0 && n > 0 && n <= kWarpCap) {
-      if (tid < 32) {
-        for (int i = lane; i < n; i += 32) sm.wc[i] = p.cand[(int64_t)row * kDecCap + i];
-        __syncwarp();
-        sort_desc_warp(sm.wc, n);
-        rr = warp_walk(sm.wc, n, rs);
-      }
+      for (int i = tid; i < n; i += kThreads) sm.wc[i] = __ldcg(p.cand + (int64_t)row * kDecCap + i);
+      __syncthreads();
+      sort_desc_block(sm.wc, n);
+      if (tid < 32) rr = warp_walk(sm.wc, n, rs);
     } else if (rs.mode == 0 && n > 0) {
       rr = resolve_many(sm, p, row, rs, n);
     } else {

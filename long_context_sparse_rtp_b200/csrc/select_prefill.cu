@@ -10,10 +10,10 @@
 // per tile, fp32 in TMEM) and one epilogue thread per query row reads its row
 // of each tile from TMEM, so all per-row state lives in that thread:
 //
-//   sweep 1  row max m                                    (1 compare / key)
-//   sweep 2  Z = sum exp(s - m) and a 32-bin mass histogram of the scores in
-//            [c0, m], c0 = m - ln(N / (1 - p)) - 1 (keys below c0 can never be
-//            kept: their total mass is < (1-p) Z)           (1 exp / key)
+//   sweep 1  row max m and a lower bound on Z (running max per thread)
+//   sweep 2  Z = sum exp(s - m) in a fixed order and a 32-bin mass histogram of
+//            the scores in [c0, m], c0 = m - ln(N / ((1 - p) Z)) - 1 (keys below
+//            c0 + 1 are never kept: together they weigh < (1 - p) Z)
 //   sweep 3+ radix refinement inside the crossing bin on the composite key
 //            (score key : 32 bits, 2^21-1-index : 21 bits), 5 bits per sweep,
 //            until the crossing bin holds <= 32 keys; those are collected,
@@ -60,7 +60,9 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 // row states: REFINE1 = 32 uniform score sub-bins of the level-0 crossing bin,
 // REFINE = 5 composite-key bits, COLLECT / LIST = gather the crossing range's keys
 enum { ST_IDLE = 0, ST_REFINE1 = 1, ST_REFINE = 2, ST_COLLECT = 3, ST_DONE = 4, ST_LIST = 5 };
-constexpr int kListCap = 1024;   // crossing-bin keys a row may park in its global list
+// Crossing-range keys a row may park in its global list: a level's even and odd
+// entries go to separate 32-bit bin sums, <= 2032 keys x 2^21 < 2^32 each.
+constexpr int kListCap = 4064;
 
 struct SelParams {
   unsigned long long* lists;  // [slots][kBM][kListCap] crossing-bin keys, or null
@@ -95,6 +97,14 @@ struct SelSmem {
       float s[kEpi / 32][kQueue];
       uint32_t jl[kEpi / 32][kQueue];  // key index | owner lane << 21
     } q;
+    struct {                           // parked-list levels: the state the warps read
+      unsigned long long prefix[kBM];
+      int pbits[kBM];
+      int n[kBM];                      // entries of the row's compacted list
+      int need[kBM];
+      float m[kBM];
+      float tk[kBM];
+    } ls;
   } t;
   float mpart[2][kBM];
   double zpart[2][kBM];
@@ -494,16 +504,43 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     };
 
-    // ---- sweep 1: row max
-    float m = -INFINITY;
-    sweep([&](int, float (&v)[kChunk]) { m = fmaxf(m, max16(v)); }, false, false);
-    sm.mpart[g][r] = m;
+    // ---- sweep 1: the row max m, and a lower bound on Z = sum exp(s - m): each
+    // thread keeps a running max mz and zs, a sum over its 16-key chunks of the
+    // larger of two partial masses, exp(chunk max - mz) and the mass of every
+    // fourth key (both at most the chunk's mass)
+    float mz = -INFINITY, zs = 0.f;
+    sweep(
+        [&](int, float (&v)[kChunk]) {
+          const float cm = max16(v);
+          if (cm > mz) {  // rescale to the new running max (rare after the first tiles)
+            zs = mz > -INFINITY ? zs * rel_w(mz, cm) : 0.f;
+            mz = cm;
+          }
+          if (mz > -INFINITY) {
+            const float a = __fadd_rn(__fadd_rn(rel_w(v[0], mz), rel_w(v[4], mz)),
+                                      __fadd_rn(rel_w(v[8], mz), rel_w(v[12], mz)));
+            zs = __fadd_rn(zs, fmaxf(a, rel_w(cm, mz)));
+          }
+        },
+        false, false);
+    sm.mpart[g][r] = mz;
+    sm.zpart[g][r] = (double)zs;
     ebar();
-    m = fmaxf(sm.mpart[0][r], sm.mpart[1][r]);
+    const float m = fmaxf(sm.mpart[0][r], sm.mpart[1][r]);
     float scale = 1.f, margin = 0.f;
     if (valid) {
+      // A key below m - ln(N / ((1 - p) Z)) is never kept: all such keys weigh
+      // less than (1 - p) Z together, so the keys above that point already pass
+      // p Z.  Z is taken from below (the partial masses, and a 1e-3 margin for
+      // the fp32 sums and ex2.approx), which only widens the range; R adds one
+      // more unit.
+      double zl = 0.0;
+      for (int h = 0; h < 2; ++h)
+        if (sm.mpart[h][r] > -INFINITY) zl += sm.zpart[h][r] * exp((double)(sm.mpart[h][r] - m));
+      zl = fmax(zl * (1.0 - 1e-3), 1e-30);
       const double N = (double)(P + 1);
-      const float R = (float)(log(N / (1.0 - (double)p.p)) + 1.0);
+      const double r_loose = log(N / (1.0 - (double)p.p)) + 1.0;  // Z >= 1
+      const float R = (float)fmin(log(N / ((1.0 - (double)p.p) * zl)) + 1.0, r_loose);
       scale = (float)kNB / R;
       margin = 1e-5f * (fabsf(m) + R + 1.f);
     }
@@ -775,50 +812,99 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       ebar();
       if (g == 0 && (state == ST_REFINE || (state == ST_LIST && !lst))) clear_row(sm, r);
-      // rows with a parked list: the remaining digit levels run over the list
-      const unsigned long long* my = lst ? lists + (size_t)r * kListCap : nullptr;
-      for (;;) {
-        const bool need = lst && n_cur > (unsigned long long)kCap && pbits < kKeyBits;
-        if (!bar_or(1, kEpi, need)) break;
-        const int wl = min(kDigit, kKeyBits - pbits);
-        if (need) {
-          for (int e = g; e < nl; e += 2) {
-            const unsigned long long ck = my[e];
-            if (pbits > 0 && (ck >> (kKeyBits - pbits)) != prefix) continue;
-            const int digit = (int)((ck >> (kKeyBits - pbits - wl)) & ((1ull << wl) - 1));
-            const float sc = key_score((uint32_t)(ck >> kIdxBits));
-            sm.wacc[g][(1 << wl) - 1 - digit][r] += fixed_u(__fmul_rn(rel_w(sc, m), tk));
+      // rows with a parked list: the remaining digit levels run over the list, a
+      // warp per row at a time (lanes read consecutive entries).  Each level keeps
+      // the entries of the current prefix in place and in order, and counts the
+      // ones above it; the row's own threads keep the selection state and publish
+      // what the warps read in shared memory
+      if (bar_or(1, kEpi, lst)) {
+        auto& ls = sm.t.ls;
+        const uint32_t lt = (1u << lane) - 1u;
+        if (g == 0) {
+          ls.n[r] = lst ? nl : 0;
+          ls.m[r] = m;
+          ls.tk[r] = tk;
+        }
+        for (;;) {
+          const bool need = lst && n_cur > (unsigned long long)kCap && pbits < kKeyBits;
+          if (g == 0) {
+            ls.need[r] = need ? 1 : 0;
+            ls.prefix[r] = prefix;
+            ls.pbits[r] = pbits;
           }
-        }
-        ebar();
-        if (need && g == 0) flush_row(sm, r);
-        ebar();
-        if (need) {
-          unsigned long long wsel = 0ull;
-          const int bsel = crossing(sm, r, 1 << wl, T, false, fd, base, inner, wsel);
-          if (bsel < 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 19);
-          prefix = (prefix << wl) | (unsigned long long)((1 << wl) - 1 - max(bsel, 0));
-          pbits += wl;
-          n_cur = bound(wsel);
-        }
-        ebar();
-        if (need && g == 0) clear_row(sm, r);
-      }
-      if (g == 0 && lst) sm.ncnt[r] = 0;
-      ebar();
-      if (lst) {  // the final range's keys become the row's candidates
-        int above = 0;
-        for (int e = g; e < nl; e += 2) {
-          const unsigned long long ck = my[e];
-          const unsigned long long px = pbits > 0 ? (ck >> (kKeyBits - pbits)) : 0ull;
-          if (px == prefix) {
-            const int slot_c = atomicAdd(&sm.ncnt[r], 1);
-            if (slot_c < kCap) sm.u.cand[slot_c][r] = ck;
-          } else if (px > prefix) {
-            ++above;
+          if (!bar_or(1, kEpi, need)) break;
+          for (int rr = warp; rr < kBM; rr += kEpi / 32) {
+            if (!ls.need[rr]) continue;
+            const unsigned long long pfx = ls.prefix[rr];
+            const int pb = ls.pbits[rr], wl = min(kDigit, kKeyBits - pb), n = ls.n[rr];
+            const float rm = ls.m[rr], rtk = ls.tk[rr];
+            unsigned long long* const L = lists + (size_t)rr * kListCap;
+            int kept = 0, above = 0;
+            for (int k0 = 0; k0 < n; k0 += 32) {
+              const int k = k0 + lane;
+              const unsigned long long ck = k < n ? __ldcg(L + k) : 0ull;
+              const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
+              const bool in = (k < n) & (px == pfx);
+              above += ((k < n) & (px > pfx)) ? 1 : 0;
+              const uint32_t ball = __ballot_sync(0xffffffffu, in);
+              if (in) {  // position <= k: never an entry still to be read
+                L[kept + __popc(ball & lt)] = ck;
+                const int digit = (int)((ck >> (kKeyBits - pb - wl)) & ((1ull << wl) - 1));
+                // even and odd entries in separate copies: <= 2032 keys x 2^21 each
+                atomicAdd(&sm.wacc[lane & 1][(1 << wl) - 1 - digit][rr],
+                          fixed_u(__fmul_rn(rel_w(key_score((uint32_t)(ck >> kIdxBits)), rm),
+                                            rtk)));
+              }
+              kept += __popc(ball);
+            }
+            above = __reduce_add_sync(0xffffffffu, above);
+            if (lane == 0) {
+              ls.n[rr] = kept;
+              sm.nabove[rr] += above;
+            }
           }
+          ebar();
+          if (need && g == 0) flush_row(sm, r);
+          ebar();
+          if (need) {
+            unsigned long long wsel = 0ull;
+            const int wl = min(kDigit, kKeyBits - pbits);
+            const int bsel = crossing(sm, r, 1 << wl, T, false, fd, base, inner, wsel);
+            if (bsel < 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 19);
+            prefix = (prefix << wl) | (unsigned long long)((1 << wl) - 1 - max(bsel, 0));
+            pbits += wl;
+            n_cur = bound(wsel);
+          }
+          ebar();
+          if (need && g == 0) clear_row(sm, r);
         }
-        atomicAdd(&sm.nabove[r], above);
+        // the final range's keys become the row's candidates
+        if (g == 0) {
+          ls.need[r] = lst ? 1 : 0;
+          ls.prefix[r] = prefix;
+          ls.pbits[r] = pbits;
+          sm.ncnt[r] = 0;
+        }
+        ebar();
+        for (int rr = warp; rr < kBM; rr += kEpi / 32) {
+          if (!ls.need[rr]) continue;
+          const unsigned long long pfx = ls.prefix[rr];
+          const int pb = ls.pbits[rr], n = ls.n[rr];
+          const unsigned long long* const L = lists + (size_t)rr * kListCap;
+          int above = 0;
+          for (int k = lane; k < n; k += 32) {
+            const unsigned long long ck = __ldcg(L + k);
+            const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
+            if (px == pfx) {
+              const int slot_c = atomicAdd(&sm.ncnt[rr], 1);
+              if (slot_c < kCap) sm.u.cand[slot_c][rr] = ck;
+            } else if (px > pfx) {
+              ++above;
+            }
+          }
+          above = __reduce_add_sync(0xffffffffu, above);
+          if (lane == 0) sm.nabove[rr] += above;
+        }
       }
       ebar();
       if (lst) {

@@ -78,6 +78,7 @@ __device__ __forceinline__ uint32_t dswz(const uint16_t (*base)[kD], int r, int 
 
 template <bool LIST>
 __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnParams p) {
+  griddep_wait();  // launched as a dependent of the previous kernel
   extern __shared__ __align__(128) unsigned char smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>(smem_raw);
   const int split = blockIdx.x;
@@ -364,6 +365,7 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
 // does not depend on which split finished last.  Launched after the split
 // kernel on the same stream.
 __global__ void __launch_bounds__(32) dec_split_merge_kernel(const DecAttnParams p) {
+  griddep_wait();  // launched as a dependent of the previous kernel
   __shared__ float fs[kMaxSplits];
   const int gg = blockIdx.x, r = blockIdx.y;  // b * groups + group, head of the group
   const int b = gg / p.groups, grp = gg % p.groups;
@@ -426,15 +428,16 @@ rtp_status launch_dec_attn(const DecAttnParams& prm, int B, cudaStream_t s) {
     return RTP_ERR_CUDA;
   dim3 grid(prm.n_splits, B * prm.groups);
   if (grid.y > 65535) return RTP_ERR_UNSUPPORTED;
+  rtp_status st;
   {
     TraceScope tr(LIST ? "dec_attn_list" : "dec_attn_range", s);
-    dec_attn_kernel<LIST><<<grid, kDecThreads, smem, s>>>(prm);
+    if ((st = check_cuda(launch_dependent(dec_attn_kernel<LIST>, grid, dim3(kDecThreads), smem, s,
+                                          prm))) != RTP_OK)
+      return st;
   }
-  rtp_status st = check_cuda(cudaGetLastError());
-  if (st != RTP_OK) return st;
   TraceScope tr(LIST ? "dec_merge_list" : "dec_merge_range", s);
-  dec_split_merge_kernel<<<dim3(B * prm.groups, prm.G), 32, 0, s>>>(prm);
-  return check_cuda(cudaGetLastError());
+  return check_cuda(launch_dependent(dec_split_merge_kernel, dim3(B * prm.groups, prm.G), dim3(32),
+                                     0, s, prm));
 }
 
 void fill_dec_common(DecAttnParams& prm, const rtp_shape* shape, const rtp_view& q,

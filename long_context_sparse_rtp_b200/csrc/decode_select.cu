@@ -443,6 +443,7 @@ struct MergeParams {
 constexpr int kBinsPerThread = kDecGBins / kThreads;  // 8
 
 __global__ void __launch_bounds__(kThreads) dec_merge_kernel(const MergeParams p) {
+  griddep_wait();  // launched as a dependent of the previous kernel
   __shared__ double wsum[kThreads / 32];
   __shared__ uint32_t wcnt[kThreads / 32];
   __shared__ int s_top;
@@ -968,6 +969,7 @@ __device__ RowRes resolve_many(ResolveSmem& sm, const CollectParams& p, int row,
 
 
 __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectParams p) {
+  griddep_wait();  // launched as a dependent of the previous kernel
   extern __shared__ __align__(16) unsigned char smem_raw[];
   CollectSmem& sm = *reinterpret_cast<CollectSmem*>(smem_raw);
   const int chunk = blockIdx.x, grp = blockIdx.y;
@@ -1039,6 +1041,7 @@ __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectPara
 
 // One CTA per retrieval row: the exact cut inside the crossing bin.
 __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectParams p) {
+  griddep_wait();  // launched as a dependent of the previous kernel
   extern __shared__ __align__(16) unsigned char smem_raw[];
   ResolveSmem& sm = *reinterpret_cast<ResolveSmem*>(smem_raw);
   const int row = blockIdx.x;
@@ -1254,8 +1257,9 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     mp.rowsel = static_cast<RowSel*>(at(L.rowsel));
     mp.p = p;
     TraceScope tr("dec_merge", s);
-    dec_merge_kernel<<<L.rows, kThreads, 0, s>>>(mp);
-    if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+    if ((st = check_cuda(launch_dependent(dec_merge_kernel, dim3(L.rows), dim3(kThreads), 0, s,
+                                          mp))) != RTP_OK)
+      return st;
   }
   {  // 3. collect, compact, exact cut
     CollectParams cp;
@@ -1288,16 +1292,18 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
       return RTP_ERR_CUDA;
     {
       TraceScope tr("dec_collect", s);
-      dec_collect_kernel<<<dim3(nc, groups), kThreads, smem, s>>>(cp);
-      if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+      if ((st = check_cuda(launch_dependent(dec_collect_kernel, dim3(nc, groups), dim3(kThreads),
+                                            smem, s, cp))) != RTP_OK)
+        return st;
     }
     const size_t rsmem = sizeof(ResolveSmem);
     if (cudaFuncSetAttribute(dec_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)rsmem) != cudaSuccess)
       return RTP_ERR_CUDA;
     TraceScope tr("dec_resolve", s);
-    dec_resolve_kernel<<<L.rows, kThreads, rsmem, s>>>(cp);
-    if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+    if ((st = check_cuda(launch_dependent(dec_resolve_kernel, dim3(L.rows), dim3(kThreads), rsmem,
+                                          s, cp))) != RTP_OK)
+      return st;
   }
   // 4. attention over the kept union
   DecodeLists dl;

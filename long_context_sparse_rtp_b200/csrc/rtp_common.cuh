@@ -147,6 +147,10 @@ __device__ __forceinline__ uint32_t score_key(float s) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
+// A kernel launched with launch_dependent: wait until the previous kernel on the
+// stream has completed and its writes are visible (no-op for a plain launch).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(DevStatus* st, int code, int where) {
   if (st != nullptr) {
     atomicCAS(&st->code, 0, code);

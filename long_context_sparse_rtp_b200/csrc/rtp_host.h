@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <utility>
+
 #include "rtp.h"
 #include "rtp_common.cuh"
 
@@ -31,6 +33,26 @@ inline rtp_status check_cuda(cudaError_t e) {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Launch with programmatic stream serialization: the kernel's CTAs may be
+// scheduled while the previous kernel on the stream drains; the kernel itself
+// waits (griddep_wait) before it touches anything that kernel wrote.  Inside a
+// CUDA graph the edge becomes a programmatic dependency.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // A [B][L][heads][width] bf16 view: non-null, rows 16-byte aligned.
 inline rtp_status check_view(const rtp_view& v, int heads, int width, bool needed) {

@@ -99,7 +99,7 @@ __device__ __forceinline__ float key_score(uint32_t key) {
 // tcgen05.mma per slot (M = 128, N = 16, K = 16), accumulating
 // D[key][head] = q16_head . k16_(key, head's slot) in TMEM: the zero blocks add
 // exact zeros, so each score is the 16-term dot product of a single MMA, as in
-// the prefill selection.  The 8 consumer warps read D, then per item: the heads'
+// the prefill selection.  Consumer warps 0-7 read D, then all 12 per item: the heads'
 // max bins, the scores' store, a 256-bin window histogram per head in shared
 // memory and its flush into the row's absolute histogram.  Producer and MMA run
 // ahead across items, bounded by the ring and by 8 TMEM accumulators.
@@ -109,7 +109,7 @@ constexpr int kSN = 16;                       // MMA N: a group's heads, zero-pa
 constexpr int kSChunkA = kSTile * kR * 2;     // 4096 B: one slot of a sub-tile
 constexpr int kSChunkB = kSN * kR * 2;        // 512 B: one query block
 constexpr int kSBufs = 8;                     // TMEM accumulators, kSN columns each
-constexpr int kSConsumers = 256;              // 8 warps
+constexpr int kSConsumers = 384;              // 12 warps; warps 0-7 also read TMEM
 constexpr int kSProdWarp = kSConsumers / 32, kSMmaWarp = kSProdWarp + 1;
 constexpr int kSThreads = kSConsumers + 64;   // + the producer and MMA warps
 constexpr int kSRingBytes = 74 * 1024;
@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(kSThreads, 2)
     return;
   }
 
-  // ---------------- consumers (threads 0..255; named barrier 1)
-  const int hh = tid & (G - 1);  // G divides 256: constant per thread
+  // ---------------- consumers (threads 0..kSConsumers-1; named barrier 1)
+  const int hh = tid & (G - 1);  // G divides kSConsumers: constant per thread
   uint32_t sub_base = 0;         // sub-tiles of the earlier items (the MMA's sequence)
   bool ok = true;
   for (int item = it0; item < it1; ++item) {
@@ -336,7 +336,7 @@ __global__ void __launch_bounds__(kSThreads, 2)
     // and 3, each its TMEM lane quarter (one key per lane, the heads in columns);
     // keys past N read as -inf
 #pragma unroll 1
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < (warp < 8 ? 2 : 0); ++u) {
       const int st = (warp >> 2) * 2 + u;
       const int x = st * kSTile + (warp & 3) * 32 + lane;
       float d[kSN];

@@ -7,19 +7,20 @@
 // b = floor(4 s) and contributes exp(s - (b+1)/4) in (0.78, 1] to that bin, as
 // 21-bit fixed point.  Integer sums are exact and order-free, so every decision
 // below is deterministic.  Per kv group of G retrieval query heads:
-//   1. score     stream the k16 cache once (HBM-bound), s = q16 . k16 in fp32
-//                with a fixed FMA order, scores kept in the workspace; each CTA
-//                bins its 1024 x G scores in shared memory (one 256-bin window per
-//                head, 32-bit atomics) and adds the occupied bins into the row's
-//                2048-bin absolute histogram in global memory;
+//   1. score     stream the k16 cache once (HBM-bound), s = q16 . k16 as one
+//                16-term tensor-core dot product (tcgen05, fp32 in TMEM), scores
+//                kept in the workspace; each CTA bins its items' scores in shared
+//                memory (one 256-bin window per head, 32-bit atomics) and adds
+//                the occupied bins into the row's 2048-bin absolute histogram;
 //   2. merge     per row: bin masses scaled to the top occupied bin in fp64, Z,
-//                T = p Z, and the crossing bin, by fixed-order block scans;
+//                T = p Z, the crossing bin and its 64-way sub-bin split;
 //   3. collect   per chunk: keys above the crossing bin are kept, keys in it are
 //                candidates (collected per row); one ordered list per kv group of
-//                every token some head may keep.  The last CTA of a group sorts
-//                each row's candidates by (score desc, index asc), one warp per
-//                row, and walks them to the exact cut (t, jtie);
-//   4. attend    gathered split-KV attention over the lists (decode.cu); the
+//                every token some head may keep;
+//   4. resolve   per row: the crossing sub-bin's candidates, compacted and sorted
+//                by (score desc, index asc) by the row's CTA, walked to the exact
+//                cut (t, jtie);
+//   5. attend    gathered split-KV attention over the lists (decode.cu); the
 //                candidate heads are settled there with s > t or (s == t, j <= jtie).
 // Rows with scores outside [-256, 256) or more than 4096 keys in the crossing bin
 // are resolved by a radix refinement over the stored scores (slower, rare).

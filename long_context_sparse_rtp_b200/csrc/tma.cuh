@@ -111,13 +111,6 @@ __device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// Byte offset of `lin` inside a 1024-byte-aligned region written by TMA with
-// 128-byte swizzling: the 16-byte chunk index (bits 4..6) is XORed with the
-// 128-byte row index within each 1024-byte block (bits 7..9).
-__device__ __forceinline__ uint32_t swizzle128(uint32_t lin) {
-  return lin ^ (((lin >> 7) & 7u) << 4);
-}
-
 // Named barrier for a subset of the CTA's warps.
 __device__ __forceinline__ void named_bar(int id, int threads) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");

@@ -11,13 +11,14 @@
 //          selection used (128 query rows x 128 keys, K = 16), so the kept set
 //          is reproduced bit for bit.
 //
-// One CTA = 128 query rows of one head, 128-key tiles.  Warp 4 loads Q once and
-// K/V (and K16) tiles into a 2-stage ring with TMA (128-byte swizzle); warp 5
+// One CTA = 128 query rows of one head, 128-key tiles.  Warp 8 loads Q once and
+// K/V (and K16) tiles into a 2-stage ring with TMA (128-byte swizzle); warp 9
 // issues S = Q K^T (8 MMAs, K = 16 each) into one of two TMEM score buffers and
-// O += P V into a TMEM accumulator; warps 0-3 hold one query row per thread:
-// read the scores with tcgen05.ld, mask, online softmax in the log2 domain,
-// write P (bf16, two per column) over the scores in TMEM, where the PV MMA
-// reads it as its A operand.  The running max is only
+// O += P V into a TMEM accumulator; warps 0-7 hold two threads per query row
+// (64 keys and 64 output dimensions each): read the scores with tcgen05.ld,
+// mask, share the tile max with the partner thread, online softmax in the log2
+// domain, write P (bf16, two per column) over the scores in TMEM, where the PV
+// MMA reads it as its A operand.  The running max is only
 // moved (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles
 // need no rescale.  P is rounded to bf16 once and the normaliser sums the
 // rounded values, so the output is an exact convex combination of them.
@@ -35,7 +36,9 @@ constexpr int kBN = 128;                  // keys per tile
 constexpr int kStages = 2;                // K/V ring
 constexpr int kHalf = 128 * 128;          // one 64-column half of a 128 x 128 bf16 tile: 16 KB
 constexpr int kTile = 2 * kHalf;          // 32 KB
-constexpr int kThreads = 192;
+constexpr int kSoftmax = 256;            // softmax threads: two per query row
+constexpr int kProdWarp = kSoftmax / 32, kMmaWarp = kProdWarp + 1;
+constexpr int kThreads = kSoftmax + 64;
 constexpr float kRescale = 8.f;           // move the max when it grows by > 2^8
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kBM, kBN);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(kBM, kD) | (1u << 16);  // V is MN-major
@@ -68,6 +71,8 @@ struct TcSmem {                      // placed on a 1024-byte boundary
   // a warp may run one tile ahead of another, never two
   uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[2], s_empty[2], s16_empty[2],
       p_full[2], o_done[2];
+  float tmax[2][2][kBM];             // [tile parity][column half][row]: partial tile maxima
+  float lpart[2][kBM];               // [column half][row]: partial row sums
   uint32_t tmem_base;
   int gave_up;
 };
@@ -159,13 +164,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_empty[i], 1);  // committed once the PV MMA reading P from it is done
       mbar_init(&sm.o_done[i], 1);   // PV MMAs of tiles with this parity
-      mbar_init(&sm.s16_empty[i], 4);
-      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.s16_empty[i], kSoftmax / 32);
+      mbar_init(&sm.p_full[i], kSoftmax / 32);
     }
     sm.gave_up = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -176,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t t_s = tmem, t_o = tmem + 256, t_s16 = tmem + 384;
   volatile int* gave_up = &sm.gave_up;
 
-  if (warp == 4) {  // ------------------------------------------------ TMA producer
+  if (warp == kProdWarp) {  // ---------------------------------------- TMA producer
     if (lane == 0) {
       bool ok = true;
       const uint32_t qbytes = kTile + (sparse ? kBM * kR * 2 : 0);
@@ -208,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(&sm.q_full, 0u);
     }
     __syncwarp();
-  } else if (warp == 5) {  // ------------------------------------------ MMA issuer
+  } else if (warp == kMmaWarp) {  // ---------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(&sm.q_full, 0u, gave_up);
       uint32_t n_pv = 0;
@@ -254,11 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (n_pv > 0) mbar_wait_drain(&sm.o_done[(n_pv - 1) & 1u], ((n_pv - 1) >> 1) & 1u);
     }
     __syncwarp();
-  } else {  // ------------------------------------- softmax: thread = query row
-    const int r = tid;
+  } else {  // ------------------------------- softmax: two threads per query row
+    // thread (r, g): TMEM lane r, key columns 64 g .. 64 g + 63 of each tile, output
+    // dimensions 64 g .. 64 g + 63.  Warps w and w + 4 hold the same rows and
+    // exchange their tile maxima through shared memory (pair barrier 1 + w % 4).
+    const int r = tid & (kBM - 1), g = tid >> 7;
     const bool valid = r < nrows;
     const int64_t P = P0 + r;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const int pair_bar = 1 + (warp & 3);
     float thr = INFINITY;
     int64_t jt = -1;
     if (sparse && valid) {
@@ -270,33 +279,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int it = 0; it < sch.n; ++it) {
       const int sb = it & 1;
-      const int64_t j0 = (int64_t)sch.tile(it) * kBN;
+      const int64_t j0 = (int64_t)sch.tile(it) * kBN + g * 64;  // this thread's first key
       ok = ok && mbar_wait_warp(&sm.s_full[sb], (uint32_t)(it >> 1) & 1u, gave_up);
       tc_fence_after();
-      bool full = false;
-      if (MODE == MODE_DENSE) full = j0 + kBN - 1 <= P;
-      if (MODE == MODE_LOCAL)
-        full = j0 + kBN - 1 <= P && (j0 > P - p.window || j0 + kBN - 1 < p.n_sink);
-      // the tile's scores, masked and scaled into the log2 domain
-      float x[kBN];
+      const uint32_t col = (uint32_t)(sb * kBN + g * 64);
+      // the thread's 64 scores, masked and scaled into the log2 domain
+      float x[64];
       if (sparse) {
         // the indexer predicate: s16 > t, or s16 == t and j <= jtie; causal j <= P.
         // One compare per key against te = t, or the float below t where the tie
-        // index lies past the tile (every tie kept); the tile holding a lane's tie
-        // index and the diagonal tile take one more select per key
-        auto clamp_off = [](int64_t d) {
-          return (int)(d < -1 ? -1 : (d > kBN - 1 ? kBN - 1 : d));
-        };
+        // index lies past these keys (every tie kept); keys holding a lane's tie
+        // index or the diagonal take one more select each
+        auto clamp_off = [](int64_t d) { return (int)(d < -1 ? -1 : (d > 63 ? 63 : d)); };
         const int ptl = clamp_off(P - j0), jtl = clamp_off(jt - j0);
-        const float te = !ok ? INFINITY : (jtl == kBN - 1 ? float_below(thr) : thr);
-        const bool mixed = __any_sync(0xffffffffu, (jtl >= 0) & (jtl < kBN - 1));
-        const bool diag = __any_sync(0xffffffffu, ptl < kBN - 1);
+        const float te = !ok ? INFINITY : (jtl == 63 ? float_below(thr) : thr);
+        const bool mixed = __any_sync(0xffffffffu, (jtl >= 0) & (jtl < 63));
+        const bool diag = __any_sync(0xffffffffu, ptl < 63);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t r16[32], rs[32];
           if (ok) {
-            tmem_ld32_nowait(t_s16 + lane_off + (uint32_t)(c * 32), r16);
-            tmem_ld32_nowait(t_s + lane_off + (uint32_t)(sb * kBN + c * 32), rs);
+            tmem_ld32_nowait(t_s16 + lane_off + (uint32_t)(g * 64 + c * 32), r16);
+            tmem_ld32_nowait(t_s + lane_off + col + (uint32_t)(c * 32), rs);
             tmem_wait_ld();
           }
 #pragma unroll
@@ -316,19 +320,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (diag) {
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) x[i] = i <= ptl ? x[i] : -INFINITY;
+          for (int i = 0; i < 64; ++i) x[i] = i <= ptl ? x[i] : -INFINITY;
         }
         tc_fence_before();  // S16 is in registers: the MMA may reuse its buffer
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s16_empty[it & 1]);
       } else {
-        if (ok) tmem_ld128(t_s + lane_off + (uint32_t)(sb * kBN), x);
+        if (ok) {
+          float a[32], c2[32];
+          tmem_ld32(t_s + lane_off + col, a);
+          tmem_ld32(t_s + lane_off + col + 32u, c2);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            x[i] = a[i];
+            x[32 + i] = c2[i];
+          }
+        }
+        bool full = false;
+        if (MODE == MODE_DENSE) full = j0 + 63 <= P;
+        if (MODE == MODE_LOCAL) full = j0 + 63 <= P && (j0 > P - p.window || j0 + 63 < p.n_sink);
         if (full && ok) {
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) x[i] *= p.scale_log2;
+          for (int i = 0; i < 64; ++i) x[i] *= p.scale_log2;
         } else {
 #pragma unroll
-          for (int i = 0; i < kBN; ++i) {
+          for (int i = 0; i < 64; ++i) {
             const int64_t j = j0 + i;
             bool kp;
             if (MODE == MODE_DENSE) kp = j <= P;
@@ -337,13 +353,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      float tm[8];  // tile max as a tree (independent chains)
+      float tm[8];  // the thread's max as a tree (independent chains)
 #pragma unroll
       for (int e = 0; e < 8; ++e) tm[e] = x[e];
 #pragma unroll
-      for (int i = 8; i < kBN; ++i) tm[i & 7] = fmaxf(tm[i & 7], x[i]);
-      const float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
-                               fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
+      for (int i = 8; i < 64; ++i) tm[i & 7] = fmaxf(tm[i & 7], x[i]);
+      float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
+                         fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
+      // the row's tile max from the partner thread (parity-paired slots)
+      sm.tmax[it & 1][g][r] = tmax;
+      named_bar(pair_bar, 64);
+      tmax = fmaxf(tmax, sm.tmax[it & 1][g ^ 1][r]);
       const float m_new = fmaxf(m_used, tmax);
       const bool first = m_used == -INFINITY && m_new > -INFINITY;  // O and l are still 0
       const bool move = m_used > -INFINITY && m_new > m_used + kRescale;
@@ -354,35 +374,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_used = m_new;
         l *= alpha;
       }
-      // O is rescaled (rarely) once the previous tile's PV MMA is done
+      // O is rescaled (rarely) once the previous tile's PV MMA is done: this
+      // thread's 64 dimensions
       if (it > 0 && __any_sync(0xffffffffu, move)) {
         ok = ok && mbar_wait_warp(&sm.o_done[(it - 1) & 1], (uint32_t)((it - 1) >> 1) & 1u,
                                   gave_up);
         tc_fence_after();
         if (ok) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < 2; ++c) {
             float o[32];
-            tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
+            tmem_ld32(t_o + lane_off + (uint32_t)(g * 64 + c * 32), o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(t_o + lane_off + (uint32_t)(c * 32), o);
+            tmem_st32(t_o + lane_off + (uint32_t)(g * 64 + c * 32), o);
           }
         }
       }
-      // P = 2^(x - m) rounded to bf16 once, packed two per column over the scores
+      // P = 2^(x - m) rounded to bf16 once, packed two per column over the scores:
+      // keys 64 g + 2e, 64 g + 2e + 1 go to column 32 g + e of the tile's buffer
       const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
       float lsum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      {
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int i = h2 * 64 + 2 * e;
-          pk[e] = pack_bf16x2(ex2_ftz(x[i] - msafe), ex2_ftz(x[i + 1] - msafe));
+          pk[e] = pack_bf16x2(ex2_ftz(x[2 * e] - msafe), ex2_ftz(x[2 * e + 1] - msafe));
           lsum[e & 3] += bf16_lo(pk[e]) + bf16_hi(pk[e]);
         }
-        if (ok) tmem_st32u(t_s + lane_off + (uint32_t)(sb * kBN + h2 * 32), pk);
+        if (ok) tmem_st32u(t_s + lane_off + (uint32_t)(sb * kBN + g * 32), pk);
       }
       tmem_wait_st();
       l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
@@ -390,18 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[it & 1]);
     }
-    // ---- epilogue: O / l from TMEM, bf16 rows to global
+    // ---- epilogue: O / l from TMEM, bf16 rows to global (64 dimensions each)
+    sm.lpart[g][r] = l;
+    named_bar(pair_bar, 64);
+    const float lrow = l + sm.lpart[g ^ 1][r];
     if (sch.n > 0)
       ok = ok && mbar_wait_warp(&sm.o_done[(sch.n - 1) & 1], (uint32_t)((sch.n - 1) >> 1) & 1u,
                                 gave_up);
     tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint16_t* orow = p.o + b * p.o_sb + (int64_t)(m0 + r) * p.o_sl + (int64_t)h * kD;
+    const float inv = lrow > 0.f ? 1.f / lrow : 0.f;
+    uint16_t* orow = p.o + b * p.o_sb + (int64_t)(m0 + r) * p.o_sl + (int64_t)h * kD + g * 64;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < 2; ++c) {
       float o[32];
       if (sch.n > 0) {
-        tmem_ld32(t_o + lane_off + (uint32_t)(c * 32), o);
+        tmem_ld32(t_o + lane_off + (uint32_t)(g * 64 + c * 32), o);
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
@@ -418,14 +441,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    if (valid && p.lse != nullptr)
+    if (g == 0 && valid && p.lse != nullptr)
       p.lse[((int64_t)b * p.H + h) * p.Lq + m0 + r] =
-          l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
-    if (!ok && r == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 43);
+          lrow > 0.f ? (m_used + log2f(lrow)) * kLn2 : -INFINITY;
+    if (!ok && r == 0 && g == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 43);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -216,3 +216,19 @@ def test_decode_graph_matches_eager():
     g.step(hq, k[:, 4999:].cpu().pin_memory(), v[:, 4999:].cpu().pin_memory(), ho)
     torch.cuda.synchronize()
     assert torch.equal(ho, eager["o"].cpu())
+
+
+def test_decode_all_scores_equal_beyond_candidate_cap():
+    """W_q16 = 0 with a 9000-token cache: every key ties, so the crossing bin
+    holds more keys than one sort resolves (4096) and the row takes the radix
+    refinement over the stored scores; the cut is the ceil(p * N)-th index."""
+    w = W["decode_128k_b8"]
+    L = 9000
+    inp = synth.make_inputs(w, "cuda", L=L, B=2)
+    inp["Wq16"] = torch.zeros_like(inp["Wq16"])
+    for p in (0.5, 0.95):
+        _, _, o, lse, sel, _ = gpu_decode(inp, w, p)
+        n = int(np.maximum(1, np.ceil(float(np.float32(p)) * L)))
+        assert np.all(sel["count"].cpu().numpy() == n)
+        assert np.all(sel["jtie"].cpu().numpy() == n - 1)
+        assert np.all(sel["thr"].cpu().numpy() == 0.0)

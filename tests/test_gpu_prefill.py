@@ -189,3 +189,26 @@ def test_prefill_all_scores_equal():
         assert np.array_equal(cnt[0, 0], expect)
         assert np.array_equal(jt[0, 0], expect - 1)
         assert np.all(res["sel"]["thr"].cpu().numpy() == 0.0)
+
+
+def test_prefill_all_scores_equal_deep():
+    """W_q16 = 0 at 10K rows: every key ties, so rows past 4064 keys take the
+    level-1 sub-bins (one sub-bin holds every key), the composite-key digits
+    through the identical score bits, and the index bits; the kept set is still
+    the ceil(p * N) lowest indices."""
+    w = W["prefill_2k"]
+    L = 10000
+    inp = synth.make_inputs(w, "cuda", L=L)
+    Wq = torch.zeros_like(inp["Wq16"])
+    N = np.arange(1, L + 1)
+    for p in (0.37, 0.95):
+        res = rtp_layer_prefill(inp["q"], inp["k"], inp["v"], Wq, inp["Wk16"], inp["kv_role"],
+                                p=p, window=w.window, n_sink=w.n_sink)
+        torch.cuda.synchronize()
+        cnt = res["sel"]["count"].cpu().numpy()
+        jt = res["sel"]["jtie"].cpu().numpy()
+        expect = np.maximum(1, np.ceil(float(np.float32(p)) * N)).astype(int)
+        for s in range(cnt.shape[1]):
+            assert np.array_equal(cnt[0, s], expect), s
+            assert np.array_equal(jt[0, s], expect - 1), s
+        assert np.all(res["sel"]["thr"].cpu().numpy() == 0.0)

@@ -45,7 +45,7 @@ constexpr int kTileBytes = kBN * kR * 2;
 constexpr int kNB = 32;          // histogram bins (5-bit digits)
 constexpr int kDigit = 5;
 constexpr int kCap = 32;         // candidates collected per row
-constexpr int kGroup = 16;       // tiles per 32-bit bin-sum group: 16 x 64 keys x 2^21 < 2^32
+constexpr int kGroup = 16;       // tiles per 32-bit bin-sum group: 16 x 64 keys x (2^21 + 1) < 2^32
 constexpr int kMaxIter = 16;     // refine / collect sweeps (53 key bits / 5 + 1 suffice)
 constexpr int kQueue = 64;       // per-warp queue of refine hits (drained at 32)
 constexpr int kChunk = 16;       // keys per TMEM load and per unrolled body
@@ -61,7 +61,7 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 // REFINE = 5 composite-key bits, COLLECT / LIST = gather the crossing range's keys
 enum { ST_IDLE = 0, ST_REFINE1 = 1, ST_REFINE = 2, ST_COLLECT = 3, ST_DONE = 4, ST_LIST = 5 };
 // Crossing-range keys a row may park in its global list: a level's even and odd
-// entries go to separate 32-bit bin sums, <= 2032 keys x 2^21 < 2^32 each.
+// entries go to separate 32-bit bin sums, <= 2032 keys x (2^21 + 1) < 2^32 each.
 constexpr int kListCap = 4064;
 
 struct SelParams {
@@ -126,10 +126,11 @@ __device__ __forceinline__ float ex2_ftz(float x) {
 __device__ __forceinline__ float rel_w(float s, float m) {
   return ex2_ftz(__fmul_rn(__fsub_rn(s, m), kLog2e));
 }
-// trunc(x) for x in [0, 2^21] (clamped): adding 2^23 with rounding toward zero
-// leaves the integer part in the low mantissa bits.
+// trunc(x) for x in [0, 2^23): adding 2^23 with rounding toward zero leaves the
+// integer part in the low mantissa bits.  Every use passes 2^21 exp(s - e) with
+// s at most its bin's edge e up to rounding, so a key adds at most 2^21 + 1.
 __device__ __forceinline__ uint32_t fixed_u(float x) {
-  return __float_as_uint(__fadd_rz(fminf(x, 2097152.0f), 8388608.0f)) - 0x4B000000u;
+  return __float_as_uint(__fadd_rz(x, 8388608.0f)) - 0x4B000000u;
 }
 // Level-0 bin of a score s <= m: floor((m - s) * scale), or kNB for a score at
 // or below c0 = m - kNB / scale (adding 1.5 * 2^23 with rounding toward -inf
@@ -560,8 +561,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           int bb[kChunk];
 #pragma unroll
           for (int i = 0; i < kChunk; ++i) {
-            e[i] = rel_w(v[i], m);
-            bb[i] = bin0_of(v[i], m, scale);  // kNB: below c0, a bin never read
+            // rel_w and bin0_of from one difference: exp2(-(m - s) log2 e) is
+            // exp2((s - m) log2 e) bit for bit
+            const float dm = __fsub_rn(m, v[i]);
+            e[i] = ex2_ftz(-__fmul_rn(dm, kLog2e));
+            bb[i] = min(__float_as_int(__fadd_rd(__fmul_rn(dm, scale), 12582912.0f)) - 0x4B400000,
+                        kNB);  // kNB: below c0, a bin never read
           }
           float t[kChunk];  // every edge factor is read before the first store
 #pragma unroll
@@ -850,7 +855,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               if (in) {  // position <= k: never an entry still to be read
                 L[kept + __popc(ball & lt)] = ck;
                 const int digit = (int)((ck >> (kKeyBits - pb - wl)) & ((1ull << wl) - 1));
-                // even and odd entries in separate copies: <= 2032 keys x 2^21 each
+                // even and odd entries in separate copies: <= 2032 keys each
                 atomicAdd(&sm.wacc[lane & 1][(1 << wl) - 1 - digit][rr],
                           fixed_u(__fmul_rn(rel_w(key_score((uint32_t)(ck >> kIdxBits)), rm),
                                             rtk)));

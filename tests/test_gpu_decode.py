@@ -212,10 +212,18 @@ def test_decode_graph_matches_eager():
         assert torch.equal(g.o, eager["o"])
         assert torch.equal(g.lse, eager["lse"])
     hq = q.cpu().pin_memory()
+    hk = k[:, 4999:].cpu().pin_memory()
+    hv = v[:, 4999:].cpu().pin_memory()
     ho = torch.empty_like(hq).pin_memory()
-    g.step(hq, k[:, 4999:].cpu().pin_memory(), v[:, 4999:].cpu().pin_memory(), ho)
+    for _ in range(2):  # captures the copies with the step, then replays that graph
+        ho.zero_()
+        g.step(hq, hk, hv, ho)
+        torch.cuda.synchronize()
+        assert torch.equal(ho, eager["o"].cpu())
+    ho2 = torch.empty_like(hq).pin_memory()  # other buffers: copies around the graph
+    g.step(hq, hk, hv, ho2)
     torch.cuda.synchronize()
-    assert torch.equal(ho, eager["o"].cpu())
+    assert torch.equal(ho2, eager["o"].cpu())
 
 
 def test_decode_all_scores_equal_beyond_candidate_cap():

@@ -370,6 +370,27 @@ def bench_decode_e2e(dec, args, world):
     return ms / args.steps, h2d, d2h
 
 
+def bench_decode_shared_k16(dec, args, world):
+    """The same decode step with one k16 per retrieval kv head (the G query heads
+    of a kv head share it: 1/8 of the k16 bytes at G = 8), replayed from a graph."""
+    import torch
+    from long_context_sparse_rtp_b200 import DecodeGraph, rtp_index_scores
+    st = dec["st"]
+    w, L = st["w"], st["L"]
+    Wk = st["Wk"][[s for s in range(0, w.H_ret, w.G)]].contiguous()
+    _, k16 = rtp_index_scores(st["q"], st["k"], st["Wq"], Wk, st["role"], k16_per_kv_head=1)
+    g = DecodeGraph(st["k"], st["v"], k16, st["Wq"], Wk, st["role"], H=w.H, pos=L - 1, p=w.p,
+                    window=w.window, n_sink=w.n_sink, k16_per_kv_head=1)
+    g.q.copy_(st["q"])
+    ms, _ = time_steps(g.replay, args.steps, args.warmup, world, dec["flush"])
+    ms = max_over_ranks(ms, world) / args.steps
+    B = st["q"].shape[0]
+    k16_bytes = B * L * len(w.ret_kv) * 16 * 2
+    del g, k16
+    torch.cuda.empty_cache()
+    return dict(ms_step=ms, tokens_per_s=B * world / (ms / 1e3), k16_bytes=k16_bytes)
+
+
 # ------------------------------------------------------------------ prefill (ours)
 def bench_prefill(args, world, rank, pk):
     import torch
@@ -517,6 +538,7 @@ def main():
     pk = peaks()
     dec = bench_decode(args, world, rank, local, pk)
     e2e_ms, h2d, d2h = bench_decode_e2e(dec, args, world)
+    shared = bench_decode_shared_k16(dec, args, world)
     pre = None if args.no_prefill else bench_prefill(args, world, rank, pk)
 
     B = dec["B"]
@@ -555,6 +577,10 @@ def main():
                 "ms_per_step": e2e_ms,
                 "api": "DecodeGraph.step (pinned host q/k/v in, o out; one graph replay)"},
     }
+    line["decode_shared_k16"] = {
+        "workload": f"{DECODE_WL} with one k16 per retrieval kv head (k16_per_kv_head = 1)",
+        "tokens_per_s": shared["tokens_per_s"], "ms_per_step": shared["ms_step"],
+        "k16_bytes_per_step": shared["k16_bytes"]}
     if pre is not None:
         per = pre["per_kernel"]
         line["prefill"] = {

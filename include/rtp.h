@@ -142,6 +142,11 @@ RTP_API rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv_ro
  *   mass[]  (nullable) kept mass / Z.
  * The scores are recomputed by rtp_sparse_attn_prefill with the identical
  * arithmetic, so (thr, jtie) reproduce S exactly there.
+ * Workspace: rtp_workspace_size(RTP_OP_TOPP_SELECT, ...) asks for the status
+ * word plus two candidate-list slots per SM (128 rows x 4064 keys x 8 bytes
+ * each, about 1.2 GB on 148 SMs).  A workspace of at least 256 bytes but
+ * smaller than that is accepted: the kernel then refines every dense crossing
+ * range with extra sweeps instead of parked lists (same results, slower).
  */
 RTP_API rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_role,
                            int32_t k16_per_kv_head, rtp_view q16, rtp_view k16, float p,
@@ -165,9 +170,9 @@ RTP_API rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint8_t
 
 /*
  * One decode step for the retrieval heads (shape->Lq == 1, q_pos0 == Lk - 1):
- * indexer scores of the new query against the whole k16 cache, exact top-p,
- * union gather of the kept K/V rows per kv head, exact attention, split-KV
- * merge.  The k16 cache must already hold the new token's key (rtp_index_scores).
+ * indexer scores of the new query against the whole k16 cache (each a 16-term
+ * tensor-core dot product, as in rtp_topp_select), exact top-p, union gather of
+ * the kept K/V rows per kv head, exact attention, split-KV merge.  The k16 cache must already hold the new token's key (rtp_index_scores).
  * Optional outputs ([B][H_ret], nullable): thr, jtie, count, mass as in
  * rtp_topp_select.
  */

@@ -143,8 +143,8 @@ RTP_API rtp_status rtp_index_scores(const rtp_shape* shape, const uint8_t* kv_ro
  * The scores are recomputed by rtp_sparse_attn_prefill with the identical
  * arithmetic, so (thr, jtie) reproduce S exactly there.
  * Workspace: rtp_workspace_size(RTP_OP_TOPP_SELECT, ...) asks for the status
- * word plus two candidate-list slots per SM (128 rows x 4064 keys x 8 bytes
- * each, about 1.2 GB on 148 SMs).  A workspace of at least 256 bytes but
+ * word plus two candidate-list slots per SM (128 rows x 8128 keys x 8 bytes
+ * each, about 2.5 GB on 148 SMs).  A workspace of at least 256 bytes but
  * smaller than that is accepted: the kernel then refines every dense crossing
  * range with extra sweeps instead of parked lists (same results, slower).
  */

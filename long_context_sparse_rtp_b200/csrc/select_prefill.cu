@@ -60,9 +60,12 @@ constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
 // row states: REFINE1 = 32 uniform score sub-bins of the level-0 crossing bin,
 // REFINE = 5 composite-key bits, COLLECT / LIST = gather the crossing range's keys
 enum { ST_IDLE = 0, ST_REFINE1 = 1, ST_REFINE = 2, ST_COLLECT = 3, ST_DONE = 4, ST_LIST = 5 };
-// Crossing-range keys a row may park in its global list: a level's even and odd
-// entries go to separate 32-bit bin sums, <= 2032 keys x (2^21 + 1) < 2^32 each.
-constexpr int kListCap = 4064;
+// Crossing-range keys a row may park in its global list.  A level's even and odd
+// entries go to separate 32-bit bin sums, and the warp that reads the list moves
+// them into the 64-bit sums after every kListFlush entries: <= 2032 keys x
+// (2^21 + 1) < 2^32 in each copy between flushes.
+constexpr int kListFlush = 4064;
+constexpr int kListCap = 2 * kListFlush;
 
 struct SelParams {
   unsigned long long* lists;  // [slots][kBM][kListCap] crossing-bin keys, or null
@@ -846,6 +849,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             unsigned long long* const L = lists + (size_t)rr * kListCap;
             int kept = 0, above = 0;
             for (int k0 = 0; k0 < n; k0 += 32) {
+              if (k0 > 0 && k0 % kListFlush == 0) {  // only this warp adds to row rr
+                __syncwarp();
+                if (lane < kNB) {
+                  sm.u.hw[lane][rr] +=
+                      (unsigned long long)sm.wacc[0][lane][rr] + sm.wacc[1][lane][rr];
+                  sm.wacc[0][lane][rr] = 0u;
+                  sm.wacc[1][lane][rr] = 0u;
+                }
+                __syncwarp();
+              }
               const int k = k0 + lane;
               const unsigned long long ck = k < n ? __ldcg(L + k) : 0ull;
               const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
@@ -856,6 +869,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 L[kept + __popc(ball & lt)] = ck;
                 const int digit = (int)((ck >> (kKeyBits - pb - wl)) & ((1ull << wl) - 1));
                 // even and odd entries in separate copies: <= 2032 keys each
+                // between flushes
                 atomicAdd(&sm.wacc[lane & 1][(1 << wl) - 1 - digit][rr],
                           fixed_u(__fmul_rn(rel_w(key_score((uint32_t)(ck >> kIdxBits)), rm),
                                             rtk)));

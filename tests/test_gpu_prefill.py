@@ -192,7 +192,7 @@ def test_prefill_all_scores_equal():
 
 
 def test_prefill_all_scores_equal_deep():
-    """W_q16 = 0 at 10K rows: every key ties, so rows past 4064 keys take the
+    """W_q16 = 0 at 10K rows: every key ties, so rows past 8128 keys take the
     level-1 sub-bins (one sub-bin holds every key), the composite-key digits
     through the identical score bits, and the index bits; the kept set is still
     the ceil(p * N) lowest indices."""

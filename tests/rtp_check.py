@@ -1,6 +1,6 @@
 """Shared checks for the GPU-vs-oracle parity tests.
 
-Tolerances ("Parity contract"):
+Tolerances:
 
 * selection: the kept set of every retrieval row equals the oracle's, except for
   keys whose indexer score lies within SEL_BAND (relative, floor 1) of the row

@@ -1,6 +1,6 @@
 """GPU parity: causal prefill of one mixed layer against the fp64 oracle.
 
-Stage by stage ("Parity contract"):
+Stage by stage:
  (i)   q16/k16 projections equal the oracle's bf16 values, or sit one bf16 ulp
        away where the exact value lies within fp32-accumulation distance of a
        rounding midpoint;

@@ -14,8 +14,10 @@ scaling, no data-path collective).  The prefill of the 128K workload (1 x 131072
 tokens, chained needles) is timed in the same run and reported in `prefill`.
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
-events on the launching stream with a 256 MB L2 flush between steps (outside the
-events); a barrier + synchronize on both sides; the max over ranks.
+events on the launching stream with an L2 flush between steps (outside the
+events: 256 MB written, then 256 MB read, so that no dirty line of the flush is
+written back inside a timed step); a barrier + synchronize on both sides; the
+max over ranks.
 
 --impl reference times the fp64 CPU oracle on this host's cores on the same
 workload (rank 0 only).
@@ -250,6 +252,25 @@ def decode_step(st, o, lse):
                             n_sink=w.n_sink)
 
 
+L2_FLUSH = ("256 MB written, then another 256 MB read, between timed steps (outside the "
+            "events): the L2 (126 MB) holds none of the step's data and no dirty lines")
+
+
+def make_l2_flush():
+    """Between timed steps: write a buffer twice the L2 size, then read another
+    one.  The read evicts the written lines, so their write-back to HBM happens
+    here and not inside the next timed step."""
+    import torch
+    wbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    rbuf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        wbuf.fill_(1.0)
+        rbuf.sum()
+
+    return flush
+
+
 def time_steps(fn, steps, warmup, world, flush, traced=False):
     """Per-step CUDA events, L2 flush between steps (outside the events)."""
     import torch
@@ -308,10 +329,7 @@ def bench_decode(args, world, rank, local, pk):
     from long_context_sparse_rtp_b200 import DecodeGraph
     st = decode_state(rank)
     w, L = st["w"], st["L"]
-    flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-
-    def flush():
-        flushbuf.fill_(1.0)
+    flush = make_l2_flush()
 
     def make(trace_on=False):
         g = DecodeGraph(st["k"], st["v"], st["k16"], st["Wq"], st["Wk"], st["role"], H=w.H,
@@ -399,10 +417,7 @@ def bench_prefill(args, world, rank, pk):
     w = w.with_(seed=rank_seed(w.seed, rank))
     inp = synth.make_inputs(w, "cuda")
     q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
-    flushbuf = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
-
-    def flush():
-        flushbuf.fill_(1.0)
+    flush = make_l2_flush()
 
     def step():
         rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
@@ -559,7 +574,7 @@ def main():
                                "32 q / 4 kv heads, 1 retrieval kv head, p=0.95, window 4096+4",
                    "global_batch": B * world, "seq_len": dec["st"]["L"],
                    "parallelism": f"dp{world}",
-                   "l2": "256 MB L2 flush between timed steps (outside the events)"},
+                   "l2": L2_FLUSH},
         "phase": "decode",
         "roofline": {"bound": "hbm", "kernel": "dec_score", "achieved": achieved,
                      "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],

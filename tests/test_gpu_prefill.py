@@ -8,6 +8,7 @@ Stage by stage:
        matches outside the threshold band and the GPU cut is a valid top-p cut;
  (iii) outputs match the oracle run end to end (its own projections).
 """
+import ctypes
 import math
 
 import numpy as np
@@ -15,7 +16,8 @@ import pytest
 import torch
 
 import oracle
-from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
+from long_context_sparse_rtp_b200 import (rtp_index_scores, rtp_layer_prefill, rtp_topp_select,
+                                          synth)
 from rtp_check import (LSE_ABS, bits, check_outputs, check_row_outputs, check_row_selection, f64,
                        gpu_kept, row_reference,
                        oracle_k16, oracle_q16, row_scores)
@@ -212,3 +214,50 @@ def test_prefill_all_scores_equal_deep():
             assert np.array_equal(cnt[0, s], expect), s
             assert np.array_equal(jt[0, s], expect - 1), s
         assert np.all(res["sel"]["thr"].cpu().numpy() == 0.0)
+
+
+def _select_small_workspace(q16, k16, kv_role, p, H):
+    """rtp_topp_select through the C ABI with a workspace of only the status
+    word: the parked candidate lists are off."""
+    from long_context_sparse_rtp_b200 import rtp as R
+    B, Lq, n_ret = q16.shape[0], q16.shape[1], q16.shape[2]
+    out = dict(thr=torch.empty(B, n_ret, Lq, dtype=torch.float32, device="cuda"),
+               jtie=torch.empty(B, n_ret, Lq, dtype=torch.int32, device="cuda"),
+               count=torch.empty(B, n_ret, Lq, dtype=torch.int32, device="cuda"),
+               mass=torch.empty(B, n_ret, Lq, dtype=torch.float32, device="cuda"))
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    shp = R._shape(B, Lq, k16.shape[1], H, len(kv_role), 0)
+    rc = R.lib().rtp_topp_select(ctypes.byref(shp), R._role(kv_role), 0, R.view(q16, 16),
+                                 R.view(k16, 16), ctypes.c_float(p), R._ptr(out["thr"]),
+                                 R._ptr(out["jtie"]), R._ptr(out["count"]), R._ptr(out["mass"]),
+                                 R._ptr(ws), ws.numel(), R._stream())
+    assert rc == 0, rc
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32)[0]) == 0  # the device status word
+    return out
+
+
+@pytest.mark.parametrize("p", [0.95, 0.99])
+def test_select_without_list_workspace(p):
+    """With a workspace too small for the candidate lists, every dense crossing
+    range is refined by further sweeps instead of a parked list; the selection
+    is the same, bit for bit."""
+    w = W["prefill_128k"]
+    inp = synth.make_inputs(w, "cuda", L=6000)
+    role = inp["kv_role"]
+    q16, k16 = rtp_index_scores(inp["q"], inp["k"], inp["Wq16"], inp["Wk16"], role)
+    full = rtp_topp_select(q16, k16, role, p, H=w.H)
+    small = _select_small_workspace(q16, k16, role, p, w.H)
+    for key in ("thr", "jtie", "count", "mass"):
+        assert torch.equal(small[key], full[key]), key
+    # every key tied: each row's crossing range holds all its keys
+    wz = torch.zeros_like(inp["Wq16"])
+    q16z, _ = rtp_index_scores(inp["q"][:, :3000], inp["k"][:, :3000], wz, inp["Wk16"], role)
+    k16z = k16[:, :3000].contiguous()
+    full = rtp_topp_select(q16z, k16z, role, p, H=w.H)
+    small = _select_small_workspace(q16z, k16z, role, p, w.H)
+    for key in ("thr", "jtie", "count", "mass"):
+        assert torch.equal(small[key], full[key]), key
+    N = np.arange(1, 3001)
+    expect = np.maximum(1, np.ceil(float(np.float32(p)) * N)).astype(int)
+    assert np.array_equal(small["count"][0, 0].cpu().numpy(), expect)

@@ -18,9 +18,9 @@ import torch
 import oracle
 from long_context_sparse_rtp_b200 import (rtp_index_scores, rtp_layer_prefill, rtp_topp_select,
                                           synth)
-from rtp_check import (LSE_ABS, bits, check_outputs, check_row_outputs, check_row_selection, f64,
-                       gpu_kept, row_reference,
-                       oracle_k16, oracle_q16, row_scores)
+from rtp_check import (LSE_ABS, SEL_BAND, bits, check_outputs, check_row_outputs,
+                       check_row_selection, f64, gpu_kept, oracle_k16, oracle_q16,
+                       row_reference, row_scores)
 
 pytestmark = pytest.mark.gpu
 
@@ -261,3 +261,38 @@ def test_select_without_list_workspace(p):
     N = np.arange(1, 3001)
     expect = np.maximum(1, np.ceil(float(np.float32(p)) * N)).astype(int)
     assert np.array_equal(small["count"][0, 0].cpu().numpy(), expect)
+
+
+def test_single_key_sets_return_that_value_row():
+    """A kept set of one key makes the softmax weight exactly 1, so the output
+    is that key's V row bit for bit: p = 0 keeps only the top-scoring key (the
+    lowest index among equal maxima) on the retrieval heads, and a window of one
+    token without sinks keeps the query's own key on the local heads."""
+    w = W["prefill_2k"]
+    L = 777
+    inp = synth.make_inputs(w, "cuda", L=L)
+    q, k, v, role = inp["q"], inp["k"], inp["v"], inp["kv_role"]
+    res = rtp_layer_prefill(q, k, v, inp["Wq16"], inp["Wk16"], role, p=0.0, window=1, n_sink=0)
+    torch.cuda.synchronize()
+    sel = res["sel"]
+    assert bool((sel["count"] == 1).all())
+    jt = sel["jtie"].long()                                   # [B, H_ret, L]
+    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
+    o = res["o"]
+    for s, h in enumerate(ret):
+        g = h // w.G
+        assert torch.equal(o[0, :, h], v[0, jt[0, s], g]), h
+        # the kept key is a causal argmax of the indexer scores, the lowest index
+        # among equal maxima: checked in fp64 up to the selection band, since the
+        # GPU compares fp32 scores
+        sc = (res["q16"][0, :, s].double() @ res["k16"][0, :, s].double().T)
+        idx = torch.arange(L, device="cuda")
+        sc = sc.masked_fill(idx[None, :] > idx[:, None], float("-inf"))
+        best = sc.max(dim=1).values
+        mine = sc.gather(1, jt[0, s][:, None])[:, 0]
+        band = SEL_BAND * best.abs().clamp(min=1.0)
+        assert bool((best - mine <= band).all())
+        before = sc.masked_fill(idx[None, :] >= jt[0, s][:, None], float("-inf"))
+        assert bool((before.max(dim=1).values < mine + band).all())
+    for h in loc:
+        assert torch.equal(o[0, :, h], v[0, :, h // w.G]), h

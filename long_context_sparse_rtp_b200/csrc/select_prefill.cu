@@ -7,28 +7,42 @@
 // rows of one retrieval head and sweeps that head's k16 rows (L2-resident)
 // several times; every sweep recomputes the 128 x 128 score tiles
 // S = Q16 . K16^T on the tensor cores (one tcgen05.mma, M = N = 128, K = 16,
-// per tile, fp32 in TMEM) and one epilogue thread per query row reads its row
-// of each tile from TMEM, so all per-row state lives in that thread:
+// per tile, fp32 in TMEM).  Two epilogue threads per query row (TMEM lane r,
+// key columns 0-63 and 64-127 of each tile) read the scores with tcgen05.ld;
+// both derive the row's decisions identically from shared memory:
 //
-//   sweep 1  row max m and a lower bound on Z (running max per thread)
-//   sweep 2  Z = sum exp(s - m) in a fixed order and a 32-bin mass histogram of
-//            the scores in [c0, m], c0 = m - ln(N / ((1 - p) Z)) - 1 (keys below
-//            c0 + 1 are never kept: together they weigh < (1 - p) Z)
-//   sweep 3+ radix refinement inside the crossing bin on the composite key
-//            (score key : 32 bits, 2^21-1-index : 21 bits), 5 bits per sweep,
-//            until the crossing bin holds <= 32 keys; those are collected,
-//            sorted and walked to the exact cut.
+//   sweep 1  row max m and a lower bound Z_lo on Z = sum exp(s - m) (per 16 keys
+//            the larger of exp(max - m) and the mass of every fourth key)
+//   sweep 2  Z in a fixed order and a 32-bin mass histogram of the scores in
+//            [m - R, m], R = min(ln(N / ((1 - p) Z_lo)), ln(N / (1 - p))) + 1:
+//            keys below m - R + 1 are never kept (together they weigh less than
+//            (1 - p) Z); the crossing bin k0 is where the mass from the top
+//            reaches p Z
+//   sweep 3+ per row, until its crossing range holds <= 32 keys, which are
+//            collected, sorted and walked to the exact cut:
+//            - level 1: 32 uniform score sub-bins of bin k0 (one sweep);
+//            - then 5-bit digits of the composite key (score key : 32 bits,
+//              2^21-1-index : 21 bits), one sweep each;
+//            - a range of <= 8128 keys is instead parked once in the row's
+//              global list, and its remaining digits are resolved over the
+//              list, a warp per row, with no further sweep.
+//            A sweep tests each key against the rows' ranges with one compare
+//            (|s - mid| <= half) and queues the hits per warp; the queue is
+//            drained 32 hits at a time.  Range counts are bounds taken from
+//            the bin sums (every key adds at least a known amount); the count
+//            of keys above the final range is exact.
 //
 // Histogram masses are kept relative to the top edge e of their bin: a key adds
-// trunc(2^21 exp(s - e)) (a value in (0.7, 1] x 2^21) to its bin, so shared-memory
-// 32-bit atomics per tile group, flushed into 64-bit sums, are exact and
-// order-free; a bin's mass is its integer sum times exp(e - m) 2^-21, taken in
-// fp64 in a fixed order.  Z is a fixed-order fp32 tree per 32 keys summed in
-// fp64.  The selection is deterministic run to run.
+// trunc(2^21 exp(s - e)) (a value in (exp(-w), 1] x 2^21, w the bin width) to
+// its bin, so 32-bit shared-memory atomics per tile group, flushed into 64-bit
+// sums, are exact and order-free; a bin's mass is its integer sum times
+// exp(e - m) 2^-21, taken in fp64 in a fixed order.  Z is a fixed-order fp32
+// tree per 16 keys summed in fp64.  The selection is deterministic run to run.
 //
-// Warp roles: warps 0-3 epilogue (thread = query row = TMEM lane), warp 4 the
-// TMA producer (Q16 tile once, K16 tiles into a ring), warp 5 the MMA issuer
-// (owns the 256 TMEM columns: two 128-column accumulators).
+// Warp roles: warps 0-7 epilogue (warps w and w + 4 share TMEM lanes 32 (w & 3)
+// .. +31, one column half each), warp 8 the TMA producer (Q16 tile once, K16
+// tiles into a ring), warp 9 the MMA issuer (owns the 256 TMEM columns: two
+// 128-column accumulators).
 #include <cuda.h>
 
 #include "rtp_host.h"

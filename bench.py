@@ -409,6 +409,21 @@ def bench_decode_shared_k16(dec, args, world):
     return dict(ms_step=ms, tokens_per_s=B * world / (ms / 1e3), k16_bytes=k16_bytes)
 
 
+def bench_decode_dense(dec, args):
+    """The dense kernel on the same decode step: every query head attends to the
+    whole cache (rtp_dense_attn with one query row), the baseline the sparse
+    step replaces.  Algorithmic bytes: the K and V rows of every kv head."""
+    import torch
+    from long_context_sparse_rtp_b200 import rtp_dense_attn
+    st = dec["st"]
+    q, k, v, L = st["q"], st["k"], st["v"], st["L"]
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[2], 1, dtype=torch.float32, device=q.device)
+    ms, _ = time_steps(lambda: rtp_dense_attn(q, k, v, q_pos0=L - 1, o=o, lse=lse),
+                       args.steps, args.warmup, 1, dec["flush"])
+    return dict(ms_step=ms / args.steps, bytes=k.shape[0] * L * k.shape[2] * 128 * 2 * 2)
+
+
 # ------------------------------------------------------------------ prefill (ours)
 def bench_prefill(args, world, rank, pk):
     import torch
@@ -555,6 +570,12 @@ def main():
     e2e_ms, h2d, d2h = bench_decode_e2e(dec, args, world)
     shared = bench_decode_shared_k16(dec, args, world)
     pre = None if args.no_prefill else bench_prefill(args, world, rank, pk)
+    dense = None
+    if world == 1:  # a reported baseline: no collective, so one rank only
+        try:
+            dense = bench_decode_dense(dec, args)
+        except Exception as e:  # report, never hide
+            dense = {"error": repr(e)}
 
     B = dec["B"]
     value = B * world / (dec["ms_step"] / 1e3)
@@ -606,6 +627,15 @@ def main():
             "dense_baseline_ms": pre["dense_ms"], "speedup_vs_dense": pre["dense_ms"] / pre["ms_step"],
             "kept_pairs": pre["sel_pairs"], "causal_pairs": pre["causal_pairs"],
         }
+    if dense is not None:
+        line["dense_decode"] = dense if "error" in dense else {
+            "workload": f"{DECODE_WL} with every query head dense over the whole cache "
+                        "(rtp_dense_attn, one query row)",
+            "ms_per_step": dense["ms_step"], "tokens_per_s": B / (dense["ms_step"] / 1e3),
+            "bytes_per_step": dense["bytes"],
+            "achieved_gbs": dense["bytes"] / (dense["ms_step"] / 1e3) / 1e9,
+            "frac_of_hbm": dense["bytes"] / (dense["ms_step"] / 1e3) / 1e9 / pk["hbm"],
+            "sparse_step_speedup": dense["ms_step"] / dec["ms_step"]}
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         try:
             stc = oracle_host_state(dec["st"]["w"], "cuda")

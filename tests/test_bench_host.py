@@ -73,3 +73,33 @@ def test_warmup_below_three_is_refused(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--warmup", "2"])
     with pytest.raises(SystemExit):
         bench.main()
+
+
+def test_dense_decode_leg_bookkeeping(monkeypatch):
+    """The dense-decode baseline leg: one rtp_dense_attn call per step with the
+    query at the last cache position, and the K/V bytes of every kv head."""
+    import long_context_sparse_rtp_b200 as pkg
+    B, L, H, Hkv = 8, 131072, 32, 4
+    st = dict(q=torch.empty(B, 1, H, 128, device="meta"),
+              k=torch.empty(B, L, Hkv, 128, device="meta"),
+              v=torch.empty(B, L, Hkv, 128, device="meta"), L=L)
+    calls = []
+
+    def fake_dense(q, k, v, *, q_pos0, o, lse):
+        calls.append((q_pos0, tuple(o.shape), tuple(lse.shape)))
+
+    def fake_time_steps(fn, steps, warmup, world, flush):
+        for _ in range(warmup + steps):
+            fn()
+        return 0.35 * steps, None
+
+    monkeypatch.setattr(pkg, "rtp_dense_attn", fake_dense)
+    monkeypatch.setattr(bench, "time_steps", fake_time_steps)
+
+    class Args:
+        steps, warmup = 4, 3
+
+    r = bench.bench_decode_dense(dict(st=st, flush=None), Args)
+    assert r["bytes"] == B * L * Hkv * 128 * 2 * 2 == 2147483648
+    assert abs(r["ms_step"] - 0.35) < 1e-12
+    assert calls == [(L - 1, (B, 1, H, 128), (B, H, 1))] * 7

@@ -131,3 +131,24 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rtp, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         rtp.lib()
+
+
+def test_product_never_reaches_the_oracle(L):
+    """The oracle is test infrastructure: no module of the package imports it,
+    and librtp.so neither links the oracle's library nor carries its symbols."""
+    import ast
+    import subprocess
+    pkg = os.path.join(ROOT, "long_context_sparse_rtp_b200")
+    for name in sorted(os.listdir(pkg)):
+        if not name.endswith(".py"):
+            continue
+        tree = ast.parse(open(os.path.join(pkg, name)).read())
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import):
+                assert all(a.name.split(".")[0] != "oracle" for a in node.names), name
+            elif isinstance(node, ast.ImportFrom):
+                assert (node.module or "").split(".")[0] != "oracle", name
+    deps = subprocess.run(["ldd", rtp.LIB_PATH], capture_output=True, text=True).stdout
+    assert "orc" not in deps
+    syms = subprocess.run(["nm", "-D", rtp.LIB_PATH], capture_output=True, text=True).stdout
+    assert not any(ln.split()[-1].startswith("orc_") for ln in syms.splitlines() if ln.split())

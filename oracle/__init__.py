@@ -20,6 +20,13 @@ Steps", arXiv 2605.16928, cited by section):
                      ties go to the lower index.
 * ``attend``      -- same section, exact softmax attention over the kept set
                      with the 1/sqrt(d_h) scale.
+* ``topk``        -- §5 Experimental Analysis, the method's static top-k
+                     variant (k = 4096): the k highest scores, ties to the
+                     lower index.
+* ``block_topp``  -- §Hardware-Aware Fast Top-p Decoding Kernel, steps 1-5:
+                     64-key blocks reduced to (max, log-sum-exp), a 256-bin
+                     histogram over the block maxima, a walk down the bins to
+                     mass p, whole blocks selected.
 * ``local_set``   -- §Local Head Attention Pattern (sinks + sliding window).
 * ``retrieval_rows`` / ``local_rows`` / ``dense_rows`` -- the above per row.
 
@@ -134,6 +141,45 @@ def topp(s: np.ndarray, p: float) -> dict:
                  ctypes.byref(mf), ctypes.byref(Z), ctypes.byref(m))
     return dict(sel=sel.astype(bool), t=t.value, jtie=jt.value, count=cnt.value,
                 mass_frac=mf.value, Z=Z.value, m=m.value)
+
+
+def topk(s: np.ndarray, k: int) -> dict:
+    """Static top-k of one row of scores.  Returns sel (bool [n]), t, jtie, count."""
+    lib = _load()
+    s = _c(s, np.float64).reshape(-1)
+    n = s.size
+    if n < 1 or k < 1:
+        raise ValueError("top-k needs at least one key and k >= 1")
+    sel = np.empty(n, np.uint8)
+    t = ctypes.c_double()
+    jt = ctypes.c_int64()
+    cnt = ctypes.c_int64()
+    lib.orc_topk(_p(s), ctypes.c_int64(n), ctypes.c_int64(k), _p(sel), ctypes.byref(t),
+                 ctypes.byref(jt), ctypes.byref(cnt))
+    return dict(sel=sel.astype(bool), t=t.value, jtie=jt.value, count=cnt.value)
+
+
+def block_topp(s: np.ndarray, p: float, block: int = 64, nbins: int = 256) -> dict:
+    """Block-level approximate top-p of one row of scores.  Returns bsel (bool
+    [nb]), bin (int [nb]), kstar, sel (bool [n], the kept tokens), count,
+    mass_frac (kept share of the token softmax mass)."""
+    lib = _load()
+    s = _c(s, np.float64).reshape(-1)
+    n = s.size
+    if n < 1:
+        raise ValueError("block top-p needs at least one key")
+    nb = (n + block - 1) // block
+    bsel = np.empty(nb, np.uint8)
+    bins = np.empty(nb, np.int64)
+    ks = ctypes.c_int64()
+    cnt = ctypes.c_int64()
+    mf = ctypes.c_double()
+    lib.orc_block_topp(_p(s), ctypes.c_int64(n), ctypes.c_double(p), ctypes.c_int64(block),
+                       ctypes.c_int64(nbins), _p(bsel), _p(bins), ctypes.byref(ks),
+                       ctypes.byref(cnt), ctypes.byref(mf))
+    bsel = bsel.astype(bool)
+    return dict(bsel=bsel, bin=bins, kstar=ks.value, sel=np.repeat(bsel, block)[:n],
+                count=cnt.value, mass_frac=mf.value)
 
 
 def attend(q_bits, K_bits, V_bits, idx, scale: float):

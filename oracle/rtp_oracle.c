@@ -210,6 +210,153 @@ void orc_topp(const double* s, int64_t n, double p, uint8_t* sel, double* t,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Static top-k  [FASB §5 Experimental Analysis: the top-k variant of the   */
+/* method, k = 4096, the fixed-budget baseline of the top-p ablation]       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Keep the k highest-scoring keys of s[0..n-1] (n >= 1, k >= 1); equal scores
+ * go to the lower index, the same (score desc, index asc) order as orc_topp.
+ * k >= n keeps every key.  Outputs as orc_topp (each nullable): sel, the
+ * threshold t (score of the last kept key), jtie (its index), count = min(k, n).
+ */
+void orc_topk(const double* s, int64_t n, int64_t k, uint8_t* sel, double* t,
+              int64_t* jtie, int64_t* count)
+{
+    orc_key* order = (orc_key*)malloc((size_t)n * sizeof(orc_key));
+    for (int64_t j = 0; j < n; ++j) {
+        order[j].s = s[j];
+        order[j].j = j;
+    }
+    qsort(order, (size_t)n, sizeof(orc_key), orc_key_cmp);
+    const int64_t kept = k < n ? k : n;
+    if (sel) {
+        memset(sel, 0, (size_t)n);
+        for (int64_t a = 0; a < kept; ++a)
+            sel[order[a].j] = 1;
+    }
+    if (t)
+        *t = order[kept - 1].s;
+    if (jtie)
+        *jtie = order[kept - 1].j;
+    if (count)
+        *count = kept;
+    free(order);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-level approximate top-p, sort-free by a histogram                  */
+/* [FASB §Hardware-Aware Fast Top-p Decoding Kernel, steps 1-5]             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The keys s[0..n-1] (n >= 1) in blocks of `block` consecutive keys (the last
+ * one may be shorter), nb = ceil(n / block):
+ *   1-2. per block b: m_b = max of its scores and l_b = log sum exp of its
+ *        scores (the block's attention mass, in log form);
+ *   3.   a histogram of nbins bins over the block maxima: the range
+ *        [lo, hi] = [min m_b, max m_b] cut into nbins equal bins,
+ *        bin(b) = min(nbins - 1, floor(((m_b - lo) / (hi - lo)) * nbins))
+ *        (every block in the top bin when hi == lo); each bin accumulates the
+ *        masses exp(l_b - hi) of its blocks (the log-sum-exp of their l_b);
+ *   4.   walk the bins from the highest down, accumulating their masses; the
+ *        first bin at which the running mass reaches p * (total mass) is the
+ *        threshold bin (p >= 1: the lowest occupied bin);
+ *   5.   block b is selected iff bin(b) >= the threshold bin: the threshold
+ *        bin is kept whole, since the histogram cannot tell its blocks apart.
+ * Outputs (each nullable): bsel[nb] (1 = selected), bin_of[nb], the threshold
+ * bin kstar, the kept token count, and the kept share of the token-level
+ * softmax mass sum_{kept j} exp(s_j - max) / sum_j exp(s_j - max).
+ * The range arithmetic is written as above in fp64 so that a caller may feed
+ * it binary32 scores and reproduce any implementation that evaluates the same
+ * expression in fp64.
+ */
+void orc_block_topp(const double* s, int64_t n, double p, int64_t block, int64_t nbins,
+                    uint8_t* bsel, int64_t* bin_of, int64_t* kstar_out,
+                    int64_t* kept_count, double* kept_mass_frac)
+{
+    const int64_t nb = (n + block - 1) / block;
+    double* mb = (double*)malloc((size_t)nb * sizeof(double));
+    double* lb = (double*)malloc((size_t)nb * sizeof(double));
+    int64_t* bin = (int64_t*)malloc((size_t)nb * sizeof(int64_t));
+    double* hist = (double*)calloc((size_t)nbins, sizeof(double));
+    for (int64_t b = 0; b < nb; ++b) {
+        const int64_t j0 = b * block, j1 = (j0 + block < n) ? j0 + block : n;
+        double m = s[j0];
+        for (int64_t j = j0 + 1; j < j1; ++j)
+            if (s[j] > m)
+                m = s[j];
+        double acc = 0.0;
+        for (int64_t j = j0; j < j1; ++j)
+            acc += exp(s[j] - m);
+        mb[b] = m;
+        lb[b] = m + log(acc);
+    }
+    double lo = mb[0], hi = mb[0];
+    for (int64_t b = 1; b < nb; ++b) {
+        if (mb[b] < lo)
+            lo = mb[b];
+        if (mb[b] > hi)
+            hi = mb[b];
+    }
+    double total = 0.0;
+    for (int64_t b = 0; b < nb; ++b) {
+        int64_t k = nbins - 1;
+        if (hi > lo) {
+            const double x = floor(((mb[b] - lo) / (hi - lo)) * (double)nbins);
+            k = x < (double)(nbins - 1) ? (int64_t)x : nbins - 1;
+        }
+        bin[b] = k;
+        const double w = exp(lb[b] - hi);
+        hist[k] += w;
+        total += w;
+    }
+    int64_t kstar = 0;
+    if (p >= 1.0) {
+        for (kstar = 0; kstar < nbins && hist[kstar] == 0.0; ++kstar) {
+        }
+    } else {
+        double cum = 0.0;
+        for (int64_t k = nbins - 1; k >= 0; --k) {
+            if (hist[k] == 0.0)
+                continue;
+            cum += hist[k];
+            kstar = k;
+            if (cum >= p * total)
+                break;
+        }
+    }
+    double m = hi, Z = 0.0, kept_m = 0.0;
+    int64_t cnt = 0;
+    for (int64_t b = 0; b < nb; ++b) {
+        const int64_t j0 = b * block, j1 = (j0 + block < n) ? j0 + block : n;
+        const int on = bin[b] >= kstar;
+        for (int64_t j = j0; j < j1; ++j) {
+            const double w = exp(s[j] - m);
+            Z += w;
+            if (on) {
+                kept_m += w;
+                ++cnt;
+            }
+        }
+        if (bsel)
+            bsel[b] = (uint8_t)on;
+        if (bin_of)
+            bin_of[b] = bin[b];
+    }
+    if (kstar_out)
+        *kstar_out = kstar;
+    if (kept_count)
+        *kept_count = cnt;
+    if (kept_mass_frac)
+        *kept_mass_frac = kept_m / Z;
+    free(mb);
+    free(lb);
+    free(bin);
+    free(hist);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Exact attention over an index set  [FASB §Dynamic Top-p ..., sparse      */
 /* attention formula]: O = sum_{n in S} softmax_S(q.k_n * scale) v_n        */
 /* ------------------------------------------------------------------------ */

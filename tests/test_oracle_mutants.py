@@ -38,6 +38,17 @@ MUTANTS = [
     ("local: window one key too wide", "j > P - window", "j >= P - window", 1),
     ("local: sinks dropped", "if (j < n_sink || j > P - window)", "if (j > P - window)", 1),
     ("GQA: kv head by modulo", "h = row_h[r], g = h / G;", "h = row_h[r], g = h % S.Hkv;", 2),
+    ("top-k: one key too many", "const int64_t kept = k < n ? k : n;",
+     "const int64_t kept = k < n ? k + 1 : n;", 1),
+    ("block top-p: bins walked from the bottom", "for (int64_t k = nbins - 1; k >= 0; --k) {",
+     "for (int64_t k = 0; k < nbins; ++k) {", 1),
+    ("block top-p: block mass from its max, not its log-sum-exp",
+     "const double w = exp(lb[b] - hi);", "const double w = exp(mb[b] - hi);", 1),
+    ("block top-p: threshold bin left out", "const int on = bin[b] >= kstar;",
+     "const int on = bin[b] > kstar;", 1),
+    ("block top-p: range from 0, not from the lowest block max",
+     "floor(((mb[b] - lo) / (hi - lo)) * (double)nbins)", "floor((mb[b] / hi) * (double)nbins)",
+     1),
 ]
 
 

@@ -392,3 +392,124 @@ def test_retrieval_rows_match_composition():
         o, lse = _numpy_causal_attention(qf[b, i:i + 1, h], kf[b, :i + 1, 0], vf[b, :i + 1, 0],
                                          mask, scale)
         np.testing.assert_allclose(r["o"][rr], o[0], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- static top-k
+# [FASB §5 Experimental Analysis]: the method's fixed-budget variant keeps the k
+# highest-scoring keys (k = 4096 there); ties go to the lower index, the order the
+# top-p rule uses.
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_equals_sorted_prefix(seed):
+    """Against numpy's lexsort of (score desc, index asc): the first k keys."""
+    rng = np.random.default_rng(200 + seed)
+    n = int(rng.integers(1, 40))
+    s = rng.integers(-3, 4, n).astype(float)  # many exact ties
+    order = np.lexsort((np.arange(n), -s))
+    for k in (1, 2, 5, n - 1, n, n + 3):
+        if k < 1:
+            continue
+        r = oracle.topk(s, k)
+        want = np.zeros(n, bool)
+        want[order[:min(k, n)]] = True
+        assert np.array_equal(r["sel"], want), (k, s)
+        assert r["count"] == min(k, n)
+        last = order[min(k, n) - 1]
+        assert r["jtie"] == last and r["t"] == s[last]
+
+
+def test_topk_special_cases():
+    s = np.array([0.5, 2.0, 2.0, -1.0, 2.0])
+    r = oracle.topk(s, 1)
+    assert list(np.nonzero(r["sel"])[0]) == [1]          # argmax, lowest index
+    r = oracle.topk(s, 2)
+    assert list(np.nonzero(r["sel"])[0]) == [1, 2]       # tie at the cut: lower index
+    assert oracle.topk(s, 99)["sel"].all()               # k >= n: every key
+    z = oracle.topk(np.zeros(10), 4)                     # all equal: the first k indices
+    assert list(np.nonzero(z["sel"])[0]) == [0, 1, 2, 3] and z["jtie"] == 3
+
+
+# ---------------------------------------------------------------- block top-p
+# [FASB §Hardware-Aware Fast Top-p Decoding Kernel], steps 1-5.
+
+def _golden_block_topp():
+    cases = []
+    with open(os.path.join(GOLDEN, "block_topp_hand.txt")) as f:
+        for line in f:
+            if not line.strip() or line.startswith("#"):
+                continue
+            _, spec, p, blocks = (c.strip() for c in line.split("|"))
+            s = np.concatenate([np.full(int(c), float(v))
+                                for v, c in (run.split("*") for run in spec.split())])
+            cases.append((s, float(p), [int(t) for t in blocks.split()]))
+    return cases
+
+
+@pytest.mark.parametrize("s,p,blocks", _golden_block_topp())
+def test_block_topp_golden(s, p, blocks):
+    r = oracle.block_topp(s, p)
+    assert list(np.nonzero(r["bsel"])[0]) == blocks
+    n = s.size
+    assert r["count"] == sum(min(64, n - 64 * b) for b in blocks)
+    assert np.array_equal(np.nonzero(r["sel"])[0],
+                          np.concatenate([np.arange(64 * b, min(64 * b + 64, n)) for b in blocks]))
+
+
+def _block_brute_force(s, p, block=64):
+    """With every block alone in its histogram bin, the selection is the shortest
+    prefix of blocks ranked by their max (descending) whose summed softmax mass
+    reaches p of the total: computed here block by block, with no histogram."""
+    nb = (s.size + block - 1) // block
+    m = s.max()
+    mass = np.array([np.exp(s[b * block:(b + 1) * block] - m).sum() for b in range(nb)])
+    mx = np.array([s[b * block:(b + 1) * block].max() for b in range(nb)])
+    order = np.argsort(-mx, kind="stable")
+    keep = np.zeros(nb, bool)
+    acc = 0.0
+    for b in order:
+        keep[b] = True
+        acc += mass[b]
+        if acc >= p * mass.sum():
+            break
+    return keep
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_block_topp_brute_force_distinct_bins(seed):
+    rng = np.random.default_rng(300 + seed)
+    nb = int(rng.integers(2, 7))
+    n = 64 * (nb - 1) + int(rng.integers(1, 65))           # a short last block
+    # block maxima at least 3 bins apart: every block in its own bin
+    tops = rng.permutation(np.linspace(0.0, 8.0, nb))
+    s = np.empty(n)
+    for b in range(nb):
+        blk = slice(64 * b, min(64 * b + 64, n))
+        w = blk.stop - blk.start
+        s[blk] = tops[b] - rng.uniform(0.0, 3.0, w)
+        s[blk.start + int(rng.integers(0, w))] = tops[b]
+    for p in (0.0, 0.3, 0.6, 0.9, 0.95, 0.999):
+        r = oracle.block_topp(s, p)
+        assert len(set(r["bin"])) == nb
+        assert np.array_equal(r["bsel"], _block_brute_force(s, p)), (p, r["bin"])
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_block_topp_invariants(seed):
+    """p >= 1 keeps every block; p = 0 keeps exactly the top bin's blocks; the
+    selection grows with p; the kept softmax mass reaches p; the block holding
+    the argmax key is always kept."""
+    rng = np.random.default_rng(400 + seed)
+    n = int(rng.integers(65, 3000))
+    s = rng.standard_normal(n) * 4.0
+    r1 = oracle.block_topp(s, 1.0)
+    assert r1["bsel"].all() and r1["count"] == n and abs(r1["mass_frac"] - 1.0) < 1e-12
+    r0 = oracle.block_topp(s, 0.0)
+    assert np.array_equal(r0["bsel"], r0["bin"] == 255)
+    prev = None
+    for p in np.linspace(0.0, 1.0, 21):
+        r = oracle.block_topp(s, p)
+        assert r["bsel"][int(np.argmax(s)) // 64]
+        assert r["mass_frac"] >= p - 1e-12
+        if prev is not None:
+            assert np.all(r["bsel"] >= prev)
+        prev = r["bsel"]

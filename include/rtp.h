@@ -160,6 +160,12 @@ RTP_API rtp_status rtp_topp_select(const rtp_shape* shape, const uint8_t* kv_rol
  * S given by (thr, jtie) from rtp_topp_select on the same q16/k16.
  * o: retrieval heads written (bf16), lse (nullable): [B][H][Lq] fp32, natural
  * log of the softmax denominator including the scale.
+ * thr == jtie == NULL selects the p >= 1 case, every causal key kept: the
+ * retrieval heads run on the dense tile schedule and q16/k16 are not read (may
+ * be null views).  That is the prefill the summary describes, retrieval heads
+ * attending densely while only the local heads are sparse [FASB
+ * §Hardware-Aware Fast Top-p Decoding Kernel, "Prefill kernel"].  Passing only
+ * one of the two is RTP_ERR_INVALID_ARG.
  */
 RTP_API rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint8_t* kv_role,
                                    int32_t k16_per_kv_head, rtp_view q, rtp_view k,
@@ -183,6 +189,46 @@ RTP_API rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8_t*
                                   float* thr, int32_t* jtie, int32_t* count, float* mass,
                                   void* ws, size_t ws_bytes, rtp_stream_t stream);
 
+/* Token selection rule of a retrieval decode step (rtp_sparse_attn_decode_select). */
+typedef enum rtp_select {
+    RTP_SELECT_TOPP = 0,       /* exact token-level top-p (as rtp_sparse_attn_decode) */
+    RTP_SELECT_BLOCK_TOPP = 1, /* block-level approximate top-p, 64-key blocks */
+    RTP_SELECT_TOPK = 2        /* static top-k */
+} rtp_select;
+
+/*
+ * One decode step for the retrieval heads with a choice of selection rule; the
+ * scores, the union gather and the split-KV attention are those of
+ * rtp_sparse_attn_decode, which equals this call with RTP_SELECT_TOPP.
+ *  - RTP_SELECT_BLOCK_TOPP [FASB §Hardware-Aware Fast Top-p Decoding Kernel,
+ *    steps 1-5]: keys 0..P in blocks of 64 (the last one shorter), each
+ *    reduced to its max m_b and the log-sum-exp l_b of its scores; a 256-bin
+ *    histogram over [min m_b, max m_b], bin = min(255, floor(((m_b - lo) /
+ *    (hi - lo)) * 256)) evaluated in fp64 from the fp32 scores (all blocks in
+ *    bin 255 when hi == lo); each bin sums exp(l_b - hi); the bins are walked
+ *    from the top until the running mass reaches p of the total (p >= 1: every
+ *    block) and every block of that bin or above is kept, all its keys
+ *    attended.  block_mask (nullable) receives, per row [B][H_ret], the
+ *    ceil(ceil((P + 1) / 64) / 32) words of one bit per block (bit b % 32 of
+ *    word b / 32).  count = kept keys, mass = their share of the indexer
+ *    softmax mass; thr and jtie are not written.
+ *  - RTP_SELECT_TOPK [FASB §5 Experimental Analysis, the method's static top-k
+ *    variant, k = 4096 there]: the top_k highest scores (top_k >= 1), ties to
+ *    the lower index; every key when top_k > P.  thr, jtie, count, mass as in
+ *    rtp_topp_select (thr = -inf when every key is kept).  p is ignored.
+ *  - scores_out (nullable): [B][H_ret][P + 1] fp32, the indexer scores the
+ *    selection used (each a 16-term tensor-core dot product of bf16 q16 and
+ *    k16 with fp32 accumulation), for tests and diagnostics.
+ * Workspace: rtp_workspace_size(RTP_OP_SPARSE_DECODE, ...), as
+ * rtp_sparse_attn_decode.
+ */
+RTP_API rtp_status rtp_sparse_attn_decode_select(
+    const rtp_shape* shape, const uint8_t* kv_role, int32_t k16_per_kv_head, rtp_view q,
+    rtp_view k_cache, rtp_view v_cache, rtp_view q16, rtp_view k16_cache, rtp_select select,
+    float p, int32_t top_k, float softmax_scale, rtp_view o, float* lse, float* thr,
+    int32_t* jtie, int32_t* count, float* mass, uint32_t* block_mask, float* scores_out,
+    void* ws, size_t ws_bytes, rtp_stream_t stream);
+
 /*
  * Local heads: keys j <= P with j < n_sink or j > P - window
  * [FASB §Local Head Attention Pattern].  Prefill (Lq > 1) and decode (Lq == 1)
@@ -192,6 +238,42 @@ RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role
                           int32_t n_sink, rtp_view q, rtp_view k, rtp_view v,
                           float softmax_scale, rtp_view o, float* lse, void* ws,
                           size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Window-only local-head cache [FASB §Local Head Attention Pattern, decode: the
+ * local heads keep only the sink tokens and the sliding window, so their cache
+ * stays O(window) however long the sequence grows].
+ *
+ * A ring cache holds the local kv heads only: k_ring / v_ring are
+ * [B][n_sink + window][n_local_kv][128] bf16 views (rtp_view with heads =
+ * number of local kv heads, in increasing kv head order).  Position j < n_sink
+ * lives in row j; position j >= n_sink in row n_sink + (j - n_sink) % window.
+ *
+ * rtp_local_ring_write copies the local kv heads of source rows into the ring:
+ * shape->Lq source rows of k / v ([B][Lq][Hkv][128], row i = absolute position
+ * shape->q_pos0 + i; shape->Lk is not used).  Only the sinks and the last
+ * `window` positions of the range are copied (earlier ones would be
+ * overwritten): after a prefill, write rows 0..L-1 once; each decode step then
+ * writes its new token (Lq = 1, q_pos0 = its position).  Positions must be
+ * written in increasing order over calls.  No workspace.
+ */
+RTP_API rtp_status rtp_local_ring_write(const rtp_shape* shape, const uint8_t* kv_role,
+                                        int32_t window, int32_t n_sink, rtp_view k, rtp_view v,
+                                        rtp_view k_ring, rtp_view v_ring, rtp_stream_t stream);
+
+/*
+ * Local-head decode from a ring cache: as rtp_local_attn with shape->Lq == 1
+ * (query at P = shape->q_pos0, shape->Lk >= P + 1), keys j <= P with
+ * j < n_sink or j > P - window read from k_ring / v_ring, which must hold every
+ * such position (rtp_local_ring_write up to P).  The keys are visited in the
+ * same order as rtp_local_attn over a full cache, so the result is the same bit
+ * for bit.  Workspace: rtp_workspace_size(RTP_OP_LOCAL, ...).
+ */
+RTP_API rtp_status rtp_local_attn_decode_ring(const rtp_shape* shape, const uint8_t* kv_role,
+                                              int32_t window, int32_t n_sink, rtp_view q,
+                                              rtp_view k_ring, rtp_view v_ring,
+                                              float softmax_scale, rtp_view o, float* lse,
+                                              void* ws, size_t ws_bytes, rtp_stream_t stream);
 
 /*
  * Local-head decode that allocates nothing (the paper has no counterpart; this
@@ -205,16 +287,19 @@ RTP_API rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_role
  * which loads the library holds until the process exits.
  *  - Same arguments and results as rtp_local_attn for one decode token, minus
  *    the workspace.  Shapes whose partials exceed the array return
- *    RTP_ERR_SCRATCH_LIMIT before anything is enqueued (the need is about
- *    8448 bytes per (batch entry, local kv head, split), with
- *    min(ceil(296 / (B * local_kv_heads)), ceil(n_keys / 64)) splits; n_keys
- *    is the number of sink and window keys, at most window + n_sink).
- *  - The first call on a device looks the array's device address up
- *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    RTP_ERR_SCRATCH_LIMIT before anything is enqueued.  The need is 256 bytes
+ *    plus 8448 bytes per (batch entry, local kv head, split), with
+ *    min(256, ceil(296 / (B * local_kv_heads)), ceil(n_keys / 64)) splits, at
+ *    least 1; n_keys is the number of sink and window keys, at most
+ *    window + n_sink.
+ *  - Every call looks the array's device address up (cudaGetSymbolAddress)
+ *    on the current device, so a device reset is harmless.  The first call on
+ *    a device also loads the library's device code there; make that first call
  *    outside any stream capture.
- *  - Every call reuses the same array; calls
- *    that overlap on the GPU (other streams, other threads) race on it and
- *    must be serialised by the caller.
+ *  - Every call reuses the same array and overwrites what the last call left
+ *    there (nothing in it needs clearing between calls); calls that overlap on
+ *    the GPU (other streams, other threads) race on it and must be serialised
+ *    by the caller.
  *  - Never calls cudaMalloc, cudaFree or any allocating routine.
  */
 #define RTP_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -257,6 +342,15 @@ RTP_API void rtp_trace_enable(int on);
 RTP_API void rtp_trace_reset(void);
 /* Fills up to max_entries entries; returns the number filled, or -1 on a CUDA error. */
 RTP_API int rtp_trace_read(rtp_trace_entry* out, int max_entries);
+
+/*
+ * Measurement aid (no counterpart in the paper): launches `blocks` CTAs of 256
+ * threads that each issue iters x 8 dependent-chain ex2.approx.f32
+ * instructions (blocks * 2048 * iters in all), for timing the device's exp
+ * rate with CUDA events.  `out`: device buffer of blocks * 256 floats, never
+ * written in practice.
+ */
+RTP_API rtp_status rtp_probe_ex2(int32_t blocks, int32_t iters, float* out, rtp_stream_t stream);
 
 /* Library version, e.g. "0.1.0". */
 RTP_API const char* rtp_version(void);

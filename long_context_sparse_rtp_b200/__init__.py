@@ -9,12 +9,16 @@ loudly if it is not built.
 """
 from .rtp import (  # noqa: F401
     RtpError,
+    local_ring_alloc,
     rtp_check_device,
     rtp_dense_attn,
     rtp_get_device_status,
     rtp_index_scores,
     rtp_local_attn,
+    rtp_local_attn_decode_ring,
+    rtp_local_ring_write,
     rtp_sparse_attn_decode,
+    rtp_sparse_attn_decode_select,
     rtp_sparse_attn_prefill,
     rtp_status_string,
     rtp_topp_select,

@@ -548,6 +548,17 @@ rtp_status prefill_dense(const rtp_shape* shape, const rtp_view& q, const rtp_vi
   return launch_tc<MODE_DENSE>(prm, shape->H, shape, q, k, v, nullptr, nullptr, 0, 0, s);
 }
 
+// Every causal key of the retrieval heads only (p >= 1: the kept set is the
+// whole causal prefix), on the dense tile schedule with no indexer recompute.
+rtp_status prefill_dense_retrieval(const rtp_shape* shape, const HeadMap& hm, const rtp_view& q,
+                                   const rtp_view& k, const rtp_view& v, float scale,
+                                   const rtp_view& o, float* lse, void* ws, cudaStream_t s) {
+  AttnParams prm;
+  fill_common(prm, shape, o, lse, scale, ws);
+  for (int hr = 0; hr < hm.n_ret; ++hr) prm.head[hr] = hm.ret_q[hr];
+  return launch_tc<MODE_DENSE>(prm, hm.n_ret, shape, q, k, v, nullptr, nullptr, 0, 0, s);
+}
+
 rtp_status prefill_sparse(const rtp_shape* shape, const HeadMap& hm, const rtp_view& q,
                           const rtp_view& k, const rtp_view& v, const rtp_view& q16,
                           const rtp_view& k16, const float* thr, const int32_t* jtie,

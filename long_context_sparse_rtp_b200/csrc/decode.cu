@@ -13,7 +13,6 @@
 //   merge    a second kernel, one CTA per (batch, kv group, head), combines the
 //            splits in split order.
 #include <algorithm>
-#include <mutex>
 
 #include "rtp_host.h"
 
@@ -24,6 +23,9 @@ rtp_status prefill_local(const rtp_shape*, const HeadMap&, int, int, const rtp_v
                          cudaStream_t);
 rtp_status prefill_dense(const rtp_shape*, const rtp_view&, const rtp_view&, const rtp_view&,
                          float, const rtp_view&, float*, void*, cudaStream_t);
+rtp_status prefill_dense_retrieval(const rtp_shape*, const HeadMap&, const rtp_view&,
+                                   const rtp_view&, const rtp_view&, float, const rtp_view&,
+                                   float*, void*, cudaStream_t);
 rtp_status prefill_sparse(const rtp_shape*, const HeadMap&, const rtp_view&, const rtp_view&,
                           const rtp_view&, const rtp_view&, const rtp_view&, const float*,
                           const int32_t*, float, const rtp_view&, float*, void*, cudaStream_t);
@@ -49,7 +51,11 @@ struct DecAttnParams {
   // range mode
   int64_t P; int n_sink_eff; int64_t win_lo; int64_t n_keys; int keys_per_split;
   float* part;                            // [B*groups][n_splits][16][2+128]
-  int16_t kvh[kMaxHeads];                 // group -> kv head
+  int16_t kvh[kMaxHeads];                 // group -> kv head (its query heads in q, o, lse)
+  int16_t kslot[kMaxHeads];               // group -> head slot of the k / v views
+  // ring cache (range mode): position j >= ring_sink lives in row
+  // ring_sink + (j - ring_sink) % ring_w of k / v; ring_w == 0: row j
+  int ring_w, ring_sink;
 };
 
 constexpr int kDecThreads = 128;
@@ -146,8 +152,8 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
     e_end = min(p.n_keys, e_begin + p.keys_per_split);
     n_entries = (int)max((int64_t)0, e_end - e_begin);
   }
-  const uint16_t* kb = p.k + b * p.k_sb + (int64_t)kvh * kD;
-  const uint16_t* vb = p.v + b * p.v_sb + (int64_t)kvh * kD;
+  const uint16_t* kb = p.k + b * p.k_sb + (int64_t)p.kslot[grp] * kD;
+  const uint16_t* vb = p.v + b * p.v_sb + (int64_t)p.kslot[grp] * kD;
 
   if (LIST) {
     if (tid < G) {
@@ -202,6 +208,8 @@ __global__ void __launch_bounds__(kDecThreads) dec_attn_kernel(const DecAttnPara
           msk = sm.emask[e];
         } else {
           j = range_key(round0 + e);
+          if (p.ring_w > 0 && j >= p.ring_sink)
+            j = p.ring_sink + (int64_t)((uint32_t)(j - p.ring_sink) % (uint32_t)p.ring_w);
           msk = allmask;
         }
       }
@@ -455,10 +463,12 @@ void fill_dec_common(DecAttnParams& prm, const rtp_shape* shape, const rtp_view&
 }
 
 // Range-mode decode over keys {j <= P : j < n_sink or j > P - window}.
+// With ring_w > 0 the k / v views are ring caches holding only these groups'
+// heads (slot i = group i) of n_sink + ring_w rows.
 rtp_status decode_range(const rtp_shape* shape, const int16_t* kv_heads, int n_groups,
                         int window, int n_sink, const rtp_view& q, const rtp_view& k,
                         const rtp_view& v, float scale, const rtp_view& o, float* lse,
-                        void* ws, size_t ws_bytes, cudaStream_t s) {
+                        void* ws, size_t ws_bytes, cudaStream_t s, int ring_w = 0) {
   if (n_groups == 0 || shape->B == 0) return RTP_OK;
   const int64_t P = shape->q_pos0;
   const int64_t n_sink_eff = std::min<int64_t>((int64_t)n_sink, P + 1);
@@ -477,8 +487,50 @@ rtp_status decode_range(const rtp_shape* shape, const int16_t* kv_heads, int n_g
   prm.n_keys = n_keys;
   prm.keys_per_split = L.keys_per_split;
   prm.part = reinterpret_cast<float*>(static_cast<char*>(ws) + L.part);
-  for (int i = 0; i < n_groups; ++i) prm.kvh[i] = kv_heads[i];
+  prm.ring_w = ring_w;
+  prm.ring_sink = n_sink;
+  for (int i = 0; i < n_groups; ++i) {
+    prm.kvh[i] = kv_heads[i];
+    prm.kslot[i] = ring_w > 0 ? (int16_t)i : kv_heads[i];
+  }
   return launch_dec_attn<false>(prm, shape->B, s);
+}
+
+// ------------------------------------------------------------------ ring cache writes
+// Copies the local kv heads of source positions into a ring cache: position
+// j < n_sink to row j, position j >= n_sink to row n_sink + (j - n_sink) % window.
+// Only the positions a later query can still see are copied: the sinks and the
+// last `window` positions of the range (an earlier one would be overwritten).
+struct RingWriteParams {
+  const uint16_t* k; int64_t k_sb, k_sl;  // source row i holds position pos0 + i
+  const uint16_t* v; int64_t v_sb, v_sl;
+  uint16_t* kr; int64_t kr_sb, kr_sl;     // ring [B][n_sink + window][n_lkv][128]
+  uint16_t* vr; int64_t vr_sb, vr_sl;
+  int64_t pos0, a0, a1, w0, w1;           // sink positions [a0, a1), window [w0, w1)
+  int n_sink, window, n_lkv;
+  int16_t lkv[kMaxHeads];
+};
+
+constexpr int kRingThreads = 256;
+
+__global__ void __launch_bounds__(kRingThreads) ring_write_kernel(const RingWriteParams p) {
+  const int64_t e = (int64_t)blockIdx.x * kRingThreads + threadIdx.x;
+  const int b = blockIdx.y;
+  const int chunk = (int)(e & 15);               // 16 bytes of a 256-byte head row
+  const int64_t rest = e >> 4;
+  const int i = (int)(rest % p.n_lkv);
+  const int64_t m = rest / p.n_lkv;
+  const int64_t n1 = p.a1 - p.a0;
+  const int64_t j = m < n1 ? p.a0 + m : p.w0 + (m - n1);
+  if (m >= n1 && j >= p.w1) return;
+  const int64_t slot =
+      j < p.n_sink ? j : p.n_sink + (int64_t)((uint64_t)(j - p.n_sink) % (uint64_t)p.window);
+  const int64_t src_k = b * p.k_sb + (j - p.pos0) * p.k_sl + (int64_t)p.lkv[i] * kD + chunk * 8;
+  const int64_t src_v = b * p.v_sb + (j - p.pos0) * p.v_sl + (int64_t)p.lkv[i] * kD + chunk * 8;
+  const int64_t dk = b * p.kr_sb + slot * p.kr_sl + (int64_t)i * kD + chunk * 8;
+  const int64_t dv = b * p.vr_sb + slot * p.vr_sl + (int64_t)i * kD + chunk * 8;
+  *reinterpret_cast<uint4*>(p.kr + dk) = *reinterpret_cast<const uint4*>(p.k + src_k);
+  *reinterpret_cast<uint4*>(p.vr + dv) = *reinterpret_cast<const uint4*>(p.v + src_v);
 }
 
 }  // namespace
@@ -499,7 +551,7 @@ rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, cons
   prm.rowres = lists.rowres;
   prm.n_ret = hm.n_ret;
   prm.part = lists.part;
-  for (int i = 0; i < hm.n_rkv; ++i) prm.kvh[i] = hm.rkv[i];
+  for (int i = 0; i < hm.n_rkv; ++i) prm.kvh[i] = prm.kslot[i] = hm.rkv[i];
   return launch_dec_attn<true>(prm, shape->B, s);
 }
 
@@ -561,6 +613,70 @@ extern "C" rtp_status rtp_local_attn(const rtp_shape* shape, const uint8_t* kv_r
   return prefill_local(shape, hm, window, n_sink, q, k, v, softmax_scale, o, lse, ws, s);
 }
 
+extern "C" rtp_status rtp_local_ring_write(const rtp_shape* shape, const uint8_t* kv_role,
+                                           int32_t window, int32_t n_sink, rtp_view k,
+                                           rtp_view v, rtp_view k_ring, rtp_view v_ring,
+                                           rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, 0, &hm)) != RTP_OK) return st;
+  if (window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+  if (shape->B == 0 || shape->Lq == 0 || hm.n_lkv == 0) return RTP_OK;
+  if ((st = check_view(k, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(k_ring, hm.n_lkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v_ring, hm.n_lkv, kD, true)) != RTP_OK) return st;
+  RingWriteParams p;
+  memset(&p, 0, sizeof(p));
+  p.k = static_cast<const uint16_t*>(k.ptr); p.k_sb = k.stride_b; p.k_sl = k.stride_l;
+  p.v = static_cast<const uint16_t*>(v.ptr); p.v_sb = v.stride_b; p.v_sl = v.stride_l;
+  p.kr = static_cast<uint16_t*>(k_ring.ptr); p.kr_sb = k_ring.stride_b; p.kr_sl = k_ring.stride_l;
+  p.vr = static_cast<uint16_t*>(v_ring.ptr); p.vr_sb = v_ring.stride_b; p.vr_sl = v_ring.stride_l;
+  const int64_t pos0 = shape->q_pos0, end = pos0 + shape->Lq;
+  p.pos0 = pos0;
+  p.a0 = pos0;
+  p.a1 = std::max(pos0, std::min<int64_t>(n_sink, end));
+  p.w0 = std::max<int64_t>(std::max<int64_t>(n_sink, end - window), pos0);
+  p.w1 = std::max(p.w0, end);
+  p.n_sink = n_sink;
+  p.window = window;
+  p.n_lkv = hm.n_lkv;
+  for (int i = 0; i < hm.n_lkv; ++i) p.lkv[i] = hm.lkv[i];
+  const int64_t items = ((p.a1 - p.a0) + (p.w1 - p.w0)) * hm.n_lkv * 16;
+  if (items == 0) return RTP_OK;
+  const int64_t blocks = (items + kRingThreads - 1) / kRingThreads;
+  if (blocks > 0x7FFFFFFF || shape->B > 65535) return RTP_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TraceScope tr("ring_write", s);
+  ring_write_kernel<<<dim3((unsigned)blocks, shape->B), kRingThreads, 0, s>>>(p);
+  return check_cuda(cudaGetLastError());
+}
+
+extern "C" rtp_status rtp_local_attn_decode_ring(const rtp_shape* shape, const uint8_t* kv_role,
+                                                 int32_t window, int32_t n_sink, rtp_view q,
+                                                 rtp_view k_ring, rtp_view v_ring,
+                                                 float softmax_scale, rtp_view o, float* lse,
+                                                 void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  if (shape->Lq != 1) return RTP_ERR_INVALID_ARG;
+  if ((st = check_causal(shape)) != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, 0, &hm)) != RTP_OK) return st;
+  if (window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return RTP_ERR_INVALID_ARG;
+  if (shape->B == 0 || hm.n_lkv == 0) return RTP_OK;
+  if (hm.G > 16 || (256 % hm.G) != 0) return RTP_ERR_UNSUPPORTED;
+  if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(k_ring, hm.n_lkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v_ring, hm.n_lkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
+  if (ws == nullptr || ws_bytes < kStatusBytes) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  return decode_range(shape, hm.lkv, hm.n_lkv, window, n_sink, q, k_ring, v_ring, softmax_scale,
+                      o, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), window);
+}
+
 extern "C" rtp_status rtp_dense_attn(const rtp_shape* shape, rtp_view q, rtp_view k, rtp_view v,
                                      float softmax_scale, rtp_view o, float* lse, void* ws,
                                      size_t ws_bytes, rtp_stream_t stream) {
@@ -602,14 +718,18 @@ extern "C" rtp_status rtp_sparse_attn_prefill(const rtp_shape* shape, const uint
   if (shape->Lk > kMaxKeys) return RTP_ERR_UNSUPPORTED;
   const bool work = shape->B > 0 && shape->Lq > 0 && hm.n_ret > 0;
   if (!work) return RTP_OK;
-  if (thr == nullptr || jtie == nullptr) return RTP_ERR_INVALID_ARG;
+  if ((thr == nullptr) != (jtie == nullptr)) return RTP_ERR_INVALID_ARG;
+  const bool all_keys = thr == nullptr;  // p >= 1: every causal key, dense tiles
   if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
   if ((st = check_view(k, shape->Hkv, kD, true)) != RTP_OK) return st;
   if ((st = check_view(v, shape->Hkv, kD, true)) != RTP_OK) return st;
   if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
-  if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
-  if ((st = check_view(k16, hm.H_k16, kR, true)) != RTP_OK) return st;
+  if ((st = check_view(q16, hm.n_ret, kR, !all_keys)) != RTP_OK) return st;
+  if ((st = check_view(k16, hm.H_k16, kR, !all_keys)) != RTP_OK) return st;
   if (ws == nullptr || ws_bytes < kStatusBytes) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  if (all_keys)
+    return prefill_dense_retrieval(shape, hm, q, k, v, softmax_scale, o, lse, ws,
+                                   reinterpret_cast<cudaStream_t>(stream));
   return prefill_sparse(shape, hm, q, k, v, q16, k16, thr, jtie, softmax_scale, o, lse, ws,
                         reinterpret_cast<cudaStream_t>(stream));
 }
@@ -622,24 +742,16 @@ namespace {
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the array on the current device (looked up once per device;
-// in host code the symbol itself is only a host-side stand-in).
+// Device address of the array on the current device.  In host code the symbol
+// itself is only a host-side stand-in, so the address is looked up on every
+// call: a lookup allocates nothing, costs far less than the launch, and stays
+// right after the context is destroyed and created again (cudaDeviceReset),
+// which reloads the module at a new address.
 rtp_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return RTP_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return RTP_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return RTP_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    return RTP_ERR_CUDA;
+  *out = p;
   return RTP_OK;
 }
 

@@ -1148,40 +1148,15 @@ __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectPara
 
 using namespace rtp;
 
-extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8_t* kv_role,
-                                             int32_t k16_per_kv_head, rtp_view q,
-                                             rtp_view k_cache, rtp_view v_cache, rtp_view q16,
-                                             rtp_view k16_cache, float p, float softmax_scale,
-                                             rtp_view o, float* lse, float* thr, int32_t* jtie,
-                                             int32_t* count, float* mass, void* ws,
-                                             size_t ws_bytes, rtp_stream_t stream) {
-  rtp_status st = check_shape(shape);
-  if (st != RTP_OK) return st;
-  if (shape->Lq != 1) return RTP_ERR_INVALID_ARG;
-  if ((st = check_causal(shape)) != RTP_OK) return st;
-  HeadMap hm;
-  if ((st = make_headmap(shape, kv_role, k16_per_kv_head, &hm)) != RTP_OK) return st;
-  if (!(p >= 0.f && p <= 1.f)) return RTP_ERR_INVALID_ARG;
-  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return RTP_ERR_INVALID_ARG;
-  if (hm.G > 16 || (256 % hm.G) != 0) return RTP_ERR_UNSUPPORTED;
-  if (shape->Lk > kMaxKeys) return RTP_ERR_UNSUPPORTED;
-  const bool work = shape->B > 0 && hm.n_ret > 0;
-  if (!work) return RTP_OK;
-  if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
-  if ((st = check_view(k_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
-  if ((st = check_view(v_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
-  if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
-  if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
-  if ((st = check_view(k16_cache, hm.H_k16, kR, true)) != RTP_OK) return st;
-  const DecodeWs L = decode_ws_layout(shape, hm);
-  if (ws == nullptr || ws_bytes < L.total) return RTP_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+namespace rtp {
+rtp_status decode_score_pass(const rtp_shape* shape, const HeadMap& hm, int k16_per_kv_head,
+                             const rtp_view& q16, const rtp_view& k16_cache, void* ws,
+                             const DecodeWs& L, cudaStream_t s) {
+  rtp_status st = RTP_OK;
   char* w = static_cast<char*>(ws);
   const int N = (int)(shape->q_pos0 + 1);  // keys 0..P
-  const int nc = (N + kDecChunk - 1) / kDecChunk;
   const int groups = shape->B * hm.n_rkv;
   auto at = [&](size_t off) { return static_cast<void*>(w + off); };
-
   // the row histograms and flags accumulate with atomics: clear them
   if (cudaMemsetAsync(at(L.hist_m), 0, L.rowsel - L.hist_m, s) != cudaSuccess)
     return RTP_ERR_CUDA;
@@ -1249,6 +1224,59 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
     TraceScope tr("dec_score", s);
     dec_score_kernel<<<grid, kSThreads, smem, s>>>(kmap, sp);
     if ((st = check_cuda(cudaGetLastError())) != RTP_OK) return st;
+  }
+  return RTP_OK;
+}
+}  // namespace rtp
+
+extern "C" rtp_status rtp_sparse_attn_decode_select(
+    const rtp_shape* shape, const uint8_t* kv_role, int32_t k16_per_kv_head, rtp_view q,
+    rtp_view k_cache, rtp_view v_cache, rtp_view q16, rtp_view k16_cache, rtp_select select,
+    float p, int32_t top_k, float softmax_scale, rtp_view o, float* lse, float* thr,
+    int32_t* jtie, int32_t* count, float* mass, uint32_t* block_mask, float* scores_out,
+    void* ws, size_t ws_bytes, rtp_stream_t stream) {
+  rtp_status st = check_shape(shape);
+  if (st != RTP_OK) return st;
+  if (shape->Lq != 1) return RTP_ERR_INVALID_ARG;
+  if ((st = check_causal(shape)) != RTP_OK) return st;
+  HeadMap hm;
+  if ((st = make_headmap(shape, kv_role, k16_per_kv_head, &hm)) != RTP_OK) return st;
+  if (select != RTP_SELECT_TOPP && select != RTP_SELECT_BLOCK_TOPP && select != RTP_SELECT_TOPK)
+    return RTP_ERR_INVALID_ARG;
+  if (select != RTP_SELECT_TOPK && !(p >= 0.f && p <= 1.f)) return RTP_ERR_INVALID_ARG;
+  if (select == RTP_SELECT_TOPK && top_k < 1) return RTP_ERR_INVALID_ARG;
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale)) return RTP_ERR_INVALID_ARG;
+  if (hm.G > 16 || (256 % hm.G) != 0) return RTP_ERR_UNSUPPORTED;
+  if (shape->Lk > kMaxKeys) return RTP_ERR_UNSUPPORTED;
+  const bool work = shape->B > 0 && hm.n_ret > 0;
+  if (!work) return RTP_OK;
+  if ((st = check_view(q, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(k_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(v_cache, shape->Hkv, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(o, shape->H, kD, true)) != RTP_OK) return st;
+  if ((st = check_view(q16, hm.n_ret, kR, true)) != RTP_OK) return st;
+  if ((st = check_view(k16_cache, hm.H_k16, kR, true)) != RTP_OK) return st;
+  const DecodeWs L = decode_ws_layout(shape, hm);
+  if (ws == nullptr || ws_bytes < L.total) return RTP_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int N = (int)(shape->q_pos0 + 1);  // keys 0..P
+  const int nc = (N + kDecChunk - 1) / kDecChunk;
+  const int groups = shape->B * hm.n_rkv;
+  auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+
+  if ((st = decode_score_pass(shape, hm, k16_per_kv_head, q16, k16_cache, ws, L, s)) != RTP_OK)
+    return st;
+  if (scores_out != nullptr && L.rows > 0 &&
+      cudaMemcpy2DAsync(scores_out, (size_t)N * 4, at(L.scores), (size_t)L.Lk_pad * 4,
+                        (size_t)N * 4, (size_t)L.rows, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  if (select != RTP_SELECT_TOPP) {  // static top-k or block-level top-p (decode_variants.cu)
+    DecodeLists dl;
+    if ((st = decode_variant_select(shape, hm, select, p, top_k, ws, L, thr, jtie, count, mass,
+                                    block_mask, &dl, s)) != RTP_OK)
+      return st;
+    return decode_list_attention(shape, hm, q, k_cache, v_cache, softmax_scale, o, lse, dl, s);
   }
   {  // 2. per-row merge
     MergeParams mp;
@@ -1318,4 +1346,17 @@ extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8
   dl.n_splits = decode_list_splits(groups, nc);
   if (dl.n_splits > L.n_splits) return RTP_ERR_WORKSPACE_TOO_SMALL;
   return decode_list_attention(shape, hm, q, k_cache, v_cache, softmax_scale, o, lse, dl, s);
+}
+
+extern "C" rtp_status rtp_sparse_attn_decode(const rtp_shape* shape, const uint8_t* kv_role,
+                                             int32_t k16_per_kv_head, rtp_view q,
+                                             rtp_view k_cache, rtp_view v_cache, rtp_view q16,
+                                             rtp_view k16_cache, float p, float softmax_scale,
+                                             rtp_view o, float* lse, float* thr, int32_t* jtie,
+                                             int32_t* count, float* mass, void* ws,
+                                             size_t ws_bytes, rtp_stream_t stream) {
+  return rtp_sparse_attn_decode_select(shape, kv_role, k16_per_kv_head, q, k_cache, v_cache, q16,
+                                       k16_cache, RTP_SELECT_TOPP, p, 0, softmax_scale, o, lse,
+                                       thr, jtie, count, mass, nullptr, nullptr, ws, ws_bytes,
+                                       stream);
 }

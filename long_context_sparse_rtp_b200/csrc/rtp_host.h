@@ -151,9 +151,13 @@ SelectWs select_ws_layout();
 
 struct DecodeWs {   // retrieval decode
   size_t scores, hist_m, hist_c, flags, sub_m, sub_c, rowsel, rowres, cand, ncand, counter, list, lcount, loff,
-      part, total;
+      part, blk, bmask, total;
   int n_chunks, n_splits, Lk_pad, rows, groups;
+  int n_blk, n_bwords;  // 64-key blocks per row (of Lk_pad) and their mask words
 };
+
+constexpr int kDecBlk = 64;    // keys per block of the block-level top-p
+constexpr int kDecHBins = 256; // its histogram bins over the block maxima
 
 inline int decode_list_splits(int groups, int n_chunks) {
   int want = groups > 0 ? (296 + groups - 1) / groups : 1;
@@ -194,9 +198,20 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
   w.lcount = take(groups * nc * 4);
   w.loff = take(groups * (nc + 1) * 4);
   w.part = take(groups * w.n_splits * 16 * kPartRow * 4);
+  w.n_blk = w.Lk_pad / kDecBlk;
+  w.n_bwords = (w.n_blk + 31) / 32;
+  w.blk = take((size_t)w.rows * w.n_blk * 8);       // (max, log-sum-exp) per block
+  w.bmask = take((size_t)w.rows * w.n_bwords * 4);  // selected blocks, one bit each
   w.total = off;
   return w;
 }
+
+// The retrieval decode's first pass (decode_select.cu): clears the row
+// histograms, then scores every key of the cache into the workspace's score
+// rows [rows][Lk_pad] and bins them.
+rtp_status decode_score_pass(const rtp_shape* shape, const HeadMap& hm, int k16_per_kv,
+                             const rtp_view& q16, const rtp_view& k16_cache, void* ws,
+                             const DecodeWs& L, cudaStream_t s);
 
 // Buffers the gathered decode attention reads (decode.cu).
 struct DecodeLists {
@@ -207,6 +222,14 @@ struct DecodeLists {
   float* part;
   int Lk_pad, n_chunks, n_splits;
 };
+
+// Static top-k or block-level top-p over the score rows decode_score_pass left
+// in the workspace (decode_variants.cu): per-row results, then the kept-key
+// union lists for decode_list_attention, described in *lists.
+rtp_status decode_variant_select(const rtp_shape* shape, const HeadMap& hm, rtp_select select,
+                                 float p, int top_k, void* ws, const DecodeWs& L, float* thr,
+                                 int32_t* jtie, int32_t* count, float* mass,
+                                 uint32_t* block_mask, DecodeLists* lists, cudaStream_t s);
 
 rtp_status decode_list_attention(const rtp_shape* shape, const HeadMap& hm, const rtp_view& q,
                                  const rtp_view& k, const rtp_view& v, float scale,

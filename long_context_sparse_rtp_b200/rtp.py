@@ -23,6 +23,8 @@ STATUS = {0: "RTP_OK", 1: "RTP_ERR_INVALID_ARG", 2: "RTP_ERR_UNSUPPORTED",
           3: "RTP_ERR_ALIGNMENT", 4: "RTP_ERR_WORKSPACE_TOO_SMALL", 5: "RTP_ERR_CUDA",
           6: "RTP_ERR_DEVICE_TIMEOUT", 7: "RTP_ERR_SCRATCH_LIMIT"}
 OP_INDEX_SCORES, OP_TOPP_SELECT, OP_SPARSE_PREFILL, OP_SPARSE_DECODE, OP_LOCAL, OP_DENSE = range(6)
+SELECT_TOPP, SELECT_BLOCK_TOPP, SELECT_TOPK = range(3)
+SELECT = {"topp": SELECT_TOPP, "block_topp": SELECT_BLOCK_TOPP, "topk": SELECT_TOPK}
 
 
 class RtpError(RuntimeError):
@@ -67,16 +69,24 @@ def lib():
                                                       P, sz, P]
                 L.rtp_sparse_attn_decode.argtypes = [S, P, i32, V, V, V, V, V, f32, f32, V, P,
                                                      P, P, P, P, P, sz, P]
+                L.rtp_sparse_attn_decode_select.argtypes = [S, P, i32, V, V, V, V, V, i32, f32,
+                                                            i32, f32, V, P, P, P, P, P, P, P,
+                                                            P, sz, P]
                 L.rtp_local_attn.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P, sz, P]
+                L.rtp_local_ring_write.argtypes = [S, P, i32, i32, V, V, V, V, P]
+                L.rtp_local_attn_decode_ring.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P,
+                                                         sz, P]
                 L.rtp_dense_attn.argtypes = [S, V, V, V, f32, V, P, P, sz, P]
                 L.rtp_local_attn_decode_noalloc.argtypes = [S, P, i32, i32, V, V, V, f32, V, P, P]
+                L.rtp_probe_ex2.argtypes = [i32, i32, P, P]
                 L.rtp_status_string.restype = ctypes.c_char_p
                 L.rtp_status_string.argtypes = [ctypes.c_int]
                 L.rtp_get_device_status.argtypes = [P, P]
                 L.rtp_version.restype = ctypes.c_char_p
                 for fn in ("rtp_workspace_init", "rtp_index_scores", "rtp_topp_select",
                            "rtp_sparse_attn_prefill", "rtp_sparse_attn_decode",
-                           "rtp_local_attn", "rtp_dense_attn", "rtp_get_device_status",
+                           "rtp_sparse_attn_decode_select", "rtp_local_attn",
+                           "rtp_local_ring_write", "rtp_local_attn_decode_ring", "rtp_probe_ex2", "rtp_dense_attn", "rtp_get_device_status",
                            "rtp_local_attn_decode_noalloc"):
                     getattr(L, fn).restype = ctypes.c_int
                 _lib = L
@@ -141,6 +151,11 @@ def rtp_status_string(code: int) -> str:
     return lib().rtp_status_string(code).decode()
 
 
+def rtp_probe_ex2(blocks: int, iters: int, out: torch.Tensor, stream=None) -> None:
+    """The ex2-rate probe kernel (blocks x 256 threads x iters x 8 ex2)."""
+    _check("rtp_probe_ex2", lib().rtp_probe_ex2(blocks, iters, _ptr(out), _stream(stream)))
+
+
 def rtp_version() -> str:
     return lib().rtp_version().decode()
 
@@ -172,15 +187,16 @@ def _n_ret(kv_role, G):
 
 
 def rtp_index_scores(q, k, Wq16, Wk16, kv_role, *, q16=None, k16=None, k16_per_kv_head=0,
-                     stream=None):
-    """16-dim indexer projections.  q [B,Lq,H,128] (or None), k [B,Lk,Hkv,128] (or None).
+                     H=None, stream=None):
+    """16-dim indexer projections.  q [B,Lq,H,128] (or None), k [B,Lk,Hkv,128] (or None;
+    then pass H, the query head count).
     Returns (q16 [B,Lq,H_ret,16], k16 [B,Lk,H_k16,16]); pass q16/k16 to write in place."""
     ref = q if q is not None else k
     B = ref.shape[0]
-    H = q.shape[2] if q is not None else None
+    H = q.shape[2] if q is not None else H
     Hkv = len(kv_role)
     if H is None:
-        raise ValueError("q is needed for the head count")
+        raise ValueError("pass q or H for the head count")
     G = H // Hkv
     n_ret = _n_ret(kv_role, G)
     H_k16 = int(sum(int(x) for x in kv_role)) if k16_per_kv_head else n_ret
@@ -221,7 +237,9 @@ def rtp_topp_select(q16, k16, kv_role, p, *, H, q_pos0=0, k16_per_kv_head=0, wan
 
 def rtp_sparse_attn_prefill(q, k, v, q16, k16, thr, jtie, kv_role, *, scale=None, q_pos0=0,
                             k16_per_kv_head=0, o=None, lse=None, stream=None):
-    """Exact attention over the kept sets (retrieval heads).  Returns (o, lse)."""
+    """Exact attention over the kept sets (retrieval heads).  Returns (o, lse).
+    thr = jtie = None keeps every causal key (p >= 1) on the dense tile schedule;
+    q16/k16 may then be None."""
     B, Lq, H, _ = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     dev = q.device
@@ -273,6 +291,50 @@ def rtp_sparse_attn_decode(q, k_cache, v_cache, q16, k16_cache, kv_role, p, *, s
     return o, lse, sel
 
 
+def rtp_sparse_attn_decode_select(q, k_cache, v_cache, q16, k16_cache, kv_role, select, *,
+                                  p=0.95, top_k=4096, scale=None, q_pos0=None,
+                                  k16_per_kv_head=0, o=None, lse=None, want_scores=False,
+                                  want_sel=True, stream=None):
+    """One decode step for the retrieval heads with selection rule `select`
+    ("topp", "block_topp" or "topk").  Returns (o, lse, sel) with sel a dict of
+    [B, H_ret] tensors (thr, jtie, count, mass; thr/jtie unwritten for
+    block_topp), plus block_mask [B, H_ret, words] int32 (block_topp) and
+    scores [B, H_ret, P + 1] fp32 (want_scores)."""
+    B, Lq, H, _ = q.shape
+    Lk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    dev = q.device
+    n_ret = q16.shape[2]
+    q_pos0 = Lk - 1 if q_pos0 is None else q_pos0
+    N = q_pos0 + 1
+    mode = SELECT[select]
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, 1), float("nan"), dtype=torch.float32, device=dev)
+    sel = {}
+    if want_sel:
+        sel = dict(thr=torch.full((B, n_ret), float("nan"), dtype=torch.float32, device=dev),
+                   jtie=torch.full((B, n_ret), -1, dtype=torch.int32, device=dev),
+                   count=torch.empty(B, n_ret, dtype=torch.int32, device=dev),
+                   mass=torch.empty(B, n_ret, dtype=torch.float32, device=dev))
+        words = ((N + 63) // 64 + 31) // 32
+        if mode == SELECT_BLOCK_TOPP:
+            sel["block_mask"] = torch.zeros(B, n_ret, words, dtype=torch.int32, device=dev)
+    if want_scores:
+        sel["scores"] = torch.empty(B, n_ret, N, dtype=torch.float32, device=dev)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, Lq, Lk, H, Hkv, q_pos0)
+    role = _role(kv_role)
+    ws = workspace(OP_SPARSE_DECODE, shp, role, k16_per_kv_head, dev, stream)
+    _check("rtp_sparse_attn_decode_select", lib().rtp_sparse_attn_decode_select(
+        ctypes.byref(shp), role, k16_per_kv_head, view(q), view(k_cache), view(v_cache),
+        view(q16, 16), view(k16_cache, 16), mode, ctypes.c_float(p), int(top_k),
+        ctypes.c_float(scale), view(o), _ptr(lse), _ptr(sel.get("thr")), _ptr(sel.get("jtie")),
+        _ptr(sel.get("count")), _ptr(sel.get("mass")), _ptr(sel.get("block_mask")),
+        _ptr(sel.get("scores")), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse, sel
+
+
 def rtp_local_attn(q, k, v, kv_role, *, window, n_sink, scale=None, q_pos0=0, o=None,
                    lse=None, stream=None):
     """Sink + sliding-window attention on the local heads (prefill or Lq == 1 decode)."""
@@ -289,6 +351,45 @@ def rtp_local_attn(q, k, v, kv_role, *, window, n_sink, scale=None, q_pos0=0, o=
     ws = workspace(OP_LOCAL, shp, role, 0, dev, stream)
     _check("rtp_local_attn", lib().rtp_local_attn(
         ctypes.byref(shp), role, window, n_sink, view(q), view(k), view(v),
+        ctypes.c_float(scale), view(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def local_ring_alloc(B, kv_role, *, window, n_sink, device):
+    """Zeroed (k_ring, v_ring) of [B, n_sink + window, n_local_kv, 128] bf16."""
+    n_lkv = sum(1 for x in kv_role if int(x) == 0)
+    shape = (B, n_sink + window, n_lkv, 128)
+    return (torch.zeros(shape, dtype=torch.bfloat16, device=device),
+            torch.zeros(shape, dtype=torch.bfloat16, device=device))
+
+
+def rtp_local_ring_write(k, v, k_ring, v_ring, kv_role, *, window, n_sink, pos0=0, H=None,
+                         stream=None):
+    """Copy the local kv heads of k, v [B, n, Hkv, 128] (row i = position pos0 + i)
+    into the ring cache; only the sinks and the last `window` positions land."""
+    B, n, Hkv, _ = k.shape
+    H = Hkv if H is None else H
+    shp = _shape(B, n, n, H, Hkv, pos0)
+    _check("rtp_local_ring_write", lib().rtp_local_ring_write(
+        ctypes.byref(shp), _role(kv_role), window, n_sink, view(k), view(v), view(k_ring),
+        view(v_ring), _stream(stream)))
+
+
+def rtp_local_attn_decode_ring(q, k_ring, v_ring, kv_role, *, window, n_sink, pos, scale=None,
+                               o=None, lse=None, stream=None):
+    """Local heads of one decode token at position `pos` from the ring cache."""
+    B, Lq, H, _ = q.shape
+    Hkv = len(kv_role)
+    if o is None:
+        o = torch.zeros_like(q)
+    if lse is None:
+        lse = torch.full((B, H, 1), float("nan"), dtype=torch.float32, device=q.device)
+    scale = 1.0 / (128 ** 0.5) if scale is None else scale
+    shp = _shape(B, 1, pos + 1, H, Hkv, pos)
+    role = _role(kv_role)
+    ws = workspace(OP_LOCAL, shp, role, 0, q.device, stream)
+    _check("rtp_local_attn_decode_ring", lib().rtp_local_attn_decode_ring(
+        ctypes.byref(shp), role, window, n_sink, view(q), view(k_ring), view(v_ring),
         ctypes.c_float(scale), view(o), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return o, lse
 

@@ -95,12 +95,16 @@ WORKLOADS = {
 }
 
 
-def _rope_(x: torch.Tensor, pos0: int) -> None:
-    """In-place RoPE on x [n, heads, 128] (fp32) for positions pos0 .. pos0+n-1."""
+def _rope_(x: torch.Tensor, pos0) -> None:
+    """In-place RoPE on x [n, heads, 128] (fp32) for positions pos0 .. pos0+n-1,
+    or for the n positions of a 1-D tensor `pos0`."""
     n = x.shape[0]
     c = torch.arange(D // 2, device=x.device, dtype=torch.float64)
     theta = ROPE_BASE ** (-2.0 * c / D)
-    pos = torch.arange(pos0, pos0 + n, device=x.device, dtype=torch.float64)
+    if isinstance(pos0, torch.Tensor):
+        pos = pos0.to(device=x.device, dtype=torch.float64)
+    else:
+        pos = torch.arange(pos0, pos0 + n, device=x.device, dtype=torch.float64)
     ang = pos[:, None] * theta[None, :]
     cos = torch.cos(ang).to(torch.float32)[:, None, :]
     sin = torch.sin(ang).to(torch.float32)[:, None, :]
@@ -132,13 +136,24 @@ def _needle_dirs(Wq: np.ndarray, Wk: np.ndarray):
     return np.stack(dirs), np.array(amps)
 
 
-def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None = None):
+def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None = None,
+                indexer_input: str = "post"):
     """Draw one workload's tensors.
 
     Returns a dict: q [B,Lq,H,128], k/v [B,Lk,Hkv,128], Wq16 [H_ret,128,16],
     Wk16 [H_ret,128,16] (all bf16 on ``device``), kv_role (numpy uint8 [Hkv]),
     and the ints Lq, Lk, q_pos0.
+
+    indexer_input="pre" also returns q_idx [B,Lq,H,128] and k_idx
+    [B,Lk,Hkv,128]: the same draws before RoPE (bf16), for an indexer that
+    projects pre-RoPE vectors as the summary's projection section describes.
+    The needles are then planted in those pre-RoPE vectors, and the planted rows
+    of q, k are the RoPE of the planted pre-RoPE rows, so the indexer sees the
+    +4 sigma uplift exactly and attention sees its rotated form.
     """
+    if indexer_input not in ("post", "pre"):
+        raise ValueError("indexer_input must be 'post' or 'pre'")
+    pre = indexer_input == "pre"
     L = w.L if L is None else L
     B = w.B if B is None else B
     dev = torch.device(device)
@@ -161,6 +176,8 @@ def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None =
     q = torch.empty(B, Lq, H, D, dtype=torch.bfloat16, device=dev)
     k = torch.empty(B, Lk, Hkv, D, dtype=torch.bfloat16, device=dev)
     v = torch.empty(B, Lk, Hkv, D, dtype=torch.bfloat16, device=dev)
+    q_idx = torch.empty_like(q) if pre else None
+    k_idx = torch.empty_like(k) if pre else None
 
     rng = np.random.default_rng(w.seed + 1000)
     Wq_np = Wq.float().cpu().numpy().astype(np.float64)
@@ -222,11 +239,15 @@ def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None =
                 tau = torch.exp(torch.empty(n, H, 1, device=dev).uniform_(
                     math.log(0.5), math.log(4.0), generator=gen))
                 x = x / tau
+            if pre:
+                q_idx[b, c0:c0 + n] = x.to(torch.bfloat16)
             _rope_(x, q_pos0 + c0)
             q[b, c0:c0 + n] = x.to(torch.bfloat16)
         for c0 in range(0, Lk, CHUNK):
             n = min(CHUNK, Lk - c0)
             x = randn(n, Hkv, D)
+            if pre:
+                k_idx[b, c0:c0 + n] = x.to(torch.bfloat16)
             _rope_(x, c0)
             k[b, c0:c0 + n] = x.to(torch.bfloat16)
             v[b, c0:c0 + n] = randn(n, Hkv, D).to(torch.bfloat16)
@@ -235,16 +256,31 @@ def make_inputs(w: Workload, device="cpu", L: int | None = None, B: int | None =
         ut = torch.tensor(u * amp[:, None], dtype=torch.float32, device=dev)
         for b, n, slot in key_adds:
             g = ret_heads[slot] // G
-            k[b, n, g] = (k[b, n, g].float() + ut[slot]).to(torch.bfloat16)
+            if pre:
+                k_idx[b, n, g] = (k_idx[b, n, g].float() + ut[slot]).to(torch.bfloat16)
+                y = k_idx[b, n:n + 1, g:g + 1].float()
+                _rope_(y, n)
+                k[b, n, g] = y[0, 0].to(torch.bfloat16)
+            else:
+                k[b, n, g] = (k[b, n, g].float() + ut[slot]).to(torch.bfloat16)
         for b, rows, slot in q_adds:
             if len(rows) == 0:
                 continue
             h = ret_heads[slot]
             ridx = torch.as_tensor(np.asarray(rows), device=dev, dtype=torch.long)
-            q[b, ridx, h] = (q[b, ridx, h].float() + ut[slot]).to(torch.bfloat16)
+            if pre:
+                q_idx[b, ridx, h] = (q_idx[b, ridx, h].float() + ut[slot]).to(torch.bfloat16)
+                y = q_idx[b, ridx, h].float()[:, None, :]
+                _rope_(y, ridx + q_pos0)
+                q[b, ridx, h] = y[:, 0].to(torch.bfloat16)
+            else:
+                q[b, ridx, h] = (q[b, ridx, h].float() + ut[slot]).to(torch.bfloat16)
 
-    return dict(q=q, k=k, v=v, Wq16=Wq, Wk16=Wk, kv_role=w.kv_role(),
-                Lq=Lq, Lk=Lk, q_pos0=q_pos0)
+    out = dict(q=q, k=k, v=v, Wq16=Wq, Wk16=Wk, kv_role=w.kv_role(),
+               Lq=Lq, Lk=Lk, q_pos0=q_pos0)
+    if pre:
+        out.update(q_idx=q_idx, k_idx=k_idx)
+    return out
 
 
 def bits(t: torch.Tensor) -> np.ndarray:

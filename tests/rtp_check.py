@@ -170,8 +170,20 @@ def check_row_outputs(o_gpu, o_ref, ref_ok, o_e2e, e2e_ok, what, max_skip=0.05):
     assert (~e2e_ok).sum() <= max(2, max_skip * n), (int((~e2e_ok).sum()), n)
     r1 = check_outputs(o_gpu[ref_ok], o_ref[ref_ok], what + " vs oracle on the GPU's kept sets")
     r2 = check_outputs(o_gpu[e2e_ok], o_e2e[e2e_ok], what + " vs oracle end to end")
-    return dict(skip_ref=int((~ref_ok).sum()), skip_e2e=int((~e2e_ok).sum()), max_abs=r1[0],
-                mean_abs=r1[1], e2e_max_abs=r2[0], e2e_mean_abs=r2[1])
+    stats = dict(rows=n, skip_ref=int((~ref_ok).sum()), skip_e2e=int((~e2e_ok).sum()),
+                 max_abs=r1[0], mean_abs=r1[1], e2e_max_abs=r2[0], e2e_mean_abs=r2[1])
+    report(what, stats)
+    return stats
+
+
+def report(what, stats):
+    """Append one JSON line of parity statistics to $RTP_PARITY_LOG (if set)."""
+    import json
+    import os
+    path = os.environ.get("RTP_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(what=what, **stats)) + "\n")
 
 
 def oracle_k16(k_bits, Wk_bits, w: synth.Workload, per_kv: bool = False):

@@ -37,7 +37,8 @@ def gpu_decode(inp, w, p, per_kv=False):
     if per_kv:
         Wk = Wk[[s for s in range(0, w.H_ret, w.G)]].contiguous()
     role = inp["kv_role"]
-    q16, k16 = rtp_index_scores(q, k, Wq, Wk, role, k16_per_kv_head=int(per_kv))
+    q16, k16 = rtp_index_scores(inp.get("q_idx", q), inp.get("k_idx", k), Wq, Wk, role,
+                                k16_per_kv_head=int(per_kv))
     o = torch.empty_like(q)
     lse = torch.empty(q.shape[0], w.H, 1, dtype=torch.float32, device=q.device)
     _, _, sel = rtp_sparse_attn_decode(q, k, v, q16, k16, role, p, k16_per_kv_head=int(per_kv),
@@ -48,13 +49,15 @@ def gpu_decode(inp, w, p, per_kv=False):
     return q16, k16, o, lse, sel, Wk
 
 
-def run_decode(w, L, B, p, per_kv=False, seed=None):
+def run_decode(w, L, B, p, per_kv=False, seed=None, indexer_input="post"):
     if seed is not None:
         w = w.with_(seed=seed)
-    inp = synth.make_inputs(w, "cuda", L=L, B=B)
+    inp = synth.make_inputs(w, "cuda", L=L, B=B, indexer_input=indexer_input)
     q16, k16, o, lse, sel, Wk = gpu_decode(inp, w, p, per_kv)
     p = float(np.float32(p))
     qb, kb, vb = bits(inp["q"]), bits(inp["k"]), bits(inp["v"])
+    qib = bits(inp["q_idx"]) if "q_idx" in inp else qb
+    kib = bits(inp["k_idx"]) if "k_idx" in inp else kb
     Wqb, Wkb = bits(inp["Wq16"]), bits(Wk)
     q16g, k16g = bits(q16), bits(k16)
     sel = {key: val.cpu().numpy() for key, val in sel.items()}
@@ -83,8 +86,8 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
     q16o = np.zeros_like(q16g)
     for b in range(B):
         for s, h in enumerate(ret):
-            q16o[b, 0, s] = oracle.project(qb[b, 0, h][None], Wqb[s])[0][0]
-    k16o = oracle_k16(kb, Wkb, w, per_kv)
+            q16o[b, 0, s] = oracle.project(qib[b, 0, h][None], Wqb[s])[0][0]
+    k16o = oracle_k16(kib, Wkb, w, per_kv)
     r3 = oracle.retrieval_rows(qb, kb, vb, q16o, k16o, rows, slots, ks, H=w.H, Hkv=w.Hkv,
                                q_pos0=P, p=p, scale=SCALE, want_sel=True)
     og = np.stack([o[b, 0, h] for (b, _, h) in rows])
@@ -98,7 +101,8 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
         lse_ref.append(l_)
         ref_ok.append(ok)
         e2e_ok.append(ok2)
-    check_row_outputs(og, np.stack(o_ref), ref_ok, r3["o"], e2e_ok, "retrieval decode")
+    stats = check_row_outputs(og, np.stack(o_ref), ref_ok, r3["o"], e2e_ok,
+                              f"retrieval decode L={L} B={B} p={p}")
     lg = np.array([lse[b, h, 0] for (b, _, h) in rows])
     assert np.abs(lg - np.array(lse_ref))[np.array(ref_ok)].max(initial=0.0) <= LSE_ABS
     if loc:
@@ -107,7 +111,7 @@ def run_decode(w, L, B, p, per_kv=False, seed=None):
                                n_sink=w.n_sink, scale=SCALE)
         check_outputs(np.stack([o[b, 0, h] for (b, _, h) in lrows]), rl["o"], "local decode")
         assert np.abs(np.array([lse[b, h, 0] for (b, _, h) in lrows]) - rl["lse"]).max() <= LSE_ABS
-    return n_band
+    return dict(n_band=n_band, stats=stats)
 
 
 @pytest.mark.parametrize("L", [1, 5, 1023, 1025, 4100, 8192])
@@ -120,6 +124,12 @@ def test_decode_per_kv_k16():
     run_decode(W["decode_128k_b8"], 6000, 2, 0.95, per_kv=True)
 
 
+def test_decode_pre_rope_indexer():
+    """The indexer projects the pre-RoPE q, k (the summary's projection input)
+    while attention uses the post-RoPE ones; the oracle takes the same split."""
+    run_decode(W["decode_128k_b8"], 6000, 2, 0.95, indexer_input="pre")
+
+
 @pytest.mark.parametrize("H", [4, 8, 16, 64])
 @pytest.mark.parametrize("per_kv", [False, True])
 def test_decode_head_groups(H, per_kv):
@@ -128,8 +138,10 @@ def test_decode_head_groups(H, per_kv):
 
 
 def test_decode_128k_batch8_full():
-    """The full 128K x batch-8 decode workload: every row of every head."""
-    run_decode(W["decode_128k_b8"], 131072, 8, 0.95)
+    """The full 128K x batch-8 decode workload: every row of every head, and at
+    most one of its 64 retrieval rows left out of either output check."""
+    st = run_decode(W["decode_128k_b8"], 131072, 8, 0.95)["stats"]
+    assert st["skip_ref"] <= 1 and st["skip_e2e"] <= 1, st
 
 
 def test_decode_equals_last_prefill_row():
@@ -145,13 +157,14 @@ def test_decode_equals_last_prefill_row():
                            p=0.9, window=w.window, n_sink=w.n_sink)
     torch.cuda.synchronize()
     assert torch.equal(k16_cache, pre["k16"])
-    # decode scores with fp32 FMAs, prefill on the tensor cores: the cut may move by
-    # an ulp of the score, never by more than one key
-    torch.testing.assert_close(dec["sel"]["thr"], pre["sel"]["thr"][:, :, L - 1], rtol=2e-6,
-                               atol=2e-6)
-    dc = dec["sel"]["count"].long()
-    pc = pre["sel"]["count"][:, :, L - 1].long()
-    assert (dc - pc).abs().max() <= 1
+    # both phases score a key by one 16-term tensor-core dot product of the same
+    # bf16 q16 and k16 with fp32 accumulation (decode's other slots add exact
+    # zeros), so they see identical scores; each sums fixed-point masses on its
+    # own bin grid, which agree to ~1e-6 relative, so the cut could move only
+    # for a row whose cumulative mass passes p * Z within that margin (none of
+    # these rows): the same row gets the same threshold, tie index and count
+    for key in ("thr", "jtie", "count"):
+        assert torch.equal(dec["sel"][key], pre["sel"][key][:, :, L - 1]), key
     torch.testing.assert_close(dec["o"][:, 0].float(), pre["o"][:, L - 1].float(), atol=2e-2,
                                rtol=0)
 

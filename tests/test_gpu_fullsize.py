@@ -1,7 +1,10 @@
 """GPU parity at the workloads' full sizes, on sampled query rows (the oracle
 computes those rows one by one): 32K with the p sweep, 128K multi-hop, 1M.
 Sampled rows always include the first and last rows and the rows around the
-local window's edge."""
+local window's edge.  At these sizes at most 2 of the 200-464 sampled
+retrieval rows may be left out of either output check (see
+rtp_check.check_row_outputs for why a row can be; the runs so far left out 0
+or 1)."""
 import numpy as np
 import pytest
 import torch
@@ -19,6 +22,12 @@ def _cuda():
         pytest.skip("needs a CUDA device")
 
 
+def bounded_skips(res):
+    st = res["stats"]
+    lim = 2
+    assert st["skip_ref"] <= lim and st["skip_e2e"] <= lim, st
+
+
 def sample_rows(L, window, n_sink, n_random, seed):
     rng = np.random.default_rng(seed)
     edge = [window - 1, window, window + 1, window + n_sink - 1, window + n_sink,
@@ -30,17 +39,19 @@ def sample_rows(L, window, n_sink, n_random, seed):
 @pytest.mark.parametrize("p", [0.8, 0.9, 0.95, 0.99])
 def test_prefill_32k_p_sweep(p):
     w = W["prefill_32k"]
-    run_prefill(w, w.L, p, positions=sample_rows(w.L, w.window, w.n_sink, 12, 30),
-                check_proj=False)
+    bounded_skips(run_prefill(w, w.L, p, positions=sample_rows(w.L, w.window, w.n_sink, 12, 30),
+                              check_proj=False))
 
 
 def test_prefill_128k_multihop():
     w = W["prefill_128k"]
-    run_prefill(w, w.L, w.p, positions=sample_rows(w.L, w.window, w.n_sink, 16, 31),
-                check_proj=False)
+    bounded_skips(run_prefill(w, w.L, w.p,
+                              positions=sample_rows(w.L, w.window, w.n_sink, 16, 31),
+                              check_proj=False))
 
 
 def test_prefill_1m():
     w = W["prefill_1m"]
-    run_prefill(w, w.L, w.p, positions=sample_rows(w.L, w.window, w.n_sink, 8, 32),
-                check_proj=False)
+    bounded_skips(run_prefill(w, w.L, w.p,
+                              positions=sample_rows(w.L, w.window, w.n_sink, 8, 32),
+                              check_proj=False))

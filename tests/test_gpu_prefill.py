@@ -51,17 +51,22 @@ def check_projection(gpu_bits, x_bits_rows, W_bits):
     return diff[0].size
 
 
-def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, seed=None):
+def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, seed=None,
+                indexer_input="post"):
+    """indexer_input="pre": the indexer projects the pre-RoPE draws (q_idx, k_idx)
+    while attention runs on the post-RoPE q, k; the oracle follows the same split."""
     if seed is not None:
         w = w.with_(seed=seed)
-    inp = synth.make_inputs(w, "cuda", L=L, B=B)
+    inp = synth.make_inputs(w, "cuda", L=L, B=B, indexer_input=indexer_input)
     q, k, v = inp["q"], inp["k"], inp["v"]
+    qi, ki = inp.get("q_idx", q), inp.get("k_idx", k)
     Wq, Wk = inp["Wq16"], inp["Wk16"]
     if per_kv:  # one indexer key per retrieval kv head: the first query head's W_k16
         Wk = Wk[[s for s in range(0, w.H_ret, w.G)]].contiguous()
     role = inp["kv_role"]
     res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=p, window=w.window, n_sink=w.n_sink,
-                            k16_per_kv_head=int(per_kv))
+                            k16_per_kv_head=int(per_kv), q_idx=inp.get("q_idx"),
+                            k_idx=inp.get("k_idx"))
     torch.cuda.synchronize()
     if positions is None:
         positions = np.arange(L)
@@ -69,8 +74,10 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     # only the sampled query rows travel to the host
     pidx = torch.as_tensor(positions, device=q.device)
     kb, vb = bits(k), bits(v)
+    kib = kb if ki is k else bits(ki)
     Wqb, Wkb = bits(Wq), bits(Wk)
     qs, q16s = bits(q[:, pidx]), bits(res["q16"][:, pidx])
+    qis = qs if qi is q else bits(qi[:, pidx])
     k16g = bits(res["k16"])
     sel = {key: val[:, :, pidx].cpu().numpy() for key, val in res["sel"].items()}
     o = res["o"][:, pidx].float().cpu().numpy()
@@ -83,11 +90,11 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
     if check_proj:
         for b in range(B):
             for s, h in enumerate(ret):
-                check_projection(q16s[b, :, s], qs[b, :, h], Wqb[s])
+                check_projection(q16s[b, :, s], qis[b, :, h], Wqb[s])
             for s in sorted(set(k16slot)):
                 g = ret[s * (w.G if per_kv else 1)] // w.G
-                check_projection(k16g[b, :, s], kb[b, :, g], Wkb[s])
-    k16o = oracle_k16(kb, Wkb, w, per_kv)
+                check_projection(k16g[b, :, s], kib[b, :, g], Wkb[s])
+    k16o = oracle_k16(kib, Wkb, w, per_kv)
 
     n_band, o_ret_g, o_ret_a, o_ret_o, o_loc_g, o_loc_o = 0, [], [], [], [], []
     ref_ok, e2e_ok = [], []
@@ -102,7 +109,7 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
                                        np.array(k16slot), H=w.H, Hkv=w.Hkv, q_pos0=int(i), p=p,
                                        scale=SCALE, want_sel=True)
             # (iii) end to end with the oracle's own projections
-            q16o = np.stack([oracle.project(qs[b, x, h][None], Wqb[s])[0][0]
+            q16o = np.stack([oracle.project(qis[b, x, h][None], Wqb[s])[0][0]
                              for s, h in enumerate(ret)])[None, None]
             r3 = oracle.retrieval_rows(q1, kb1, vb1, q16o, k16o[b:b + 1], rows,
                                        np.arange(len(ret)), np.array(k16slot), H=w.H, Hkv=w.Hkv,
@@ -134,7 +141,8 @@ def run_prefill(w, L, p, B=1, positions=None, per_kv=False, check_proj=True, see
                 o_loc_g.append(o[b, x, loc])
                 lse_err = max(lse_err, float(np.abs(lse[b, loc, x] - rl["lse"]).max()))
     stats = check_row_outputs(np.concatenate(o_ret_g), np.stack(o_ret_a), ref_ok,
-                              np.concatenate(o_ret_o), e2e_ok, "retrieval heads")
+                              np.concatenate(o_ret_o), e2e_ok,
+                              f"retrieval prefill {w.name} L={L} B={B} p={p}")
     if loc:
         check_outputs(np.concatenate(o_loc_g), np.concatenate(o_loc_o), "local heads")
     assert lse_err <= LSE_ABS, lse_err

@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=3)
+    ap.add_argument("--no-1m", action="store_true", help="skip the 1M prefill workload")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the block top-p / top-k / ring-cache decode lines")
     ap.add_argument("--case", default=None, choices=["decode", "select", "prefill", "dense"],
                     help="run one small case twice and exit (for profilers)")
     ap.add_argument("--L", type=int, default=16384, help="sequence length for --case")
@@ -222,6 +225,21 @@ def trace_read():
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(max(n, 0))}
 
 
+def trace_timeline():
+    """(name, start us, end us) of each launch recorded since the last reset."""
+    from long_context_sparse_rtp_b200 import rtp
+
+    class Launch(ctypes.Structure):
+        _fields_ = [("name", ctypes.c_char * 48), ("start_ms", ctypes.c_double),
+                    ("end_ms", ctypes.c_double)]
+    L = rtp.lib()
+    L.rtp_trace_timeline.restype = ctypes.c_int
+    arr = (Launch * 256)()
+    n = L.rtp_trace_timeline(arr, 256)
+    return [(arr[i].name.decode(), round(arr[i].start_ms * 1e3, 2), round(arr[i].end_ms * 1e3, 2))
+            for i in range(max(n, 0))]
+
+
 def trace(on: bool):
     from long_context_sparse_rtp_b200 import rtp
     rtp.lib().rtp_trace_reset()
@@ -354,6 +372,7 @@ def bench_decode(args, world, rank, local, pk):
         for name, (n, t) in trace_read().items():
             a0, a1 = kern.get(name, (0, 0.0))
             kern[name] = (a0 + n, a1 + t)
+    timeline = trace_timeline()  # the last replay: each launch's start and end
     trace(False)
     res = decode_step(st, None, None)
     torch.cuda.synchronize()
@@ -363,7 +382,8 @@ def bench_decode(args, world, rank, local, pk):
     B = st["q"].shape[0]
     nbytes = decode_bytes(st, union)
     return dict(st=st, ms_step=ms_step, clocks=clk, kern=kern, union=union,
-                compute_sel=compute_sel, bytes=nbytes, B=B, flush=flush, graph=g)
+                compute_sel=compute_sel, bytes=nbytes, B=B, flush=flush, graph=g,
+                timeline=timeline)
 
 
 def bench_decode_e2e(dec, args, world):
@@ -424,43 +444,296 @@ def bench_decode_dense(dec, args):
     return dict(ms_step=ms / args.steps, bytes=k.shape[0] * L * k.shape[2] * 128 * 2 * 2)
 
 
-# ------------------------------------------------------------------ prefill (ours)
-def bench_prefill(args, world, rank, pk):
+def _keep_mask(scores, thr, jtie):
     import torch
-    from long_context_sparse_rtp_b200 import rtp_layer_prefill, synth
-    w = synth.WORKLOADS[PREFILL_WL]
+    j = torch.arange(scores.shape[-1], device=scores.device)
+    t, jt = thr[..., None], jtie[..., None]
+    return (scores > t) | ((scores == t) & (j <= jt))
+
+
+def bench_decode_variants(dec, args, world):
+    """The same decode step with block-level top-p and with static top-k
+    (k = 4096) on the retrieval heads (graph replay), and their recall of the
+    exact top-p kept keys: the share of those keys, and of the indexer softmax
+    mass, that each keeps."""
+    import torch
+    from long_context_sparse_rtp_b200 import (DecodeGraph, rtp_index_scores,
+                                              rtp_sparse_attn_decode_select)
+    st = dec["st"]
+    w, L = st["w"], st["L"]
+    out = {}
+    for select in ("block_topp", "topk"):
+        g = DecodeGraph(st["k"], st["v"], st["k16"], st["Wq"], st["Wk"], st["role"], H=w.H,
+                        pos=L - 1, p=w.p, window=w.window, n_sink=w.n_sink, select=select,
+                        top_k=4096)
+        g.q.copy_(st["q"])
+        ms, _ = time_steps(g.replay, args.steps, args.warmup, world, dec["flush"])
+        ms = max_over_ranks(ms, world) / args.steps
+        out[select] = {"ms_per_step": ms, "tokens_per_s": st["q"].shape[0] * world / (ms / 1e3)}
+        del g
+    q16, _ = rtp_index_scores(st["q"], None, st["Wq"], st["Wk"], st["role"], H=w.H)
+    args_ = (st["q"], st["k"], st["v"], q16, st["k16"], st["role"])
+    _, _, ex = rtp_sparse_attn_decode_select(*args_, "topp", p=w.p, want_scores=True)
+    _, _, bl = rtp_sparse_attn_decode_select(*args_, "block_topp", p=w.p)
+    _, _, tk = rtp_sparse_attn_decode_select(*args_, "topk", top_k=4096)
+    s = ex["scores"]
+    exact = _keep_mask(s, ex["thr"], ex["jtie"])
+    masks = {"topk": _keep_mask(s, tk["thr"], tk["jtie"])}
+    wb = bl["block_mask"].to(torch.int64) & 0xFFFFFFFF
+    blk = ((wb[..., :, None] >> torch.arange(32, device=s.device)) & 1).flatten(-2)
+    masks["block_topp"] = blk[..., torch.arange(s.shape[-1], device=s.device) // 64].bool()
+    wgt = torch.exp(s - s.max(dim=-1, keepdim=True).values)
+    for name, m in masks.items():
+        out[name].update({
+            "mean_keys": float(m.sum(-1).float().mean()),
+            "token_recall_of_exact_topp": float((m & exact).sum() / exact.sum()),
+            "indexer_mass_kept": float(((wgt * m).sum(-1) / wgt.sum(-1)).mean())})
+    out["exact_topp_mean_keys"] = float(exact.sum(-1).float().mean())
+    del s, ex, bl, tk, exact, masks, wgt
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_decode_ring(dec, args, world):
+    """The same decode step with the local heads on the window-only ring cache
+    (written from the cache's first L - 1 positions; each step appends its token)."""
+    import torch
+    from long_context_sparse_rtp_b200 import DecodeGraph, local_ring_alloc, rtp_local_ring_write
+    st = dec["st"]
+    w, L = st["w"], st["L"]
+    B = st["q"].shape[0]
+    kr, vr = local_ring_alloc(B, st["role"], window=w.window, n_sink=w.n_sink, device="cuda")
+    rtp_local_ring_write(st["k"][:, :L - 1], st["v"][:, :L - 1], kr, vr, st["role"],
+                         window=w.window, n_sink=w.n_sink, pos0=0, H=w.H)
+    g = DecodeGraph(st["k"], st["v"], st["k16"], st["Wq"], st["Wk"], st["role"], H=w.H,
+                    pos=L - 1, p=w.p, window=w.window, n_sink=w.n_sink, local_ring=(kr, vr))
+    g.q.copy_(st["q"])
+    ms, _ = time_steps(g.replay, args.steps, args.warmup, world, dec["flush"])
+    ms = max_over_ranks(ms, world) / args.steps
+    n_lkv = int(sum(1 for x in st["role"] if int(x) == 0))
+    ring_bytes = (kr.numel() + vr.numel()) * 2
+    full_bytes = B * L * n_lkv * 128 * 2 * 2
+    del g, kr, vr
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": B * world / (ms / 1e3),
+            "local_kv_bytes_ring": ring_bytes, "local_kv_bytes_full_cache": full_bytes}
+
+
+# ------------------------------------------------------------------ prefill (ours)
+PREFILL_SET = ("prefill_2k", "prefill_32k", "prefill_128k", "prefill_1m")
+PREFILL_DESC = {
+    "prefill_2k": "causal prefill 1 x 2048, 8 q / 2 kv, kv0 retrieval, window 256+4, p=0.9, "
+                  "8 needles per retrieval head",
+    "prefill_32k": "causal prefill 1 x 32768, 32 q / 4 kv, kv0-1 retrieval, window 2048+4, "
+                   "per-query temperature, p swept",
+    "prefill_128k": "causal prefill 1 x 131072, 32 q / 4 kv, kv0 retrieval, window 4096+4, "
+                    "p=0.95, 4-key needle chains",
+    "prefill_1m": "causal prefill 1 x 1048576, 32 q / 4 kv, kv0 retrieval, window 4096+4, "
+                  "p=0.95, needles per 4096-row group",
+}
+ATTN_FLOP_PER_PAIR = 4 * 128  # QK^T and PV: 2 x 2 x 128 per (query row, key)
+
+
+def tile_pairs(L, window=None, n_sink=0):
+    """(query row, key) pairs the 128 x 128 tile schedule of attn_tc computes per
+    head: every causal tile (dense, sparse) or the sink and window tiles (local)."""
+    import numpy as np
+    nb = (L + 127) // 128
+    rb = np.arange(nb, dtype=np.int64)
+    P0 = rb * 128
+    t_end = (np.minimum(L, P0 + 128) - 1) // 128
+    if window is None:
+        n = t_end + 1
+    else:
+        sink_end = np.full(nb, (n_sink + 127) // 128)
+        win_begin = np.maximum(np.maximum(P0 - window + 1, 0) // 128, sink_end)
+        sink_end = np.minimum(sink_end, t_end + 1)
+        n = sink_end + np.maximum(0, t_end - win_begin + 1)
+    return int(n.sum()) * 128 * 128
+
+
+def local_pairs(L, window, n_sink):
+    """Pairs of the sink + window rule per local head: sum over P of min(P + 1, n_sink + window)."""
+    c = window + n_sink
+    if L <= c:
+        return L * (L + 1) // 2
+    return c * (c + 1) // 2 + (L - c) * c
+
+
+def measure_ex2_rate():
+    """Sustained ex2.approx.f32 rate of the device (per second), from the
+    library's probe kernel timed with CUDA events (best of 5 after a warm-up)."""
+    import torch
+    from long_context_sparse_rtp_b200.rtp import rtp_probe_ex2
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    blocks, iters = n_sm * 8, 4096
+    out = torch.empty(blocks * 256, dtype=torch.float32, device="cuda")
+    rtp_probe_ex2(blocks, iters, out)
+    best = None
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        rtp_probe_ex2(blocks, iters, out)
+        b.record()
+        b.synchronize()
+        t = a.elapsed_time(b) / 1e3
+        best = t if best is None else min(best, t)
+    return blocks * 256 * iters * 8 / best
+
+
+def bench_prefill_config(name, args, world, rank, pk, ex2_rate, cpu=False):
+    """One prefill workload: the whole layer (index, select, sparse, local) per p,
+    the dense kernel and the summary's own prefill (retrieval heads dense) at
+    the same L, per-kernel times and rooflines."""
+    import torch
+    from long_context_sparse_rtp_b200 import rtp_check_device, rtp_dense_attn, rtp_layer_prefill
+    from long_context_sparse_rtp_b200 import synth
+    w = synth.WORKLOADS[name]
     w = w.with_(seed=rank_seed(w.seed, rank))
     inp = synth.make_inputs(w, "cuda")
     q, k, v, Wq, Wk, role = (inp[x] for x in ("q", "k", "v", "Wq16", "Wk16", "kv_role"))
-    flush = make_l2_flush()
-
-    def step():
-        rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
-
-    steps = args.prefill_steps
-    ms, kern = time_steps(step, steps, 1, world, flush, traced=True)
-    ms = max_over_ranks(ms, world)
-    res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p, window=w.window, n_sink=w.n_sink)
-    torch.cuda.synchronize()
-    from long_context_sparse_rtp_b200 import rtp_check_device
-    rtp_check_device()
-    cnt = res["sel"]["count"].double()
     L = q.shape[1]
-    sel_pairs = float(cnt.sum())
-    causal_pairs = w.H_ret * L * (L + 1) / 2
-    loc_heads = w.H - w.H_ret
-    loc_pairs = loc_heads * sum(min(i + 1, w.window + w.n_sink) for i in range(0, L, 1)) \
-        if L <= 1 << 16 else loc_heads * (L * (w.window + w.n_sink) - (w.window + w.n_sink) ** 2 / 2)
-    ms_step = ms / steps
-    per = {k_: dict(launches=n // steps, ms=t / steps) for k_, (n, t) in kern.items()}
-    # dense baseline at the same L (one run, for the ratio)
-    from long_context_sparse_rtp_b200 import rtp_dense_attn
+    big = L >= (1 << 20)
+    steps = 1 if big else args.prefill_steps
+    warm = 0 if big else 1  # a 1M layer runs for seconds; the kernels are loaded already
+    flush = make_l2_flush()
+    peak = pk["bf16_sus"] if big else pk["bf16"]
+    peak_kind = "sustained" if big else "burst"
+    causal = L * (L + 1) / 2
+    dense_tiles = tile_pairs(L)
+    loc_tiles = tile_pairs(L, w.window, w.n_sink)
+    H_loc = w.H - w.H_ret
+    out = {"workload": f"{name}: {PREFILL_DESC[name]}", "L": L, "steps": steps,
+           "peak_kind": peak_kind}
+
+    def tensor(kernel_ms, method_pairs, computed_pairs):
+        t = kernel_ms / 1e3
+        fm = method_pairs * ATTN_FLOP_PER_PAIR / t / 1e12
+        ft = computed_pairs * ATTN_FLOP_PER_PAIR / t / 1e12
+        return {"ms": kernel_ms, "tflops_method_pairs": fm, "frac_method_pairs": fm / peak,
+                "tflops_computed_tiles": ft, "frac_computed_tiles": ft / peak}
+
+    runs = []
+    for p in (w.p_sweep or (w.p,)):
+        def step(p=p):
+            rtp_layer_prefill(q, k, v, Wq, Wk, role, p=p, window=w.window, n_sink=w.n_sink)
+        ms, kern = time_steps(step, steps, warm, world, flush, traced=True)
+        ms = max_over_ranks(ms, world) / steps
+        per = {k_: t / n for k_, (n, t) in kern.items()}
+        res = rtp_layer_prefill(q, k, v, Wq, Wk, role, p=p, window=w.window, n_sink=w.n_sink)
+        torch.cuda.synchronize()
+        rtp_check_device()
+        kept = float(res["sel"]["count"].double().sum())
+        del res
+        r = {"p": p, "ms": ms, "tokens_per_s": L * world / (ms / 1e3), "per_kernel_ms": per,
+             "kept_pairs": kept, "kept_share": kept / (w.H_ret * causal)}
+        roof = {}
+        if "attn_prefill_sparse" in per:
+            roof["attn_prefill_sparse"] = tensor(per["attn_prefill_sparse"], kept,
+                                                 w.H_ret * dense_tiles)
+        if "attn_prefill_local" in per:
+            roof["attn_prefill_local"] = tensor(per["attn_prefill_local"],
+                                                H_loc * local_pairs(L, w.window, w.n_sink),
+                                                H_loc * loc_tiles)
+        if "topp_select" in per:
+            t = per["topp_select"] / 1e3
+            exp_ms = w.H_ret * causal / ex2_rate * 1e3
+            roof["topp_select"] = {
+                "ms": per["topp_select"], "bound": "alu (one exp per causal pair at least)",
+                "exp_bound_ms": exp_ms, "frac_of_exp_bound": exp_ms / per["topp_select"],
+                "tensor_frac_3_sweeps": 3 * 32 * w.H_ret * dense_tiles / t / 1e12 / peak}
+        r["roofline"] = roof
+        runs.append(r)
+    out["runs"] = runs
+    # the dense kernel on every head at the same L
     o = torch.empty_like(q)
-    dms, dkern = time_steps(lambda: rtp_dense_attn(q, k, v, o=o), 1, 1, world, flush,
-                            traced=True)
-    return dict(ms_step=ms_step, tokens_per_s=L / (ms_step / 1e3) * world, L=L, per_kernel=per,
-                sel_pairs=sel_pairs, causal_pairs=causal_pairs, loc_pairs=loc_pairs,
-                dense_ms=dms, w=w)
+    dms, _ = time_steps(lambda: rtp_dense_attn(q, k, v, o=o), 1, warm, world, flush)
+    dms = max_over_ranks(dms, world)
+    out["dense"] = {"ms": dms, "tokens_per_s": L / (dms / 1e3),
+                    **{k_: v_ for k_, v_ in tensor(dms, w.H * causal, w.H * dense_tiles).items()
+                       if k_ != "ms"}}
+    for r in runs:
+        r["speedup_vs_dense"] = dms / r["ms"]
+    # the summary's own prefill: retrieval heads dense (with the k16 projection
+    # the decode steps need), local heads sink + window
+    pms, pk_ = time_steps(lambda: rtp_layer_prefill(q, k, v, Wq, Wk, role, p=w.p,
+                                                    window=w.window, n_sink=w.n_sink,
+                                                    retrieval="dense"),
+                          1, warm, world, flush, traced=True)
+    pms = max_over_ranks(pms, world)
+    out["pages_mode"] = {
+        "what": "retrieval heads dense, local heads sink + window (the summary's prefill)",
+        "ms": pms, "tokens_per_s": L / (pms / 1e3), "speedup_vs_dense": dms / pms,
+        "per_kernel_ms": {k_: t / n for k_, (n, t) in pk_.items()}}
+    if cpu:
+        try:
+            out["cpu_baseline"] = oracle_prefill_baseline(w, inp)
+        except Exception as e:  # report, never hide
+            out["cpu_baseline"] = {"error": repr(e)}
+    del o, inp, q, k, v
+    torch.cuda.empty_cache()
+    return out, w
+
+
+def oracle_prefill_baseline(w, inp, n_pos=4):
+    """The oracle on a seeded sample of one prefill workload, extrapolated to the
+    whole layer: the k16 projection timed on up to 16384 key rows and scaled to
+    every key and k16 slot; retrieval rows (full sort per row) at n_pos
+    positions fitted to c * P * log2(P); local rows at n_pos positions fitted to
+    c' * min(P + 1, window + n_sink); q16 projections scaled per row."""
+    import numpy as np
+    import oracle
+    from long_context_sparse_rtp_b200 import synth
+    L = inp["q"].shape[1]
+    ret, loc = w.retrieval_q_heads(), w.local_q_heads()
+    rng = np.random.default_rng(77)
+    pos = sorted(set([L - 1] + [int(x) for x in rng.integers(L // 4, L, n_pos - 1)]))
+    pidx = __import__("torch").as_tensor(pos, device="cuda")
+    qb = synth.bits(inp["q"][:, pidx])
+    kb, vb = synth.bits(inp["k"]), synth.bits(inp["v"])
+    Wqb, Wkb = synth.bits(inp["Wq16"]), synth.bits(inp["Wk16"])
+    scale = 1.0 / math.sqrt(128)
+    nproj = min(L, 16384)
+    t0 = time.perf_counter()
+    oracle.project(kb[0, :nproj, ret[0] // w.G], Wkb[0])
+    t_proj_row = (time.perf_counter() - t0) / nproj
+    k16 = np.empty((1, L, len(ret), 16), np.uint16)
+    t_k16 = 0.0
+    for s, h in enumerate(ret):
+        t0 = time.perf_counter()
+        k16[0, :, s] = oracle.project(kb[0, :, h // w.G], Wkb[s])[0]
+        t_k16 += time.perf_counter() - t0
+    c_ret, c_loc, sample_s = [], [], t_k16
+    for x, P in enumerate(pos):
+        q16 = np.stack([oracle.project(qb[0, x, h][None], Wqb[s])[0][0]
+                        for s, h in enumerate(ret)])[None, None]
+        rows = np.array([(0, 0, h) for h in ret])
+        t0 = time.perf_counter()
+        oracle.retrieval_rows(qb[:, x:x + 1], kb, vb, q16, k16, rows, np.arange(len(ret)),
+                              np.arange(len(ret)), H=w.H, Hkv=w.Hkv, q_pos0=P,
+                              p=float(np.float32(w.p)), scale=scale)
+        dt = time.perf_counter() - t0
+        sample_s += dt
+        c_ret.append(dt / len(ret) / ((P + 1) * math.log2(P + 2)))
+        lrows = np.array([(0, 0, h) for h in loc])
+        t0 = time.perf_counter()
+        oracle.local_rows(qb[:, x:x + 1], kb, vb, lrows, H=w.H, Hkv=w.Hkv, q_pos0=P,
+                          window=w.window, n_sink=w.n_sink, scale=scale)
+        dt = time.perf_counter() - t0
+        sample_s += dt
+        c_loc.append(dt / len(loc) / min(P + 1, w.window + w.n_sink))
+    Pv = np.arange(L, dtype=np.float64)
+    t_ret = float(np.mean(c_ret)) * len(ret) * float(((Pv + 1) * np.log2(Pv + 2)).sum())
+    t_loc = float(np.mean(c_loc)) * len(loc) * float(np.minimum(Pv + 1,
+                                                                w.window + w.n_sink).sum())
+    t_q16 = t_proj_row * L * len(ret)
+    total = t_k16 + t_q16 + t_ret + t_loc
+    return {"value": L / total, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "extrapolated": True, "sample_cpu_s": sample_s,
+            "sample": f"{w.name}: k16 projection of all {L} keys x {len(ret)} slots timed; "
+                      f"retrieval and local rows timed at positions {pos}, extrapolated to "
+                      f"all {L} rows by c*P*log2(P) (retrieval) and c*min(P+1, W+S) (local)",
+            "extrapolated_total_s": total}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -569,7 +842,19 @@ def main():
     dec = bench_decode(args, world, rank, local, pk)
     e2e_ms, h2d, d2h = bench_decode_e2e(dec, args, world)
     shared = bench_decode_shared_k16(dec, args, world)
-    pre = None if args.no_prefill else bench_prefill(args, world, rank, pk)
+    variants = ring = None
+    if not args.no_variants:
+        variants = bench_decode_variants(dec, args, world)
+        ring = bench_decode_ring(dec, args, world)
+    pres, ex2 = {}, None
+    if not args.no_prefill:
+        ex2 = measure_ex2_rate()
+        for name in PREFILL_SET:
+            if name == "prefill_1m" and args.no_1m:
+                continue
+            pres[name], _ = bench_prefill_config(
+                name, args, world, rank, pk, ex2,
+                cpu=(rank == 0 and world == 1 and not args.no_cpu_baseline))
     dense = None
     if world == 1:  # a reported baseline: no collective, so one rank only
         try:
@@ -605,6 +890,7 @@ def main():
                           "achieved": step_gbs, "frac": step_gbs / pk["hbm"],
                           "frac_of_8tbs": step_gbs / 8000.0},
         "per_kernel_ms": {k_: t / n for k_, (n, t) in kern.items()},
+        "timeline_us": dec["timeline"],
         "selection": {"union_keys": dec["union"], "kept_pairs": dec["compute_sel"]},
         "gpu_launches": n_launch * args.steps,
         "clocks": dec["clocks"],
@@ -617,16 +903,20 @@ def main():
         "workload": f"{DECODE_WL} with one k16 per retrieval kv head (k16_per_kv_head = 1)",
         "tokens_per_s": shared["tokens_per_s"], "ms_per_step": shared["ms_step"],
         "k16_bytes_per_step": shared["k16_bytes"]}
-    if pre is not None:
-        per = pre["per_kernel"]
+    if variants is not None:
+        line["decode_variants"] = {
+            "workload": f"{DECODE_WL} with block-level top-p (p = 0.95, 64-key blocks, 256 "
+                        "bins) or static top-k (k = 4096) on the retrieval heads", **variants}
+        line["decode_ring"] = {
+            "workload": f"{DECODE_WL} with the local heads on the window-only ring cache",
+            **ring}
+    if pres:
         line["prefill"] = {
-            "workload": f"{PREFILL_WL}: causal prefill 1 x 131072, 32 q / 4 kv, 1 retrieval kv "
-                        "head, p=0.95, window 4096+4, chained needles",
-            "tokens_per_s": pre["tokens_per_s"], "ms_per_step": pre["ms_step"],
-            "steps": args.prefill_steps, "per_kernel_ms": {k_: d["ms"] for k_, d in per.items()},
-            "dense_baseline_ms": pre["dense_ms"], "speedup_vs_dense": pre["dense_ms"] / pre["ms_step"],
-            "kept_pairs": pre["sel_pairs"], "causal_pairs": pre["causal_pairs"],
-        }
+            "ex2_rate_per_s": ex2,
+            "note": "per config: the whole mixed layer per p, the dense kernel on every head and "
+                    "the summary's own prefill (retrieval heads dense) at the same L; "
+                    "attention rooflines on the method's own pairs and on the computed tiles",
+            **pres}
     if dense is not None:
         line["dense_decode"] = dense if "error" in dense else {
             "workload": f"{DECODE_WL} with every query head dense over the whole cache "

@@ -338,10 +338,21 @@ typedef struct rtp_trace_entry {
     double total_ms;
 } rtp_trace_entry;
 
+/* One recorded launch: start and end, in ms after the start of the first
+ * launch recorded since the last rtp_trace_reset (as of its last completion). */
+typedef struct rtp_trace_launch {
+    char name[48];
+    double start_ms;
+    double end_ms;
+} rtp_trace_launch;
+
 RTP_API void rtp_trace_enable(int on);
 RTP_API void rtp_trace_reset(void);
 /* Fills up to max_entries entries; returns the number filled, or -1 on a CUDA error. */
 RTP_API int rtp_trace_read(rtp_trace_entry* out, int max_entries);
+/* The recorded launches in recording order (up to max_entries); returns the
+ * number filled, or -1 on a CUDA error. */
+RTP_API int rtp_trace_timeline(rtp_trace_launch* out, int max_entries);
 
 /*
  * Measurement aid (no counterpart in the paper): launches `blocks` CTAs of 256

@@ -118,6 +118,27 @@ extern "C" void rtp_trace_reset(void) {
   rtp::g_trace.clear();
 }
 
+extern "C" int rtp_trace_timeline(rtp_trace_launch* out, int max_entries) {
+  std::lock_guard<std::mutex> lk(rtp::g_trace_mu);
+  if (rtp::g_trace.empty()) return 0;
+  const cudaEvent_t t0 = rtp::g_trace.front().start;
+  int n = 0;
+  for (auto& r : rtp::g_trace) {
+    if (n >= max_entries) break;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return -1;
+    float a = 0.f, b = 0.f;
+    if (cudaEventElapsedTime(&a, t0, r.start) != cudaSuccess ||
+        cudaEventElapsedTime(&b, t0, r.stop) != cudaSuccess)
+      return -1;
+    memset(&out[n], 0, sizeof(out[n]));
+    strncpy(out[n].name, r.name.c_str(), sizeof(out[n].name) - 1);
+    out[n].start_ms = a;
+    out[n].end_ms = b;
+    ++n;
+  }
+  return n;
+}
+
 extern "C" int rtp_trace_read(rtp_trace_entry* out, int max_entries) {
   std::lock_guard<std::mutex> lk(rtp::g_trace_mu);
   int n = 0;

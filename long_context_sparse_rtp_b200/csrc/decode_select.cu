@@ -7,7 +7,8 @@
 // b = floor(4 s) and contributes exp(s - (b+1)/4) in (0.78, 1] to that bin, as
 // 21-bit fixed point.  Integer sums are exact and order-free, so every decision
 // below is deterministic.  Per kv group of G retrieval query heads:
-//   1. score     stream the k16 cache once (HBM-bound), s = q16 . k16 as one
+//   1. score     stream the k16 cache once (HBM-bound; loaded evict-first, so
+//                the score rows stay in L2 for steps 3-5), s = q16 . k16 as one
 //                16-term tensor-core dot product (tcgen05, fp32 in TMEM), scores
 //                kept in the workspace; each CTA bins its items' scores in shared
 //                memory (one 256-bin window per head, 32-bit atomics) and adds
@@ -26,6 +27,7 @@
 // are resolved by a radix refinement over the stored scores (slower, rare).
 #include <algorithm>
 
+#include "dec_bins.cuh"
 #include "rtp_host.h"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -40,17 +42,6 @@ constexpr int kThreads = 256;
 constexpr double kFix21 = 1.0 / 2097152.0;  // 2^-21
 constexpr int kWarpCap = 512;               // candidates one warp sorts on its own
 
-// Absolute score bin floor(s * kappa), rounding toward -inf.  kappa * s is
-// clamped to +-2^21 (far outside the histogram's range); adding 1.5 * 2^23 with
-// rounding toward -inf leaves floor(x) in the low mantissa bits, exactly, for
-// |x| < 2^22.  sbin_m returns that sum: the bin is bin_f / bin_i of it.
-__device__ __forceinline__ float sbin_m(float s) {
-  const float x = fminf(fmaxf(__fmul_rn(s, kDecKappa), -2097152.0f), 2097152.0f);
-  return __fadd_rd(x, 12582912.0f);
-}
-__device__ __forceinline__ float bin_f(float m) { return __fsub_rn(m, 12582912.0f); }
-__device__ __forceinline__ int bin_i(float m) { return __float_as_int(m) - 0x4B400000; }
-__device__ __forceinline__ int sbin(float s) { return bin_i(sbin_m(s)); }
 // 2^x for x <= 0 (no subnormal results matter here: x >= -0.37 in every use
 // that feeds a decision, and tiny results only need to stay tiny).
 __device__ __forceinline__ float ex2_ftz(float x) {
@@ -133,6 +124,8 @@ struct ScoreParams {
   int quad;          // 1: kw >= 4, the slots load as four-slot 128-byte-swizzled boxes
   int batch_coord;   // 1, or 0 when every batch entry shares one k16 cache
   int items_per_group, n_items;
+  float2* blk;       // block-stats mode: [rows][n_blk] (max, log-sum-exp) of 64-key blocks
+  int n_blk;         // (null: the histograms of the exact top-p instead)
 };
 
 struct ScoreSmemTail {
@@ -216,6 +209,9 @@ __global__ void __launch_bounds__(kSThreads, 2)
   const int it0 = (int)blockIdx.x * per_cta, it1 = min(it0 + per_cta, p.n_items);
 
   if (warp == kSProdWarp) {  // ---------------- producer (the whole warp)
+    // the k16 stream is read once: evict it first, so that the score rows this
+    // kernel writes stay in L2 for the kernels that read them back
+    const uint64_t pol = l2_policy_evict_first();
     int stage = 0, n_issued = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -250,12 +246,12 @@ __global__ void __launch_bounds__(kSThreads, 2)
           mbar_arrive_expect_tx(&tl->full[stage], (uint32_t)(kw * kSChunkA));
           if (p.quad) {  // four slots (128-byte rows) per box
             for (int qd = 0; qd < kw / 4; ++qd)
-              tma_load_4d(sb + qd * 4 * kSChunkA, &kmap, 0, slot0 / 4 + qd, j0 + st * kSTile,
-                          b * p.batch_coord, &tl->full[stage]);
+              tma_load_4d_hint(sb + qd * 4 * kSChunkA, &kmap, 0, slot0 / 4 + qd,
+                               j0 + st * kSTile, b * p.batch_coord, &tl->full[stage], pol);
           } else {
             for (int h = 0; h < kw; ++h)
-              tma_load_4d(sb + h * kSChunkA, &kmap, 0, slot0 + h, j0 + st * kSTile,
-                          b * p.batch_coord, &tl->full[stage]);
+              tma_load_4d_hint(sb + h * kSChunkA, &kmap, 0, slot0 + h, j0 + st * kSTile,
+                               b * p.batch_coord, &tl->full[stage], pol);
           }
         }
         ++n_issued;
@@ -362,6 +358,25 @@ __global__ void __launch_bounds__(kSThreads, 2)
     }
     sub_base += (uint32_t)nsub;
     named_bar(1, kSConsumers);
+    if (p.blk != nullptr) {  // block-level top-p: (max, log-sum-exp) per 64-key block and head
+      const int nblk = (nvalid + 63) / 64;
+      for (int task = warp; task < G * nblk; task += kSConsumers / 32) {
+        const int h = task / nblk, bi = task % nblk;
+        const float* row = sc + h * (kSItem + 4) + bi * 64;
+        const float s0 = row[lane], s1 = row[lane + 32];  // keys past N read -inf
+        const float mb = warp_max(fmaxf(s0, s1));
+        float e = expf(s0 - mb) + expf(s1 - mb);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+        if (lane == 0)
+          p.blk[(int64_t)(row0 + h) * p.n_blk + j0 / 64 + bi] = make_float2(mb, mb + logf(e));
+        float* dst = p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0 + bi * 64;
+        dst[lane] = s0;
+        dst[lane + 32] = s1;
+      }
+      named_bar(1, kSConsumers);  // sc is rewritten by the next item
+      continue;
+    }
     for (int h = warp; h < G; h += kSConsumers / 32) {  // max bin per head, scores' store
       const float* row = sc + h * (kSItem + 4);
       float mx = -INFINITY;
@@ -1151,7 +1166,7 @@ using namespace rtp;
 namespace rtp {
 rtp_status decode_score_pass(const rtp_shape* shape, const HeadMap& hm, int k16_per_kv_head,
                              const rtp_view& q16, const rtp_view& k16_cache, void* ws,
-                             const DecodeWs& L, cudaStream_t s) {
+                             const DecodeWs& L, cudaStream_t s, bool block_stats) {
   rtp_status st = RTP_OK;
   char* w = static_cast<char*>(ws);
   const int N = (int)(shape->q_pos0 + 1);  // keys 0..P
@@ -1187,6 +1202,8 @@ rtp_status decode_score_pass(const rtp_shape* shape, const HeadMap& hm, int k16_
     sp.batch_coord = (k16_cache.stride_b != 0 || shape->B == 1) ? 1 : 0;
     sp.items_per_group = L.Lk_pad / kSItem;
     sp.n_items = groups * sp.items_per_group;
+    sp.blk = block_stats ? static_cast<float2*>(at(L.blk)) : nullptr;
+    sp.n_blk = L.n_blk;
     // k16 as a 4-D tensor {16 x slots per box, slot boxes, keys 0..N-1, batch}
     // (keys past N read as 0); boxes of 128 keys x one slot (32-byte swizzled) or
     // x four slots (128-byte swizzled)
@@ -1265,7 +1282,8 @@ extern "C" rtp_status rtp_sparse_attn_decode_select(
   const int groups = shape->B * hm.n_rkv;
   auto at = [&](size_t off) { return static_cast<void*>(w + off); };
 
-  if ((st = decode_score_pass(shape, hm, k16_per_kv_head, q16, k16_cache, ws, L, s)) != RTP_OK)
+  if ((st = decode_score_pass(shape, hm, k16_per_kv_head, q16, k16_cache, ws, L, s,
+                              select == RTP_SELECT_BLOCK_TOPP)) != RTP_OK)
     return st;
   if (scores_out != nullptr && L.rows > 0 &&
       cudaMemcpy2DAsync(scores_out, (size_t)N * 4, at(L.scores), (size_t)L.Lk_pad * 4,

@@ -12,18 +12,19 @@
 //                 keys share the prefix, then sorts those in shared memory.
 //                 Counts are integers, so the cut is exact.
 //   block top-p   the summary's sort-free decode selection ("Hardware-Aware
-//                 Fast Top-p Decoding Kernel", steps 1-5): 64-key blocks reduced
-//                 to (max m_b, log-sum-exp l_b), a 256-bin histogram over
-//                 [min m_b, max m_b] whose bins sum exp(l_b - max) as 2^-40 fixed
-//                 point (order-free, so deterministic), a walk down the bins to
-//                 mass p, one bit per selected block.  One CTA per row, a warp
-//                 per block.
+//                 Fast Top-p Decoding Kernel", steps 1-5): the score pass reduces
+//                 64-key blocks to (max m_b, log-sum-exp l_b) as it scores them
+//                 (fused, as the summary's kernel is); here a 256-bin histogram
+//                 over [min m_b, max m_b] whose bins sum exp(l_b - max) as 2^-40
+//                 fixed point (order-free, so deterministic), a walk down the
+//                 bins to mass p, one bit per selected block.  One CTA per row.
 //
 // A list kernel then writes, per (batch entry, retrieval kv head) and chunk of
 // 1024 keys, the ordered list of keys some head keeps with their kept-head bits,
 // which the split-KV list attention of decode.cu consumes unchanged.
 #include <algorithm>
 
+#include "dec_bins.cuh"
 #include "rtp_host.h"
 
 namespace rtp {
@@ -39,6 +40,8 @@ constexpr int kVBuckets = 1 << kVDigit;
 
 struct VarParams {
   const float* scores;      // [rows][Lk_pad]
+  const uint32_t* hist_c;   // [rows][kDecGBins]: keys per absolute score bin
+  const uint32_t* flags;    // [rows]: 1 = a score fell outside the histogram's range
   RowRes* rowres;           // [rows]
   float2* blk;              // [rows][n_blk]: (m_b, l_b)
   uint32_t* bmask;          // [rows][n_bwords]
@@ -147,42 +150,25 @@ __global__ void __launch_bounds__(kVThreads) dec_topk_kernel(const VarParams p) 
     rr.count = N;
     rr.mass = 1.f;
   } else {
-    float mx = -INFINITY;
-    for (int j = tid; j < N; j += kVThreads) mx = fmaxf(mx, srow[j]);
-    const float m = block_max_f(mx, sm.fred);
-    unsigned long long zl = 0;
-    for (int j = tid; j < N; j += kVThreads) zl += mass_fixed40(vexp(srow[j] - m));
-    const unsigned long long Z = block_sum_ull(zl, sm.ured);
-    // radix levels: the k-th largest composite key, by counts
-    int pb = 0;
-    unsigned long long prefix = 0, acc_above = 0;
+    // Pick the first digit level: the score pass's absolute bins when every
+    // score fell inside them (one more pass then collects the crossing bin),
+    // else 11-bit radix digits of the composite keys.
+    const bool use_hist = p.flags[row] == 0u;
+    float m;  // mass reference >= every score: the top occupied bin's upper edge, or the max
+    int pb = 0, gstar = 0;  // the crossing absolute bin (use_hist)
+    unsigned long long prefix = 0, acc_above = 0, Z = 0;
     uint32_t need = (uint32_t)p.top_k, n_in = (uint32_t)N;
-    while (n_in > (uint32_t)kVCap && pb < kVKeyBits) {
-      const int w = min(kVDigit, kVKeyBits - pb);
-      const int nbk = 1 << w;
-      for (int d = tid; d < nbk; d += kVThreads) {
-        sm.hc[d] = 0;
-        sm.hm[d] = 0;
-      }
-      __syncthreads();
-      for (int j = tid; j < N; j += kVThreads) {
-        const float s = srow[j];
-        const unsigned long long ck = vkey(s, j);
-        if (pb > 0 && (ck >> (kVKeyBits - pb)) != prefix) continue;
-        const int d = (int)((ck >> (kVKeyBits - pb - w)) & (unsigned long long)(nbk - 1));
-        atomicAdd(&sm.hc[d], 1u);
-        atomicAdd(&sm.hm[d], mass_fixed40(vexp(s - m)));
-      }
-      __syncthreads();
-      // buckets in descending digit order: thread t owns positions 2t, 2t + 1
+    // inclusive scan over 2048 buckets in descending order (thread t: positions
+    // 2t, 2t + 1); returns the crossing position's bucket via shared memory
+    auto cross = [&](const uint32_t* hc, const unsigned long long* hm, int nbk) {
       uint32_t c2[2] = {0, 0};
       unsigned long long m2[2] = {0, 0};
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int pos = 2 * tid + u;
         if (pos < nbk) {
-          c2[u] = sm.hc[nbk - 1 - pos];
-          m2[u] = sm.hm[nbk - 1 - pos];
+          c2[u] = hc[nbk - 1 - pos];
+          m2[u] = hm ? hm[nbk - 1 - pos] : 0ull;
         }
       }
       uint32_t ci = c2[0] + c2[1];
@@ -220,6 +206,70 @@ __global__ void __launch_bounds__(kVThreads) dec_topk_kernel(const VarParams p) 
         mb += m2[u];
       }
       __syncthreads();
+    };
+    if (use_hist) {
+      const uint32_t* hrow = p.hist_c + (int64_t)row * kDecGBins;
+      int top = -1;
+      for (int g = tid; g < kDecGBins; g += kVThreads)
+        if (hrow[g]) top = max(top, g);
+      top = (int)block_max_f((float)top, sm.fred);
+      m = (float)(top + kDecGLo + 1) / kDecKappa;
+      cross(hrow, nullptr, kDecGBins);
+      gstar = sm.s_d + kDecGLo;  // the crossing absolute bin
+      need -= sm.s_cnt;
+      n_in = sm.s_nin;
+      // one pass: Z, the mass above the crossing bin, its keys as candidates
+      if (tid == 0) sm.ncand = 0;
+      __syncthreads();
+      unsigned long long zl = 0, al = 0;
+      for (int j = tid; j < N; j += kVThreads) {
+        const float s = srow[j];
+        const unsigned long long w = mass_fixed40(vexp(s - m));
+        const int bb = sbin(s);
+        zl += w;
+        if (bb > gstar) {
+          al += w;
+        } else if (bb == gstar && n_in <= (uint32_t)kVCap) {
+          const int idx = atomicAdd(&sm.ncand, 1);
+          if (idx < kVCap) sm.cand[idx] = vkey(s, j);
+        }
+      }
+      Z = block_sum_ull(zl, sm.ured);
+      acc_above = block_sum_ull(al, sm.ured);
+      if (n_in > (uint32_t)kVCap) {  // a crowded bin: radix digits below its bin bits
+        prefix = 0;
+        pb = 0;
+      }
+    } else {
+      float mx = -INFINITY;
+      for (int j = tid; j < N; j += kVThreads) mx = fmaxf(mx, srow[j]);
+      m = block_max_f(mx, sm.fred);
+      unsigned long long zl = 0;
+      for (int j = tid; j < N; j += kVThreads) zl += mass_fixed40(vexp(srow[j] - m));
+      Z = block_sum_ull(zl, sm.ured);
+    }
+    // radix levels over the composite keys (restricted to the crossing bin when
+    // the histogram chose one) while too many keys share the prefix
+    const bool radix = !use_hist || n_in > (uint32_t)kVCap;
+    while (radix && n_in > (uint32_t)kVCap && pb < kVKeyBits) {
+      const int w = min(kVDigit, kVKeyBits - pb);
+      const int nbk = 1 << w;
+      for (int d = tid; d < nbk; d += kVThreads) {
+        sm.hc[d] = 0;
+        sm.hm[d] = 0;
+      }
+      __syncthreads();
+      for (int j = tid; j < N; j += kVThreads) {
+        const float s = srow[j];
+        if (use_hist && sbin(s) != gstar) continue;
+        const unsigned long long ck = vkey(s, j);
+        if (pb > 0 && (ck >> (kVKeyBits - pb)) != prefix) continue;
+        const int d = (int)((ck >> (kVKeyBits - pb - w)) & (unsigned long long)(nbk - 1));
+        atomicAdd(&sm.hc[d], 1u);
+        atomicAdd(&sm.hm[d], mass_fixed40(vexp(s - m)));
+      }
+      __syncthreads();
+      cross(sm.hc, sm.hm, nbk);
       need -= sm.s_cnt;
       acc_above += sm.s_acc;
       n_in = sm.s_nin;
@@ -227,16 +277,20 @@ __global__ void __launch_bounds__(kVThreads) dec_topk_kernel(const VarParams p) 
       pb += w;
       __syncthreads();
     }
-    // the keys sharing the prefix, sorted; the cut is the need-th of them
-    if (tid == 0) sm.ncand = 0;
-    __syncthreads();
-    for (int j = tid; j < N; j += kVThreads) {
-      const unsigned long long ck = vkey(srow[j], j);
-      if (pb > 0 && (ck >> (kVKeyBits - pb)) != prefix) continue;
-      const int idx = atomicAdd(&sm.ncand, 1);
-      if (idx < kVCap) sm.cand[idx] = ck;
+    if (radix) {  // the keys sharing the prefix
+      if (tid == 0) sm.ncand = 0;
+      __syncthreads();
+      for (int j = tid; j < N; j += kVThreads) {
+        const float s = srow[j];
+        if (use_hist && sbin(s) != gstar) continue;
+        const unsigned long long ck = vkey(s, j);
+        if (pb > 0 && (ck >> (kVKeyBits - pb)) != prefix) continue;
+        const int idx = atomicAdd(&sm.ncand, 1);
+        if (idx < kVCap) sm.cand[idx] = ck;
+      }
     }
     __syncthreads();
+    // sorted, the cut is the need-th of them
     const int n = min(sm.ncand, kVCap);
     if (sm.ncand > kVCap && tid == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 41);
     vsort_desc(sm.cand, n);
@@ -287,24 +341,16 @@ __global__ void __launch_bounds__(kVThreads) dec_block_topp_kernel(const VarPara
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int N = p.N;
   const int nb = (N + kDecBlk - 1) / kDecBlk;
-  const float* srow = p.scores + (int64_t)row * p.Lk_pad;
   float2* brow = p.blk + (int64_t)row * p.n_blk;
-  // 1-2. per block: max and log-sum-exp (a warp per block)
+  // 1-2. per block: max and log-sum-exp, written by the score pass
   float lo = INFINITY, hi = -INFINITY;
-  for (int bb = warp; bb < nb; bb += kVThreads / 32) {
-    const int j0 = bb * kDecBlk + lane, j1 = j0 + 32;
-    const float s0 = j0 < N ? srow[j0] : -INFINITY;
-    const float s1 = j1 < N ? srow[j1] : -INFINITY;
-    const float mb = warp_max(fmaxf(s0, s1));
-    float e = (j0 < N ? expf(s0 - mb) : 0.f) + (j1 < N ? expf(s1 - mb) : 0.f);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    if (lane == 0) brow[bb] = make_float2(mb, mb + logf(e));
+  for (int bb = tid; bb < nb; bb += kVThreads) {
+    const float mb = brow[bb].x;
     lo = fminf(lo, mb);
     hi = fmaxf(hi, mb);
   }
   for (int k = tid; k < kDecHBins; k += kVThreads) sm.hist[k] = 0;
-  lo = block_min_f(lo, sm.fred);  // the block barriers also publish brow to the CTA
+  lo = block_min_f(lo, sm.fred);
   hi = block_max_f(hi, sm.fred);
   // 3. histogram over the block maxima
   for (int bb = tid; bb < nb; bb += kVThreads) {
@@ -480,6 +526,8 @@ rtp_status decode_variant_select(const rtp_shape* shape, const HeadMap& hm, rtp_
   VarParams vp;
   memset(&vp, 0, sizeof(vp));
   vp.scores = static_cast<const float*>(at(L.scores));
+  vp.hist_c = static_cast<const uint32_t*>(at(L.hist_c));
+  vp.flags = static_cast<const uint32_t*>(at(L.flags));
   vp.rowres = static_cast<RowRes*>(at(L.rowres));
   vp.blk = static_cast<float2*>(at(L.blk));
   vp.bmask = static_cast<uint32_t*>(at(L.bmask));

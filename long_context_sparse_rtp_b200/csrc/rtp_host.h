@@ -208,10 +208,11 @@ inline DecodeWs decode_ws_layout(const rtp_shape* s, const HeadMap& hm) {
 
 // The retrieval decode's first pass (decode_select.cu): clears the row
 // histograms, then scores every key of the cache into the workspace's score
-// rows [rows][Lk_pad] and bins them.
+// rows [rows][Lk_pad] and bins them; with block_stats, instead of binning, it
+// reduces every 64-key block to (max, log-sum-exp) in the workspace's blk rows.
 rtp_status decode_score_pass(const rtp_shape* shape, const HeadMap& hm, int k16_per_kv,
                              const rtp_view& q16, const rtp_view& k16_cache, void* ws,
-                             const DecodeWs& L, cudaStream_t s);
+                             const DecodeWs& L, cudaStream_t s, bool block_stats);
 
 // Buffers the gathered decode attention reads (decode.cu).
 struct DecodeLists {

@@ -103,3 +103,26 @@ def test_dense_decode_leg_bookkeeping(monkeypatch):
     assert r["bytes"] == B * L * Hkv * 128 * 2 * 2 == 2147483648
     assert abs(r["ms_step"] - 0.35) < 1e-12
     assert calls == [(L - 1, (B, 1, H, 128), (B, H, 1))] * 7
+
+
+def test_attention_pair_counts_against_brute_force():
+    """The roofline pair counts: the sink + window rule summed over rows, and
+    the 128 x 128 tiles the causal / local schedules visit, against explicit
+    enumeration on small sizes."""
+    import numpy as np
+    for L, W, S in [(1, 1, 0), (5, 3, 1), (300, 37, 4), (1000, 256, 4), (700, 1000, 0)]:
+        brute = sum(len([j for j in range(P + 1) if j < S or j > P - W]) for P in range(L))
+        assert bench.local_pairs(L, W, S) == brute
+    for L, W, S in [(1, 1, 0), (200, 64, 4), (1000, 256, 4), (1300, 300, 130)]:
+        nb = (L + 127) // 128
+        dense = local = 0
+        for rb in range(nb):
+            P0, Pl = rb * 128, min(L, rb * 128 + 128) - 1
+            for t in range(Pl // 128 + 1):
+                dense += 1
+                keys = range(t * 128, t * 128 + 128)
+                # a tile is visited iff some row of the block keeps some key of it
+                if any(j <= P and (j < S or j > P - W) for P in range(P0, Pl + 1) for j in keys):
+                    local += 1
+        assert bench.tile_pairs(L) == dense * 128 * 128
+        assert bench.tile_pairs(L, W, S) == local * 128 * 128, (L, W, S)

@@ -236,3 +236,25 @@ def test_recall_against_exact_topp():
     out["topp"] = dict(keys=float(exact.sum(-1).float().mean()))
     report("recall vs exact top-p, decode 32K x 4, p=0.95, k=4096", out)
     assert out["block_topp"]["mass_kept"] >= w.p - 1e-3   # whole bins: at least p
+
+
+def test_topk_scores_outside_histogram_range():
+    """W_q16 scaled by 64: scores spread far beyond the score pass's absolute
+    bins ([-256, 256)), so the row is flagged and top-k takes its generic radix
+    path over all keys; the cut is still exact (checked against the oracle on
+    the same fp32 scores)."""
+    w = W["decode_128k_b8"]
+    inp = synth.make_inputs(w, "cuda", L=6000, B=2)
+    q, k, v, Wk, role = (inp[x] for x in ("q", "k", "v", "Wk16", "kv_role"))
+    Wq = (inp["Wq16"].float() * 64).to(torch.bfloat16)
+    q16, k16 = rtp_index_scores(q, k, Wq, Wk, role)
+    _, _, s = rtp_sparse_attn_decode_select(q, k, v, q16, k16, role, "topk", top_k=700,
+                                            want_scores=True)
+    torch.cuda.synchronize()
+    sc = s["scores"].cpu().numpy().astype(np.float64)
+    assert np.abs(sc).max() > 256
+    for b in range(2):
+        for r in range(w.H_ret):
+            o = oracle.topk(sc[b, r], 700)
+            assert float(s["thr"][b, r]) == o["t"] and int(s["jtie"][b, r]) == o["jtie"]
+            assert int(s["count"][b, r]) == 700

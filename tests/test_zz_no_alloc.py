@@ -5,7 +5,8 @@ allocator they do not own (a host framework's fixed pool, a plugin interface
 that hands over only inputs and outputs) or in a phase where device allocation
 is not allowed.  rtp_local_attn_decode_noalloc keeps its scratch in a fixed
 8 MiB device array instead.  These tests call it through the C ABI and check it
-against rtp_local_attn, which takes a caller workspace, on two calls in a row.
+against rtp_local_attn, which takes a caller workspace, on two calls in a row,
+and against the fp64 oracle's sink + window attention.
 This file is collected last on purpose, so that a run stopping at the first
 failure has run every other test before it.
 """
@@ -16,8 +17,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from long_context_sparse_rtp_b200 import build, rtp, synth
-from rtp_check import check_outputs
+from rtp_check import LSE_ABS, bits, check_outputs
 
 
 def _args(inp, q_pos0):
@@ -69,9 +71,14 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert code == 0, rtp.STATUS.get(code, code)
         torch.cuda.synchronize()
         outs.append((o, lse))
+    rows = np.array([(b, 0, h) for b in range(q.shape[0]) for h in loc])
+    orc = oracle.local_rows(bits(q), bits(k), bits(v), rows, H=w.H, Hkv=w.Hkv, q_pos0=5999,
+                            window=w.window, n_sink=w.n_sink, scale=scale)
     for o, lse in outs:
         a = o[:, 0, loc].float().cpu().numpy().reshape(-1, 128)
         b = o_ref[:, 0, loc].float().cpu().numpy().reshape(-1, 128)
         check_outputs(a, b.astype(np.float64), "no-alloc local decode")
         np.testing.assert_allclose(lse[:, loc].cpu().numpy(), lse_ref[:, loc].cpu().numpy(),
                                    atol=2e-2, rtol=0)
+        check_outputs(a, orc["o"], "no-alloc local decode vs the oracle")
+        assert np.abs(lse[:, loc, 0].cpu().numpy().reshape(-1) - orc["lse"]).max() <= LSE_ABS

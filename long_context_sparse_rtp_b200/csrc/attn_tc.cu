@@ -20,8 +20,8 @@
 // domain, write P (bf16, two per column) over the scores in TMEM, where the PV
 // MMA reads it as its A operand.  The running max is only
 // moved (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles
-// need no rescale.  P is rounded to bf16 once and the normaliser sums the
-// rounded values, so the output is an exact convex combination of them.
+// need no rescale.  P is rounded to bf16 once for the PV MMA; the normaliser
+// sums the fp32 values.
 #include <cuda.h>
 
 #include "rtp_host.h"
@@ -307,14 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i) {
             reg_fence(r16[i]);
             reg_fence(rs[i]);
-            x[c * 32 + i] = __uint_as_float(r16[i]) > te ? __uint_as_float(rs[i]) * p.scale_log2
-                                                          : -INFINITY;
+            x[c * 32 + i] = __uint_as_float(r16[i]) > te ? __uint_as_float(rs[i]) : -INFINITY;
           }
           if (mixed) {  // ties up to the tie index (-0 and +0 compare equal)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const bool tie = ok & (__uint_as_float(r16[i]) == thr) & (c * 32 + i <= jtl);
-              x[c * 32 + i] = tie ? __uint_as_float(rs[i]) * p.scale_log2 : x[c * 32 + i];
+              x[c * 32 + i] = tie ? __uint_as_float(rs[i]) : x[c * 32 + i];
             }
           }
         }
@@ -339,17 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool full = false;
         if (MODE == MODE_DENSE) full = j0 + 63 <= P;
         if (MODE == MODE_LOCAL) full = j0 + 63 <= P && (j0 > P - p.window || j0 + 63 < p.n_sink);
-        if (full && ok) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) x[i] *= p.scale_log2;
-        } else {
+        if (!(full && ok)) {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int64_t j = j0 + i;
             bool kp;
             if (MODE == MODE_DENSE) kp = j <= P;
             else kp = (j <= P) & ((j < p.n_sink) | (j > P - p.window));
-            x[i] = (ok & kp) ? x[i] * p.scale_log2 : -INFINITY;
+            x[i] = (ok & kp) ? x[i] : -INFINITY;
           }
         }
       }
@@ -358,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < 8; ++e) tm[e] = x[e];
 #pragma unroll
       for (int i = 8; i < 64; ++i) tm[i & 7] = fmaxf(tm[i & 7], x[i]);
+      // in the log2 domain (scale > 0 keeps the order; -inf stays -inf)
       float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
-                         fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
+                         fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7]))) *
+                   p.scale_log2;
       // the row's tile max from the partner thread (parity-paired slots)
       sm.tmax[it & 1][g][r] = tmax;
       named_bar(pair_bar, 64);
@@ -399,8 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          pk[e] = pack_bf16x2(ex2_ftz(x[2 * e] - msafe), ex2_ftz(x[2 * e + 1] - msafe));
-          lsum[e & 3] += bf16_lo(pk[e]) + bf16_hi(pk[e]);
+          const float p0 = ex2_ftz(__fmaf_rn(x[2 * e], p.scale_log2, -msafe));
+          const float p1 = ex2_ftz(__fmaf_rn(x[2 * e + 1], p.scale_log2, -msafe));
+          pk[e] = pack_bf16x2(p0, p1);
+          lsum[e & 3] += p0 + p1;
         }
         if (ok) tmem_st32u(t_s + lane_off + (uint32_t)(sb * kBN + g * 32), pk);
       }
@@ -454,6 +454,313 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// DENSE and LOCAL on two query tiles per CTA.
+//
+// One CTA = 256 query rows of one head (two 128-row tiles A and B) and one pass
+// over the union of their key tiles.  TMEM holds, per query tile, a 128-column
+// score buffer (P is written over it) and a 128-column O accumulator.  Warp 9
+// issues, per key tile t: PV_A(t), S_A(t+1), PV_B(t), S_B(t+1), so the softmax
+// of one tile runs while the tensor cores work on the other's.  Warps 0-3 hold
+// the rows of tile A, warps 4-7 those of B: one thread per query row, all 128
+// keys of a key tile (read from TMEM twice: the row max, then P), no exchange
+// with another thread.  Warp 8 loads both Q tiles once and K/V tiles into a
+// 2-stage ring with TMA.  Same arithmetic as the single-tile kernel: scores
+// scaled into the log2 domain, the running max moved (and O rescaled) only when
+// it grows by more than 2^8, P rounded to bf16 once for the MMA and summed in fp32,
+// in the single-tile kernel's order (the two give the same bits).
+constexpr int kPQ = 2;                     // query tiles per CTA
+constexpr int kPRows = kPQ * kBM;          // 256
+
+struct PpSmem {                            // placed on a 1024-byte boundary
+  uint8_t q[kPQ][kTile];
+  uint8_t k[kStages][kTile];
+  uint8_t v[kStages][kTile];
+  // each completes once per key tile: s_full[q] (the S MMAs of tile q),
+  // p_full[q] (tile q's four softmax warps wrote P), pv_done[q] (its PV MMAs)
+  uint64_t q_full, kv_full[kStages], kv_empty[kStages], s_full[kPQ], p_full[kPQ], pv_done[kPQ];
+  uint32_t tmem_base;
+  int gave_up;
+};
+
+// A key tile of the two-tile kernel that some row of the warp attends to only in
+// part: the scores of keys outside the rule (key i kept iff i <= dp and (i < ds
+// or i > dw)) become -inf in this thread's TMEM lane (columns ts .. ts + 127),
+// 32 columns at a time, skipping chunks no row of the warp masks.
+__device__ __forceinline__ void pp_mask(uint32_t ts, int dp, int ds, int dw) {
+#pragma unroll 1
+  for (int w = 0; w < 4; ++w) {
+    const int k0 = 32 * w;
+    const bool whole = k0 + 31 <= dp && (ds >= k0 + 32 || dw < k0);
+    if (__all_sync(0xffffffffu, whole)) continue;
+    uint32_t ra[32];
+    tmem_ld32_nowait(ts + (uint32_t)k0, ra);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      reg_fence(ra[i]);
+      const int k = k0 + i;
+      ra[i] = (k <= dp && (k < ds || k > dw)) ? ra[i] : 0xFF800000u;  // -inf
+    }
+    tmem_st32u(ts + (uint32_t)k0, ra);
+  }
+  tmem_wait_st();
+}
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_pp_kernel(const __grid_constant__ CUtensorMap qmap,
+                   const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  PpSmem& sm = *reinterpret_cast<PpSmem*>(smem_raw +
+                                          ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hidx = blockIdx.y;
+  const int h = p.head[hidx];
+  const int kvh = h / p.G;
+  const int b = blockIdx.z;
+  const int rb = gridDim.x - 1 - blockIdx.x;  // heavy (late) row blocks first
+  const int m0 = rb * kPRows;
+  const int nrows = min(kPRows, p.Lq - m0);
+  const int64_t P0 = p.q_pos0 + m0;
+  const int64_t Plast = P0 + nrows - 1;
+  const Sched sch = make_sched<MODE>(p, P0, Plast);  // the union of both tiles' key tiles
+
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int q = 0; q < kPQ; ++q) {
+      mbar_init(&sm.s_full[q], 1);
+      mbar_init(&sm.p_full[q], 4);
+      mbar_init(&sm.pv_done[q], 1);
+    }
+    sm.gave_up = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* gave_up = &sm.gave_up;
+  auto t_s = [&](int q) { return tmem + (uint32_t)(q * 256); };
+  auto t_o = [&](int q) { return tmem + (uint32_t)(q * 256 + 128); };
+
+  if (warp == kProdWarp) {  // ---------------------------------------- TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(kPQ * kTile));
+      for (int q = 0; q < kPQ; ++q) {  // rows past the tensor read as zeros
+        tma_load_4d(sm.q[q], &qmap, 0, h, m0 + q * kBM, b * p.bq, &sm.q_full);
+        tma_load_4d(sm.q[q] + kHalf, &qmap, 64, h, m0 + q * kBM, b * p.bq, &sm.q_full);
+      }
+      int n_issued = 0;
+      for (int it = 0; it < sch.n; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait(&sm.kv_empty[st], ((uint32_t)(it >> 1) & 1u) ^ 1u, gave_up)) {
+          ok = false;
+          break;
+        }
+        const int j0 = sch.tile(it) * kBN;
+        mbar_arrive_expect_tx(&sm.kv_full[st], (uint32_t)(2 * kTile));
+        tma_load_4d(sm.k[st], &kmap, 0, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.k[st] + kHalf, &kmap, 64, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.v[st], &vmap, 0, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        tma_load_4d(sm.v[st] + kHalf, &vmap, 64, kvh, j0, b * p.bk, &sm.kv_full[st]);
+        ++n_issued;
+      }
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 44);
+      for (int k = max(0, n_issued - kStages); k < n_issued; ++k)
+        mbar_wait_drain(&sm.kv_full[k & 1], (uint32_t)(k >> 1) & 1u);
+      mbar_wait_drain(&sm.q_full, 0u);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {  // ---------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.q_full, 0u, gave_up);
+      int n_pv = 0;
+      auto S = [&](int q, int it) {  // S_q = Q_q K(it)^T into the tile's score buffer
+        const int st = it & 1;
+        if (!mbar_wait(&sm.kv_full[st], (uint32_t)(it >> 1) & 1u, gave_up)) return false;
+        // P of the previous key tile is read by its PV MMAs before S overwrites it
+        if (it > 0 && !mbar_wait(&sm.pv_done[q], (uint32_t)(it - 1) & 1u, gave_up)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(t_s(q), kdesc(sm.q[q], kk), kdesc(sm.k[st], kk), kIdescQK, kk > 0);
+        mma_commit(&sm.s_full[q]);
+        return true;
+      };
+      auto PV = [&](int q, int it) {  // O_q += P_q V(it), P read from TMEM
+        if (!mbar_wait(&sm.p_full[q], (uint32_t)it & 1u, gave_up)) return false;
+        tc_fence_after();
+        const int st = it & 1;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(t_o(q), t_s(q) + (uint32_t)(kk * 8), vdesc(sm.v[st], kk), kIdescPV,
+                      it > 0 || kk > 0);
+        mma_commit(&sm.pv_done[q]);
+        if (q == kPQ - 1) mma_commit(&sm.kv_empty[st]);  // the stage's last reader
+        ++n_pv;
+        return true;
+      };
+      if (ok && sch.n > 0) ok = S(0, 0) && S(1, 0);
+      for (int it = 0; ok && it < sch.n; ++it) {
+        ok = PV(0, it);
+        if (ok && it + 1 < sch.n) ok = S(0, it + 1);
+        if (ok) ok = PV(1, it);
+        if (ok && it + 1 < sch.n) ok = S(1, it + 1);
+      }
+      if (!ok) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 45);
+      if (n_pv > 0)  // the last MMAs are complete before TMEM is released
+        for (int q = 0; q < kPQ; ++q)
+          mbar_wait_drain(&sm.pv_done[q], (uint32_t)(sch.n - 1) & 1u);
+    }
+    __syncwarp();
+  } else {  // ------------------------------------ softmax: one thread per query row
+    const int q = warp >> 2;                  // query tile
+    const int r = (warp & 3) * 32 + lane;     // row in the tile = TMEM lane
+    const int row = q * kBM + r;              // row in the CTA
+    const bool valid = row < nrows;
+    const int64_t P = P0 + row;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t ts = t_s(q) + lane_off, to = t_o(q) + lane_off;
+    const float c = p.scale_log2;
+    float m_used = -INFINITY, l0 = 0.f, l1 = 0.f;  // row sums of keys 0-63 / 64-127 of the tiles
+    bool ok = true;
+    for (int it = 0; it < sch.n; ++it) {
+      const int64_t j0 = (int64_t)sch.tile(it) * kBN;
+      ok = ok && mbar_wait_warp(&sm.s_full[q], (uint32_t)it & 1u, gave_up);
+      tc_fence_after();
+      // key j0 + i is attended to iff i <= dp and (i < ds or i > dw)
+      auto clamp_off = [](int64_t d) { return (int)(d < -1 ? -1 : (d > kBN ? kBN : d)); };
+      const int dp = clamp_off(P - j0);
+      const int ds = MODE == MODE_LOCAL ? clamp_off((int64_t)p.n_sink - j0) : kBN;
+      const int dw = MODE == MODE_LOCAL ? clamp_off(P - p.window - j0) : -1;
+      // every key of the tile attended to, for every row of the warp: no mask
+      const bool wfull = __all_sync(0xffffffffu, dp >= kBN - 1 && (ds >= kBN || dw < 0));
+      if (!wfull && ok) pp_mask(ts, dp, ds, dw);
+      // the tile's 128 raw scores with one wait; the row max (scale > 0 keeps
+      // the order) in the log2 domain
+      uint32_t sr[4][32];
+      if (ok) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) tmem_ld32_nowait(ts + (uint32_t)(w * 32), sr[w]);
+        tmem_wait_ld();
+      }
+      float tm[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tm[e] = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          reg_fence(sr[w][i]);
+          tm[i & 7] = fmaxf(tm[i & 7], __uint_as_float(sr[w][i]));
+        }
+      const float smax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
+                               fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
+      const float tmax = ok ? smax * c : -INFINITY;  // -inf stays -inf
+      const float m_new = fmaxf(m_used, tmax);
+      const bool first = m_used == -INFINITY && m_new > -INFINITY;  // O and l are still 0
+      const bool move = m_used > -INFINITY && m_new > m_used + kRescale;
+      float alpha = 1.f;
+      if (first) m_used = m_new;
+      if (move) {
+        alpha = exp2f(m_used - m_new);
+        m_used = m_new;
+        l0 *= alpha;
+        l1 *= alpha;
+      }
+      // P = 2^(s c - m) rounded to bf16 once, keys 2e, 2e + 1 of the tile into
+      // column e (columns already read); the per-half sums gather the fp32
+      // values, pair e of a half into slot e % 4 in order of e
+      const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {  // keys 64 hf .. 64 hf + 63
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int w = 2 * hf; w < 2 * hf + 2; ++w) {  // keys 32 w .. + 31 -> columns 16 w .. + 15
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_ftz(__fmaf_rn(__uint_as_float(sr[w][2 * e]), c, -msafe));
+            const float p1 = ex2_ftz(__fmaf_rn(__uint_as_float(sr[w][2 * e + 1]), c, -msafe));
+            pk[e] = pack_bf16x2(p0, p1);
+            ls[e & 3] += p0 + p1;
+          }
+          if (ok) tmem_st16u(ts + (uint32_t)(w * 16), pk);
+        }
+        (hf ? l1 : l0) += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      }
+      // O is rescaled (rarely) once the previous key tile's PV MMAs are done (the
+      // next PV waits for this tile's P)
+      if (it > 0 && __any_sync(0xffffffffu, move)) {
+        ok = ok && mbar_wait_warp(&sm.pv_done[q], (uint32_t)(it - 1) & 1u, gave_up);
+        tc_fence_after();
+        if (ok) {
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float o[32];
+            tmem_ld32(to + (uint32_t)(cc * 32), o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(to + (uint32_t)(cc * 32), o);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[q]);
+    }
+    // ---- epilogue: O / l from TMEM, the row's 128 dimensions to global
+    if (sch.n > 0)
+      ok = ok && mbar_wait_warp(&sm.pv_done[q], (uint32_t)(sch.n - 1) & 1u, gave_up);
+    tc_fence_after();
+    const float l = l0 + l1;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint16_t* orow = p.o + b * p.o_sb + (int64_t)(m0 + row) * p.o_sl + (int64_t)h * kD;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      float o[32];
+      if (sch.n > 0) {
+        tmem_ld32(to + (uint32_t)(cc * 32), o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+      if (valid) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 w;
+          w.x = pack_bf16x2(o[q4 * 8 + 0] * inv, o[q4 * 8 + 1] * inv);
+          w.y = pack_bf16x2(o[q4 * 8 + 2] * inv, o[q4 * 8 + 3] * inv);
+          w.z = pack_bf16x2(o[q4 * 8 + 4] * inv, o[q4 * 8 + 5] * inv);
+          w.w = pack_bf16x2(o[q4 * 8 + 6] * inv, o[q4 * 8 + 7] * inv);
+          *reinterpret_cast<uint4*>(orow + cc * 32 + q4 * 8) = w;
+        }
+      }
+    }
+    if (valid && p.lse != nullptr)
+      p.lse[((int64_t)b * p.H + h) * p.Lq + m0 + row] =
+          l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    if (!ok && row == 0) set_status(p.status, RTP_ERR_DEVICE_TIMEOUT, 46);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // A bf16 [B][L][heads][width] view as a 4-D TMA map {width, heads, L, B} with
 // boxes of {box0, 1, 128, 1}; a batch stride of 0 (one tensor shared by every
 // batch entry) maps to a single batch coordinate.
@@ -494,17 +801,29 @@ rtp_status launch_tc(AttnParams& prm, int n_heads, const rtp_shape* shape, const
   if (bk != bv) return RTP_ERR_UNSUPPORTED;
   prm.bq = bq;
   prm.bk = bk;
+  static const char* kName[3] = {"attn_prefill_dense", "attn_prefill_local",
+                                 "attn_prefill_sparse"};
+  if constexpr (MODE != MODE_SPARSE) {  // two query tiles per CTA
+    const size_t psmem = sizeof(PpSmem) + 1024;
+    if (cudaFuncSetAttribute(attn_pp_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)psmem) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    dim3 pgrid((prm.Lq + kPRows - 1) / kPRows, n_heads, B);
+    if (pgrid.y > 65535 || pgrid.z > 65535) return RTP_ERR_UNSUPPORTED;
+    TraceScope tr(kName[MODE], s);
+    attn_pp_kernel<MODE><<<pgrid, kThreads, psmem, s>>>(qm, km, vm, prm);
+    return check_cuda(cudaGetLastError());
+  } else {
   const size_t smem = sizeof(TcSmem) + 1024;
   if (cudaFuncSetAttribute(attn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return RTP_ERR_CUDA;
   dim3 grid((prm.Lq + kBM - 1) / kBM, n_heads, B);
   if (grid.y > 65535 || grid.z > 65535) return RTP_ERR_UNSUPPORTED;
-  static const char* kName[3] = {"attn_prefill_dense", "attn_prefill_local",
-                                 "attn_prefill_sparse"};
   TraceScope tr(kName[MODE], s);
   attn_tc_kernel<MODE><<<grid, kThreads, smem, s>>>(qm, km, vm, q16m, k16m, prm);
   return check_cuda(cudaGetLastError());
+  }
 }
 
 void fill_common(AttnParams& prm, const rtp_shape* shape, const rtp_view& o, float* lse,

@@ -156,3 +156,57 @@ def test_index_scores_keys_only():
     _, k16b = rtp_index_scores(None, k, Wq, Wk, role, H=w.H)
     torch.cuda.synchronize()
     assert torch.equal(k16a, k16b)
+
+
+def check_local_rows(q, k, v, o, lse, role, window, n_sink, q_pos0, what):
+    """Every local head of every query row against oracle.local_rows."""
+    B, Lq, H, _ = q.shape
+    Hkv = k.shape[2]
+    G = H // Hkv
+    loc = [h for h in range(H) if role[h // G] == 0]
+    qb, kb, vb = bits(q), bits(k), bits(v)
+    og = o.float().cpu().numpy()
+    lg = lse.cpu().numpy()
+    got, ref, lerr = [], [], 0.0
+    for i in range(Lq):
+        rows = np.array([(b, 0, h) for b in range(B) for h in loc])
+        r = oracle.local_rows(qb[:, i:i + 1], kb, vb, rows, H=H, Hkv=Hkv, q_pos0=q_pos0 + i,
+                              window=window, n_sink=n_sink, scale=SCALE)
+        got.append(np.stack([og[b, i, h] for (b, _, h) in rows]))
+        ref.append(r["o"])
+        lerr = max(lerr, float(np.abs(np.array([lg[b, h, i] for (b, _, h) in rows])
+                                      - r["lse"]).max()))
+    check_outputs(np.concatenate(got), np.concatenate(ref), what)
+    assert lerr <= LSE_ABS, (what, lerr)
+
+
+@pytest.mark.parametrize("Lq", [77, 256, 333])
+def test_chunked_prefill_dense_every_row(Lq):
+    """A prefill chunk: Lq query rows at positions 300 .. 300 + Lq - 1 over a
+    cache of 300 + Lq keys, batch 2.  The kernel holds 256 query rows per CTA as
+    two 128-row tiles: 77 rows leave the second tile empty, 333 leave the last
+    CTA's second tile part-filled, and position 300 is not tile-aligned."""
+    q_pos0 = 300
+    inp = synth.make_inputs(W["prefill_2k"], "cuda", L=q_pos0 + Lq, B=2)
+    q = inp["q"][:, q_pos0:].contiguous()
+    k, v = inp["k"], inp["v"]
+    o, lse = rtp_dense_attn(q, k, v, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    check_dense_rows(q, k, v, o, lse, list(range(Lq)), q_pos0, f"dense chunk Lq={Lq}")
+
+
+@pytest.mark.parametrize("window,n_sink", [(5, 0), (100, 4), (200, 130), (700, 0)])
+def test_chunked_prefill_local_every_row(window, n_sink):
+    """Sinks + sliding window on a prefill chunk (300 rows at positions 300 ..
+    599 over 600 keys, batch 2): windows narrower than a tile, sinks that span
+    more than one 128-key tile, a window wider than the whole cache, no sinks."""
+    from long_context_sparse_rtp_b200 import rtp_local_attn
+    q_pos0, Lq = 300, 300
+    w = W["prefill_2k"]
+    inp = synth.make_inputs(w, "cuda", L=q_pos0 + Lq, B=2)
+    q = inp["q"][:, q_pos0:].contiguous()
+    k, v, role = inp["k"], inp["v"], inp["kv_role"]
+    o, lse = rtp_local_attn(q, k, v, role, window=window, n_sink=n_sink, q_pos0=q_pos0)
+    torch.cuda.synchronize()
+    check_local_rows(q, k, v, o, lse, [int(x) for x in role], window, n_sink, q_pos0,
+                     f"local chunk window={window} sinks={n_sink}")

@@ -100,6 +100,41 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
   return y;
 }
+// max(a, b, c) in one instruction (exact, like two fmaxf).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Two fp32 lanes in one 64-bit register: packed fma (one rounding per lane, as
+// __fmaf_rn) and add, one instruction for both lanes.
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// The row-sum slots of a half tile (pairs e of keys 2e, 2e + 1 go to slot e % 4,
+// even keys in the low lane, odd in the high), folded in a fixed order.
+__device__ __forceinline__ float fold_sums(const unsigned long long (&ls)[4]) {
+  float a[4], b[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) f2_unpack(ls[k], a[k], b[k]);
+  return ((a[0] + b[0]) + (a[1] + b[1])) + ((a[2] + b[2]) + (a[3] + b[3]));
+}
 
 template <int MODE>
 __device__ __forceinline__ Sched make_sched(const AttnParams& p, int64_t P0, int64_t Plast) {
@@ -353,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) tm[e] = x[e];
 #pragma unroll
-      for (int i = 8; i < 64; ++i) tm[i & 7] = fmaxf(tm[i & 7], x[i]);
+      for (int i = 8; i < 64; i += 2) tm[(i >> 1) & 7] = max3f(tm[(i >> 1) & 7], x[i], x[i + 1]);
       // in the log2 domain (scale > 0 keeps the order; -inf stays -inf)
       float tmax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
                          fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7]))) *
@@ -392,20 +427,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = 2^(x - m) rounded to bf16 once, packed two per column over the scores:
       // keys 64 g + 2e, 64 g + 2e + 1 go to column 32 g + e of the tile's buffer
       const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
-      float lsum[4] = {0.f, 0.f, 0.f, 0.f};
+      unsigned long long lsum[4] = {0ull, 0ull, 0ull, 0ull};  // (+0, +0) pairs
       {
+        const unsigned long long cc = f2_pack(p.scale_log2, p.scale_log2);
+        const unsigned long long mm = f2_pack(-msafe, -msafe);
         uint32_t pk[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_ftz(__fmaf_rn(x[2 * e], p.scale_log2, -msafe));
-          const float p1 = ex2_ftz(__fmaf_rn(x[2 * e + 1], p.scale_log2, -msafe));
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), cc, mm), x0, x1);
+          const float p0 = ex2_ftz(x0), p1 = ex2_ftz(x1);
           pk[e] = pack_bf16x2(p0, p1);
-          lsum[e & 3] += p0 + p1;
+          lsum[e & 3] = f2_add(lsum[e & 3], f2_pack(p0, p1));
         }
         if (ok) tmem_st32u(t_s + lane_off + (uint32_t)(sb * kBN + g * 32), pk);
       }
       tmem_wait_st();
-      l += (lsum[0] + lsum[1]) + (lsum[2] + lsum[3]);
+      l += fold_sums(lsum);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[it & 1]);
@@ -660,9 +698,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int w = 0; w < 4; ++w)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
+        for (int i = 0; i < 32; i += 2) {
           reg_fence(sr[w][i]);
-          tm[i & 7] = fmaxf(tm[i & 7], __uint_as_float(sr[w][i]));
+          reg_fence(sr[w][i + 1]);
+          tm[(i >> 1) & 7] =
+              max3f(tm[(i >> 1) & 7], __uint_as_float(sr[w][i]), __uint_as_float(sr[w][i + 1]));
         }
       const float smax = fmaxf(fmaxf(fmaxf(tm[0], tm[1]), fmaxf(tm[2], tm[3])),
                                fmaxf(fmaxf(tm[4], tm[5]), fmaxf(tm[6], tm[7])));
@@ -682,22 +722,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // column e (columns already read); the per-half sums gather the fp32
       // values, pair e of a half into slot e % 4 in order of e
       const float msafe = m_used == -INFINITY ? 0.f : m_used;  // masked keys: 2^-inf = 0
+      const unsigned long long cc = f2_pack(c, c), mm = f2_pack(-msafe, -msafe);
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {  // keys 64 hf .. 64 hf + 63
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        unsigned long long ls[4] = {0ull, 0ull, 0ull, 0ull};  // (+0, +0) pairs
 #pragma unroll
         for (int w = 2 * hf; w < 2 * hf + 2; ++w) {  // keys 32 w .. + 31 -> columns 16 w .. + 15
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_ftz(__fmaf_rn(__uint_as_float(sr[w][2 * e]), c, -msafe));
-            const float p1 = ex2_ftz(__fmaf_rn(__uint_as_float(sr[w][2 * e + 1]), c, -msafe));
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[w][2 * e]), __uint_as_float(sr[w][2 * e + 1])),
+                             cc, mm),
+                      x0, x1);
+            const float p0 = ex2_ftz(x0), p1 = ex2_ftz(x1);
             pk[e] = pack_bf16x2(p0, p1);
-            ls[e & 3] += p0 + p1;
+            // pair e of the half (16 (w - 2 hf) + e) into slot e % 4: the same slot
+            ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
           }
           if (ok) tmem_st16u(ts + (uint32_t)(w * 16), pk);
         }
-        (hf ? l1 : l0) += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        (hf ? l1 : l0) += fold_sums(ls);
       }
       // O is rescaled (rarely) once the previous key tile's PV MMAs are done (the
       // next PV waits for this tile's P)

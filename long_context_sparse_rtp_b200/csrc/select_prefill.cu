@@ -225,14 +225,11 @@ __device__ __forceinline__ void flush_row(SelSmem& sm, int r) {
 }
 
 __device__ __forceinline__ float max16(const float (&v)[kChunk]) {
-  float t[kChunk / 2];
-#pragma unroll
-  for (int i = 0; i < kChunk / 2; ++i) t[i] = fmaxf(v[i], v[i + kChunk / 2]);
-#pragma unroll
-  for (int w = kChunk / 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) t[i] = fmaxf(t[i], t[i + w]);
-  return t[0];
+  // three-input maxima: 16 -> 6 -> 2 -> 1 (the max is exact in any order)
+  const float a = max3f(v[0], v[1], v[2]), b = max3f(v[3], v[4], v[5]),
+              c = max3f(v[6], v[7], v[8]), d = max3f(v[9], v[10], v[11]),
+              e = max3f(v[12], v[13], v[14]);
+  return fmaxf(max3f(a, b, c), max3f(d, e, v[15]));
 }
 
 // Level-1 sub-bin of a key of level-0 bin k0: the 32 uniform score sub-bins of
@@ -574,29 +571,44 @@ __global__ void __launch_bounds__(kThreads, 2)
     sweep(
         [&](int, float (&v)[kChunk]) {
           if (!valid) return;
-          float e[kChunk];
+          // two keys per packed instruction, each lane rounded as the scalar
+          // forms: rel_w and bin0_of from one difference (exp2(-(m - s) log2 e)
+          // is exp2((s - m) log2 e) bit for bit), fixed_u as add.rz of 2^23
+          const unsigned long long m2 = f2_pack(m, m), nl2 = f2_pack(-kLog2e, -kLog2e),
+                                   sc2 = f2_pack(scale, scale),
+                                   fl2 = f2_pack(12582912.0f, 12582912.0f),
+                                   tz2 = f2_pack(8388608.0f, 8388608.0f);
+          unsigned long long ee[kChunk / 2];
           int bb[kChunk];
 #pragma unroll
-          for (int i = 0; i < kChunk; ++i) {
-            // rel_w and bin0_of from one difference: exp2(-(m - s) log2 e) is
-            // exp2((s - m) log2 e) bit for bit
-            const float dm = __fsub_rn(m, v[i]);
-            e[i] = ex2_ftz(-__fmul_rn(dm, kLog2e));
-            bb[i] = min(__float_as_int(__fadd_rd(__fmul_rn(dm, scale), 12582912.0f)) - 0x4B400000,
-                        kNB);  // kNB: below c0, a bin never read
+          for (int k = 0; k < kChunk / 2; ++k) {
+            const unsigned long long dm = f2_sub(m2, f2_pack(v[2 * k], v[2 * k + 1]));
+            float a0, a1, y0, y1;
+            f2_unpack(f2_mul(dm, nl2), a0, a1);
+            ee[k] = f2_pack(ex2_ftz(a0), ex2_ftz(a1));
+            f2_unpack(f2_add_rm(f2_mul(dm, sc2), fl2), y0, y1);
+            bb[2 * k] = min(__float_as_int(y0) - 0x4B400000, kNB);  // kNB: below c0, never read
+            bb[2 * k + 1] = min(__float_as_int(y1) - 0x4B400000, kNB);
           }
           float t[kChunk];  // every edge factor is read before the first store
 #pragma unroll
           for (int i = 0; i < kChunk; ++i) t[i] = sm.t.tab[bb[i]][r];
           // no-return atomics: the stores of one chunk need not wait for each other
 #pragma unroll
-          for (int i = 0; i < kChunk; ++i)
-            atomicAdd(&sm.wacc[g][bb[i]][r], fixed_u(__fmul_rn(e[i], t[i])));
+          for (int k = 0; k < kChunk / 2; ++k) {
+            float f0, f1;
+            f2_unpack(f2_add_rz(f2_mul(ee[k], f2_pack(t[2 * k], t[2 * k + 1])), tz2), f0, f1);
+            atomicAdd(&sm.wacc[g][bb[2 * k]][r], __float_as_uint(f0) - 0x4B000000u);
+            atomicAdd(&sm.wacc[g][bb[2 * k + 1]][r], __float_as_uint(f1) - 0x4B000000u);
+          }
+          // the fixed-order tree e[i] += e[i + w], w = 8, 4, 2, 1, on the pairs
 #pragma unroll
-          for (int w = kChunk / 2; w >= 1; w >>= 1)
+          for (int w = kChunk / 4; w >= 1; w >>= 1)
 #pragma unroll
-            for (int i = 0; i < w; ++i) e[i] = __fadd_rn(e[i], e[i + w]);
-          Zp += (double)e[0];
+            for (int k = 0; k < w; ++k) ee[k] = f2_add(ee[k], ee[k + w]);
+          float z0, z1;
+          f2_unpack(ee[0], z0, z1);
+          Zp += (double)__fadd_rn(z0, z1);
         },
         true, valid);
     sm.zpart[g][r] = Zp;

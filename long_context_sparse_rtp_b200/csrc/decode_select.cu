@@ -657,6 +657,24 @@ __device__ void sort_desc_block(unsigned long long* a, int n) {
 }
 
 // The same, one warp.
+// 32 keys, one per lane, sorted descending across the warp (bitonic, in registers):
+// lane i returns the i-th largest.
+__device__ __forceinline__ unsigned long long sort32_desc(unsigned long long v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, j);
+      const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), j);
+      const unsigned long long o = ((unsigned long long)hi << 32) | lo;
+      // the pair's lower lane keeps the larger key in a descending block
+      const bool desc = (lane & k) == 0, lower = (lane & j) == 0;
+      v = (lower == desc) ? (v > o ? v : o) : (v < o ? v : o);
+    }
+  return v;
+}
+
 __device__ void sort_desc_warp(unsigned long long* a, int n) {
   const int lane = threadIdx.x & 31;
   int n2 = 1;
@@ -1062,6 +1080,9 @@ __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectPara
   ResolveSmem& sm = *reinterpret_cast<ResolveSmem*>(smem_raw);
   const int row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31;
+  // the row's first kThreads candidate slots, loaded with its descriptor (the
+  // slots past the count are read but unused; the row has kDecCap of them)
+  const unsigned long long ck_pre = __ldcg(p.cand + (int64_t)row * kDecCap + tid);
   const RowSel rs = p.rowsel[row];
   RowRes rr;
   if (rs.mode == 1) {
@@ -1124,7 +1145,7 @@ __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectPara
         unsigned long long ck = 0;
         bool in = false;
         if (i < n) {
-          ck = __ldcg(src + i);
+          ck = i0 == 0 ? ck_pre : __ldcg(src + i);
           in = subbin(key_score((uint32_t)(ck >> kIdxBits)), rs.bstar) == ksub;
         }
         const unsigned ball = __ballot_sync(0xffffffffu, in);
@@ -1136,8 +1157,16 @@ __global__ void __launch_bounds__(kThreads) dec_resolve_kernel(const CollectPara
         for (int w2 = 0; w2 < kThreads / 32; ++w2) m += (int)sm.hc[w2];
         __syncthreads();
       }
-      sort_desc_block(sm.wc, m);
-      if (tid < 32) rr = warp_walk(sm.wc, m, r2);
+      if (m <= 32) {  // one warp: a register sort, no block barriers
+        if (tid < 32) {
+          sm.wc[lane] = sort32_desc(lane < m ? sm.wc[lane] : 0ull);
+          __syncwarp();
+          rr = warp_walk(sm.wc, m, r2);
+        }
+      } else {
+        sort_desc_block(sm.wc, m);
+        if (tid < 32) rr = warp_walk(sm.wc, m, r2);
+      }
     } else if (rs.mode == 0 && n > 0 && n <= kWarpCap) {
       for (int i = tid; i < n; i += kThreads) sm.wc[i] = __ldcg(p.cand + (int64_t)row * kDecCap + i);
       __syncthreads();

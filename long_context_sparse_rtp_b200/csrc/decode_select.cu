@@ -598,6 +598,7 @@ struct CollectParams {
 
 struct CollectSmem {
   RowSel rs[16];
+  float lo[16], hi[16];  // the crossing bin's edges bstar / kappa, (bstar + 1) / kappa
   int wsum[kThreads / 32];
 };
 
@@ -1002,7 +1003,7 @@ __device__ RowRes resolve_many(ResolveSmem& sm, const CollectParams& p, int row,
 }
 
 
-__global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectParams p) {
+__global__ void __launch_bounds__(kThreads, 8) dec_collect_kernel(const CollectParams p) {
   griddep_wait();  // launched as a dependent of the previous kernel
   extern __shared__ __align__(16) unsigned char smem_raw[];
   CollectSmem& sm = *reinterpret_cast<CollectSmem*>(smem_raw);
@@ -1011,31 +1012,41 @@ __global__ void __launch_bounds__(kThreads) dec_collect_kernel(const CollectPara
   const int tid = threadIdx.x;
   const int G = p.G;
   const int row0 = b * p.n_ret + rk * G;
-  if (tid < G) sm.rs[tid] = p.rowsel[row0 + tid];
+  if (tid < G) {
+    const RowSel rs = p.rowsel[row0 + tid];
+    sm.rs[tid] = rs;
+    // sbin(s) = floor(kappa s) on exact multiples of 1 / kappa, clamped far outside
+    // the histogram's range: sbin(s) > bstar iff s >= hi, sbin(s) == bstar iff
+    // lo <= s < hi (NaN is neither, as sbin puts it at the bottom)
+    sm.lo[tid] = (float)rs.bstar * (1.0f / kDecKappa);
+    sm.hi[tid] = (float)(rs.bstar + 1) * (1.0f / kDecKappa);
+  }
   __syncthreads();
   const int j0 = chunk * kDecChunk + tid * 4;
+  bool valid[4];  // keys past N are skipped
+#pragma unroll
+  for (int e = 0; e < 4; ++e) valid[e] = j0 + e < p.N;
   uint32_t keep[4] = {0, 0, 0, 0}, cand[4] = {0, 0, 0, 0};
   for (int h = 0; h < G; ++h) {
-    const RowSel& rs = sm.rs[h];
+    const int mode = sm.rs[h].mode;  // the same for every thread of the CTA
     const float4 v =
         *reinterpret_cast<const float4*>(p.scores + (int64_t)(row0 + h) * p.Lk_pad + j0);
     const float vs[4] = {v.x, v.y, v.z, v.w};
+    if (mode != 0) {  // 1: every key kept; 2: settled per key by the attention kernel
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (valid[e]) (mode == 1 ? keep[e] : cand[e]) |= 1u << h;
+      continue;
+    }
+    const float lo = sm.lo[h], hi = sm.hi[h];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
+      if (!valid[e]) continue;
       const int j = j0 + e;
-      if (j >= p.N) continue;
-      if (rs.mode == 1) {
+      if (vs[e] >= hi) {
         keep[e] |= 1u << h;
-        continue;
-      }
-      if (rs.mode == 2) {  // settled per key by the attention kernel
-        cand[e] |= 1u << h;
-        continue;
-      }
-      const int bb = sbin(vs[e]);
-      if (bb > rs.bstar) {
-        keep[e] |= 1u << h;
-      } else if (bb == rs.bstar) {
+      } else if (vs[e] >= lo) {
+        const RowSel& rs = sm.rs[h];
         cand[e] |= 1u << h;
         const uint32_t idx = atomicAdd(&p.ncand[row0 + h], 1u);
         if (idx < (uint32_t)kDecCap)

@@ -27,8 +27,10 @@
 //              global list, and its remaining digits are resolved over the
 //              list, a warp per row, with no further sweep.
 //            A sweep tests each key against the rows' ranges with one compare
-//            (|s - mid| <= half) and queues the hits per warp; the queue is
-//            drained 32 hits at a time.  Range counts are bounds taken from
+//            (|s - mid| <= half) and queues the hits per warp (a chunk in which
+//            no lane has two hits places them by one ballot, others by a prefix
+//            sum); the queue is drained 32 hits at a time.  The list levels
+//            load kListBatch entries per lane before compacting them in place.  Range counts are bounds taken from
 //            the bin sums (every key adds at least a known amount); the count
 //            of keys above the final range is exact.
 //
@@ -80,6 +82,7 @@ enum { ST_IDLE = 0, ST_REFINE1 = 1, ST_REFINE = 2, ST_COLLECT = 3, ST_DONE = 4, 
 // (2^21 + 1) < 2^32 in each copy between flushes.
 constexpr int kListFlush = 4064;
 constexpr int kListCap = 2 * kListFlush;
+constexpr int kListBatch = 4;    // list entries per lane loaded together
 
 struct SelParams {
   unsigned long long* lists;  // [slots][kBM][kListCap] crossing-bin keys, or null
@@ -260,6 +263,18 @@ __device__ __forceinline__ int classify(float s, unsigned long long ck, float m,
 }
 
 enum { MODE_SUB1 = 0, MODE_DIGIT = 1, MODE_COLLECT = 2, MODE_PARK = 3 };
+
+// v[i] for a run-time i in [0, 16): a four-level select tree on the bits of i
+// (registers cannot be indexed at run time).
+__device__ __forceinline__ float pick16(const float (&v)[kChunk], int i) {
+  float a[8], b[4];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a[k] = (i & 1) ? v[2 * k + 1] : v[2 * k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) b[k] = (i & 2) ? a[2 * k + 1] : a[2 * k];
+  const float c0 = (i & 4) ? b[1] : b[0], c1 = (i & 4) ? b[3] : b[2];
+  return (i & 8) ? c1 : c0;
+}
 
 // Processes the first n (<= 32) queued prefilter hits of this warp, one per
 // lane, for the owning row (whose state is fetched from the owner lane):
@@ -770,6 +785,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int i = 0; i < kChunk; ++i)
               hits |= (fabsf(__fsub_rn(v[i], mid)) <= half ? 1u : 0u) << i;
             // -0 -> +0 below: one composite key per score
+            if (!__any_sync(0xffffffffu, (hits & (hits - 1u)) != 0u)) {
+              // at most one hit per lane (the usual case): each hit lane writes
+              // its key at its rank among the hit lanes (qn < 32 here, so the
+              // queue holds them)
+              const uint32_t bal = __ballot_sync(0xffffffffu, hits != 0u);
+              if (hits != 0u) {
+                const int i = __ffs(hits) - 1;
+                const int pos = qn + __popc(bal & ((1u << lane) - 1u));
+                sm.t.q.s[wq][pos] = pick16(v, i) + 0.0f;
+                sm.t.q.jl[wq][pos] = (uint32_t)(j0 + i) | ((uint32_t)lane << 21);
+              }
+              qn += __popc(bal);
+              if (qn >= 32) drain32();
+              return;
+            }
             const int nh = __popc(hits);
             int incl = nh;  // inclusive prefix sum of the lanes' hit counts
 #pragma unroll
@@ -874,33 +904,47 @@ __global__ void __launch_bounds__(kThreads, 2)
             const float rm = ls.m[rr], rtk = ls.tk[rr];
             unsigned long long* const L = lists + (size_t)rr * kListCap;
             int kept = 0, above = 0;
-            for (int k0 = 0; k0 < n; k0 += 32) {
-              if (k0 > 0 && k0 % kListFlush == 0) {  // only this warp adds to row rr
-                __syncwarp();
-                if (lane < kNB) {
-                  sm.u.hw[lane][rr] +=
-                      (unsigned long long)sm.wacc[0][lane][rr] + sm.wacc[1][lane][rr];
-                  sm.wacc[0][lane][rr] = 0u;
-                  sm.wacc[1][lane][rr] = 0u;
+            // kListBatch entries per lane are loaded before any is written back:
+            // the compacted entries land at or below the batch's own positions,
+            // never on an entry still to be loaded
+            for (int kb0 = 0; kb0 < n; kb0 += 32 * kListBatch) {
+              unsigned long long cb[kListBatch];
+#pragma unroll
+              for (int u = 0; u < kListBatch; ++u) {
+                const int k = kb0 + 32 * u + lane;
+                cb[u] = k < n ? __ldcg(L + k) : 0ull;
+              }
+#pragma unroll
+              for (int u = 0; u < kListBatch; ++u) {
+                const int k0 = kb0 + 32 * u;
+                if (k0 >= n) break;
+                if (k0 > 0 && k0 % kListFlush == 0) {  // only this warp adds to row rr
+                  __syncwarp();
+                  if (lane < kNB) {
+                    sm.u.hw[lane][rr] +=
+                        (unsigned long long)sm.wacc[0][lane][rr] + sm.wacc[1][lane][rr];
+                    sm.wacc[0][lane][rr] = 0u;
+                    sm.wacc[1][lane][rr] = 0u;
+                  }
+                  __syncwarp();
                 }
-                __syncwarp();
+                const int k = k0 + lane;
+                const unsigned long long ck = cb[u];
+                const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
+                const bool in = (k < n) & (px == pfx);
+                above += ((k < n) & (px > pfx)) ? 1 : 0;
+                const uint32_t ball = __ballot_sync(0xffffffffu, in);
+                if (in) {
+                  L[kept + __popc(ball & lt)] = ck;
+                  const int digit = (int)((ck >> (kKeyBits - pb - wl)) & ((1ull << wl) - 1));
+                  // even and odd entries in separate copies: <= 2032 keys each
+                  // between flushes
+                  atomicAdd(&sm.wacc[lane & 1][(1 << wl) - 1 - digit][rr],
+                            fixed_u(__fmul_rn(rel_w(key_score((uint32_t)(ck >> kIdxBits)), rm),
+                                              rtk)));
+                }
+                kept += __popc(ball);
               }
-              const int k = k0 + lane;
-              const unsigned long long ck = k < n ? __ldcg(L + k) : 0ull;
-              const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
-              const bool in = (k < n) & (px == pfx);
-              above += ((k < n) & (px > pfx)) ? 1 : 0;
-              const uint32_t ball = __ballot_sync(0xffffffffu, in);
-              if (in) {  // position <= k: never an entry still to be read
-                L[kept + __popc(ball & lt)] = ck;
-                const int digit = (int)((ck >> (kKeyBits - pb - wl)) & ((1ull << wl) - 1));
-                // even and odd entries in separate copies: <= 2032 keys each
-                // between flushes
-                atomicAdd(&sm.wacc[lane & 1][(1 << wl) - 1 - digit][rr],
-                          fixed_u(__fmul_rn(rel_w(key_score((uint32_t)(ck >> kIdxBits)), rm),
-                                            rtk)));
-              }
-              kept += __popc(ball);
             }
             above = __reduce_add_sync(0xffffffffu, above);
             if (lane == 0) {
@@ -937,14 +981,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int pb = ls.pbits[rr], n = ls.n[rr];
           const unsigned long long* const L = lists + (size_t)rr * kListCap;
           int above = 0;
-          for (int k = lane; k < n; k += 32) {
-            const unsigned long long ck = __ldcg(L + k);
-            const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
-            if (px == pfx) {
-              const int slot_c = atomicAdd(&sm.ncnt[rr], 1);
-              if (slot_c < kCap) sm.u.cand[slot_c][rr] = ck;
-            } else if (px > pfx) {
-              ++above;
+          for (int kb0 = 0; kb0 < n; kb0 += 32 * kListBatch) {
+            unsigned long long cb[kListBatch];
+#pragma unroll
+            for (int u = 0; u < kListBatch; ++u) {
+              const int k = kb0 + 32 * u + lane;
+              cb[u] = k < n ? __ldcg(L + k) : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < kListBatch; ++u) {
+              if (kb0 + 32 * u + lane >= n) break;
+              const unsigned long long ck = cb[u];
+              const unsigned long long px = pb > 0 ? (ck >> (kKeyBits - pb)) : 0ull;
+              if (px == pfx) {
+                const int slot_c = atomicAdd(&sm.ncnt[rr], 1);
+                if (slot_c < kCap) sm.u.cand[slot_c][rr] = ck;
+              } else if (px > pfx) {
+                ++above;
+              }
             }
           }
           above = __reduce_add_sync(0xffffffffu, above);

@@ -774,10 +774,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       sweep(
           [&](int j0, float (&v)[kChunk]) {
             bool hit = false;
+            const unsigned long long mid2 = f2_pack(mid, mid);
 #pragma unroll
-            for (int i = 0; i < kChunk; ++i) {
-              hit |= fabsf(__fsub_rn(v[i], mid)) <= half;
-              n_above += v[i] > hic ? 1u : 0u;
+            for (int k = 0; k < kChunk / 2; ++k) {  // v - mid two lanes per instruction
+              float d0, d1;
+              f2_unpack(f2_sub(f2_pack(v[2 * k], v[2 * k + 1]), mid2), d0, d1);
+              hit |= fabsf(d0) <= half;
+              hit |= fabsf(d1) <= half;
+              n_above += v[2 * k] > hic ? 1u : 0u;
+              n_above += v[2 * k + 1] > hic ? 1u : 0u;
             }
             if (__ballot_sync(0xffffffffu, hit) == 0u) return;
             uint32_t hits = 0u;

@@ -535,24 +535,61 @@ __global__ void __launch_bounds__(kThreads, 2)
     };
 
     // ---- sweep 1: the row max m, and a lower bound on Z = sum exp(s - m): each
-    // thread keeps a running max mz and zs, a sum over its 16-key chunks of the
-    // larger of two partial masses, exp(chunk max - mz) and the mass of every
-    // fourth key (both at most the chunk's mass)
+    // thread keeps a running max mz, moved once per tile to the max of its 64
+    // keys there, and zs, a sum over its 16-key chunks of the larger of two
+    // partial masses, exp(chunk max - mz) and the mass of every fourth key (both
+    // at most the chunk's mass).  The tile's 64 scores come with one TMEM wait
+    // and its four chunks are independent.
     float mz = -INFINITY, zs = 0.f;
-    sweep(
-        [&](int, float (&v)[kChunk]) {
-          const float cm = max16(v);
-          if (cm > mz) {  // rescale to the new running max (rare after the first tiles)
-            zs = mz > -INFINITY ? zs * rel_w(mz, cm) : 0.f;
-            mz = cm;
+    for (int kt = 0; kt < n_tiles; ++kt) {
+      const int buf = (int)(tcount & 1u);
+      ok = ok && mbar_wait_warp(&sm.tfull[buf], (tcount >> 1) & 1u, gave_up);
+      tc_fence_after();
+      if (ok) {
+        uint32_t rr[2][32];
+        tmem_ld32_nowait(lane_addr + (uint32_t)(buf * kBN), rr[0]);
+        tmem_ld32_nowait(lane_addr + (uint32_t)(buf * kBN + 32), rr[1]);
+        tmem_wait_ld();
+        float v[4][kChunk];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < kChunk; ++i) {
+            reg_fence(rr[c >> 1][(c & 1) * kChunk + i]);
+            v[c][i] = __uint_as_float(rr[c >> 1][(c & 1) * kChunk + i]);
           }
-          if (mz > -INFINITY) {
-            const float a = __fadd_rn(__fadd_rn(rel_w(v[0], mz), rel_w(v[4], mz)),
-                                      __fadd_rn(rel_w(v[8], mz), rel_w(v[12], mz)));
-            zs = __fadd_rn(zs, fmaxf(a, rel_w(cm, mz)));
+        const int64_t jt0 = (int64_t)kt * kBN + g * 64;
+        if (jt0 + 63 > P) {  // keys past the causal limit read as -inf
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i)
+              if (jt0 + c * kChunk + i > P) v[c][i] = -INFINITY;
+        }
+        float cm[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) cm[c] = max16(v[c]);
+        const float tmx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+        if (tmx > mz) {  // rescale to the new running max (rare after the first tiles)
+          zs = mz > -INFINITY ? zs * rel_w(mz, tmx) : 0.f;
+          mz = tmx;
+        }
+        if (mz > -INFINITY) {
+          float t[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float a = __fadd_rn(__fadd_rn(rel_w(v[c][0], mz), rel_w(v[c][4], mz)),
+                                      __fadd_rn(rel_w(v[c][8], mz), rel_w(v[c][12], mz)));
+            t[c] = fmaxf(a, rel_w(cm[c], mz));
           }
-        },
-        false, false);
+          zs = __fadd_rn(__fadd_rn(zs, __fadd_rn(t[0], t[1])), __fadd_rn(t[2], t[3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tempty[buf]);
+      ++tcount;
+    }
     sm.mpart[g][r] = mz;
     sm.zpart[g][r] = (double)zs;
     ebar();

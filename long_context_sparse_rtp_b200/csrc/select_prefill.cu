@@ -65,6 +65,7 @@ constexpr int kGroup = 16;       // tiles per 32-bit bin-sum group: 16 x 64 keys
 constexpr int kMaxIter = 16;     // refine / collect sweeps (53 key bits / 5 + 1 suffice)
 constexpr int kQueue = 64;       // per-warp queue of refine hits (drained at 32)
 constexpr int kChunk = 16;       // keys per TMEM load and per unrolled body
+constexpr double kRangePad = 1.0 / 16;  // level-0 range beyond the never-kept point
 constexpr int kEpi = 256;        // epilogue threads: two per query row (column halves)
 constexpr int kProdWarp = kEpi / 32, kMmaWarp = kEpi / 32 + 1;
 constexpr int kThreads = kEpi + 64;
@@ -599,15 +600,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       // A key below m - ln(N / ((1 - p) Z)) is never kept: all such keys weigh
       // less than (1 - p) Z together, so the keys above that point already pass
       // p Z.  Z is taken from below (the partial masses, and a 1e-3 margin for
-      // the fp32 sums and ex2.approx), which only widens the range; R adds one
-      // more unit.
+      // the fp32 sums and ex2.approx), which only widens the range; R adds
+      // kRangePad, so the cut lies at least that far above the range's lower
+      // edge, far beyond the rounding of the bin arithmetic there.
       double zl = 0.0;
       for (int h = 0; h < 2; ++h)
         if (sm.mpart[h][r] > -INFINITY) zl += sm.zpart[h][r] * exp((double)(sm.mpart[h][r] - m));
       zl = fmax(zl * (1.0 - 1e-3), 1e-30);
       const double N = (double)(P + 1);
-      const double r_loose = log(N / (1.0 - (double)p.p)) + 1.0;  // Z >= 1
-      const float R = (float)fmin(log(N / ((1.0 - (double)p.p) * zl)) + 1.0, r_loose);
+      const double r_loose = log(N / (1.0 - (double)p.p)) + kRangePad;  // Z >= 1
+      const float R = (float)fmin(log(N / ((1.0 - (double)p.p) * zl)) + kRangePad, r_loose);
       scale = (float)kNB / R;
       margin = 1e-5f * (fabsf(m) + R + 1.f);
     }

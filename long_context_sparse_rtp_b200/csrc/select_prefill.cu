@@ -12,11 +12,12 @@
 // both derive the row's decisions identically from shared memory:
 //
 //   sweep 1  row max m and a lower bound Z_lo on Z = sum exp(s - m) (per 16 keys
-//            the larger of exp(max - m) and the mass of every fourth key)
+//            the larger of exp(max - m) and the mass of every fourth key), 64
+//            scores of a tile per TMEM wait
 //   sweep 2  Z in a fixed order and a 32-bin mass histogram of the scores in
-//            [m - R, m], R = min(ln(N / ((1 - p) Z_lo)), ln(N / (1 - p))) + 1:
-//            keys below m - R + 1 are never kept (together they weigh less than
-//            (1 - p) Z); the crossing bin k0 is where the mass from the top
+//            [m - R, m], R = min(ln(N / ((1 - p) Z_lo)), ln(N / (1 - p))) + 1/16:
+//            keys below m - R + 1/16 are never kept (together they weigh less
+//            than (1 - p) Z); the crossing bin k0 is where the mass from the top
 //            reaches p Z
 //   sweep 3+ per row, until its crossing range holds <= 32 keys, which are
 //            collected, sorted and walked to the exact cut:
@@ -30,9 +31,10 @@
 //            (|s - mid| <= half) and queues the hits per warp (a chunk in which
 //            no lane has two hits places them by one ballot, others by a prefix
 //            sum); the queue is drained 32 hits at a time.  The list levels
-//            load kListBatch entries per lane before compacting them in place.  Range counts are bounds taken from
-//            the bin sums (every key adds at least a known amount); the count
-//            of keys above the final range is exact.
+//            load kListBatch entries per lane before compacting them in place.
+//            Range counts are bounds taken from the bin sums (every key adds at
+//            least a known amount); the count of keys above the final range is
+//            exact.
 //
 // Histogram masses are kept relative to the top edge e of their bin: a key adds
 // trunc(2^21 exp(s - e)) (a value in (exp(-w), 1] x 2^21, w the bin width) to

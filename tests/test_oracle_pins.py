@@ -191,6 +191,34 @@ def test_topp_limits_and_invariants():
             assert abs(r["mass_frac"] - mass / Z) < 1e-12
 
 
+def test_topp_cut_above_the_never_kept_point():
+    """A key below m - ln(N / ((1 - p) Z)) is never kept: the N keys below that
+    point weigh less than (1 - p) Z together, so the keys above it already
+    reach p Z and the shortest prefix stops before them (Eq. 5's minimality).
+    The prefill selection sizes its first histogram range by this bound (Z
+    taken from below, which only widens it).  Rows include heavy and flat
+    score spreads and keys packed just under the bound."""
+    rng = np.random.default_rng(11)
+    for trial in range(120):
+        n = int(rng.integers(2, 3000))
+        s = rng.standard_normal(n) * rng.uniform(0.2, 8)
+        p = float(rng.choice([0.0, 0.5, 0.8, 0.9, 0.95, 0.99]))
+        m = s.max()
+        Z = np.exp(s - m).sum()
+        bound = m - math.log(n / ((1 - p) * Z)) if p < 1 else -math.inf
+        if trial % 4 == 0 and np.isfinite(bound):
+            # half the keys just below the bound: the cut must still stay above
+            lo = rng.random(n) < 0.5
+            lo[int(np.argmax(s))] = False
+            s[lo] = bound - rng.uniform(1e-9, 1e-3, lo.sum())
+            m = s.max()
+            Z = np.exp(s - m).sum()
+            bound = m - math.log(n / ((1 - p) * Z))
+        r = oracle.topp(s, p)
+        assert r["t"] >= bound, (n, p, r["t"], bound)
+        assert not r["sel"][s < bound].any()
+
+
 def test_topp_all_equal_scores():
     for n in (1, 7, 100):
         s = np.zeros(n)
